@@ -1,0 +1,50 @@
+"""CPU oracle for the NF4 grouped mixture-of-experts layer.
+
+TEST INFRASTRUCTURE ONLY.  This package is the plain, slow, obviously
+correct statement of what the GPU library computes.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it.  It shares no code, tables or constants
+with the CUDA library and never imports it; the library never imports this.
+
+Sources (web pages on the method, cited by page title and section):
+
+* "Jordan Anderson" (jordananderson-pages.pages.dev), section
+  "grouped-nf4-gemm & experts-4bit", first bullet: the MoE matmuls run on
+  4-bit packed weights, one launch for all active experts, the codebook
+  decoded inside the GEMM, the bitsandbytes packed layout consumed unchanged;
+  third bullet: the codebook has sixteen entries (NF4).
+* "Jordan Anderson" (jordananderson.work), section "4-bit Mixture-of-Experts
+  fine-tuning on small GPUs", first two bullets: each MoE layer's experts are
+  one fused 3-D parameter, and that fused stack is what gets quantized.
+* The problem statement of this library fixes the rest: blocksize 64, fp32
+  absmax, two codes per byte, top-k softmax routing, SiLU(gate)*up, a
+  routing-weighted combine.
+
+Where the pages are silent the oracle takes one reading, documented at each
+function.  Every function is pinned by tests in ``tests/test_oracle_*.py``
+against closed forms, invariants, brute force and a published table; there
+is no function whose parity is unpinned except the ones that say so.
+
+Precision: decisions that produce integers (NF4 codes, top-k indices) are
+taken in fp32, the precision the kernels use; everything else is fp64.
+"""
+
+from .nf4 import (  # noqa: F401
+    BLOCKSIZE,
+    nf4_levels,
+    nf4_levels_from_quantiles,
+    nf4_midpoints,
+    quantize_blockwise,
+    dequantize_blockwise,
+    unpack_codes,
+)
+from .routing import route_topk, permute_by_expert  # noqa: F401
+from .moe import (  # noqa: F401
+    swiglu,
+    grouped_gemm,
+    unpermute_combine,
+    moe_layer,
+    moe_layer_dense,
+    moe_layer_permuted,
+    ExpertStack,
+)
