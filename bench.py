@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 grouped mixture-of-experts layer on B200.
+
+One step = one pass of the whole hot path -- route + permute, grouped gate_up
+GEMM with fused SwiGLU, grouped down GEMM, combine -- over one token batch,
+through a stack of independent MoE layers whose NF4 weights together exceed
+the 126 MB L2 (every layer's weights stream from HBM once per step).
+
+Default workload: OLMoE-shaped decode (E=64, top-8, hidden 2048, expert
+intermediate 1024, plain softmax weights), T=64 tokens, 16 layers
+(3.6 GB of NF4 weights).  ``--config`` selects the other shapes.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead (bounded samples of the same workload).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import moe_synth  # noqa: E402
+
+CONFIGS = {
+    # name: (shape, T, layers)
+    "olmoe-decode": (moe_synth.OLMOE, 64, 16),
+    "qwen3-30b-decode": (moe_synth.QWEN3_30B, 64, 48),
+    "qwen3-30b-prefill": (moe_synth.QWEN3_30B, 4096, 2),
+    "qwen3-235b-decode": (moe_synth.QWEN3_235B, 32, 8),
+    "qwen3-235b-prefill": (moe_synth.QWEN3_235B, 2048, 1),
+    "tiny": (moe_synth.TINY, 16, 1),
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", choices=sorted(CONFIGS), default="olmoe-decode")
+    p.add_argument("--tokens", type=int, default=None, help="token batch T")
+    p.add_argument("--layers", type=int, default=None)
+    p.add_argument("--algo", choices=["auto", "gemv", "tc"], default="auto")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------- utilities
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- workload
+
+class Workload:
+    def __init__(self, shape, T, layers, seed, device="cuda"):
+        import bit_mixture_experts_route_b200 as moe
+        self.moe = moe
+        self.shape, self.T, self.L = shape, T, layers
+        self.stacks = []
+        for layer in range(layers):
+            s = seed * 1000 + layer
+            w = moe_synth.weights(shape, "gate_up", s, device=device)
+            p_gu, a_gu = moe.nf4_quantize(w)
+            del w
+            w = moe_synth.weights(shape, "down", s, device=device)
+            p_d, a_d = moe.nf4_quantize(w)
+            del w
+            self.stacks.append((p_gu, a_gu, p_d, a_d))
+        torch.cuda.empty_cache()
+        self.X = moe_synth.activations(T, shape.H, seed, device=device)
+        self.logits = torch.stack([moe_synth.logits(shape, T, seed * 1000 + layer, device=device)
+                                   for layer in range(layers)])
+        k, E, H, I = shape.k, shape.E, shape.H, shape.I
+        M = T * k
+        dev = device
+        self.route = {
+            "topk_idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "topk_w": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "expert_offsets": torch.empty((E + 1,), dtype=torch.int32, device=dev),
+            "sorted_rows": torch.empty((M,), dtype=torch.int32, device=dev),
+            "inv_perm": torch.empty((M,), dtype=torch.int32, device=dev),
+        }
+        self.rws = torch.empty((max(moe.route_permute_workspace_size(T, E, k), 256),),
+                               dtype=torch.uint8, device=dev)
+        self.Hbuf = torch.empty((M, I), dtype=torch.float16, device=dev)
+        self.Yp = torch.empty((M, H), dtype=torch.float16, device=dev)
+        self.Y = torch.empty((T, H), dtype=torch.float32, device=dev)
+        self.lws = torch.empty((max(moe.layer_workspace_size(T, E, k, H, I), 256),),
+                               dtype=torch.uint8, device=dev)
+
+    def layer(self, layer, algo="auto", ev=None):
+        moe, sh, T = self.moe, self.shape, self.T
+        p_gu, a_gu, p_d, a_d = self.stacks[layer]
+        r = moe.route_permute(self.logits[layer], sh.k, sh.renormalize, workspace=self.rws,
+                              out=self.route)
+        M = T * sh.k
+        if ev is not None:
+            ev[0].record()
+        moe.nf4_grouped_gemm(self.X, p_gu, a_gu, r["expert_offsets"], M,
+                             gather=r["sorted_rows"], k=sh.k, epilogue="swiglu",
+                             out=self.Hbuf, algo=algo)
+        if ev is not None:
+            ev[1].record()
+        moe.nf4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
+                             out=self.Yp, algo=algo)
+        moe.unpermute_combine(self.Yp, r["inv_perm"], r["topk_w"], out=self.Y)
+
+    def step(self, algo="auto", evs=None):
+        for layer in range(self.L):
+            self.layer(layer, algo, None if evs is None else evs[layer])
+
+    # Algorithmic work ----------------------------------------------------
+    def distinct_experts(self):
+        """Experts with >= 1 routed row, per layer (from expert_offsets)."""
+        out = []
+        for layer in range(self.L):
+            r = self.moe.route_permute(self.logits[layer], self.shape.k, self.shape.renormalize)
+            off = r["expert_offsets"].cpu().numpy()
+            out.append(int(np.count_nonzero(np.diff(off))))
+        return out
+
+    def gate_up_bytes(self, d):
+        sh, T = self.shape, self.T
+        w = d * (2 * sh.I * sh.H) * 0.5625
+        return w + T * sh.H * 2 + T * sh.k * sh.I * 2
+
+    def layer_bytes(self, d):
+        sh, T = self.shape, self.T
+        return d * 3 * sh.H * sh.I * 0.5625 + T * sh.H * 2 + T * sh.E * 4 + T * sh.H * 4
+
+    def gate_up_flops(self):
+        sh = self.shape
+        return 2.0 * self.T * sh.k * sh.H * 2 * sh.I
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(shape, T, seed, n_tokens, start_token=0, threads=None):
+    """Time the oracle on ``n_tokens`` tokens of layer 0: dequantize the NF4
+    experts they need and run the per-token expert MLPs.  Weights come from
+    the same generator as the GPU run; quantization is untimed setup."""
+    import oracle
+    s = seed * 1000
+    X = moe_synth.activations(T, shape.H, seed).float().numpy()
+    lg = moe_synth.logits(shape, T, s).numpy()
+    idx, _ = oracle.route_topk(lg, shape.k, shape.renormalize)
+    toks = [(start_token + i) % T for i in range(n_tokens)]
+    experts = sorted({int(e) for t in toks for e in idx[t]})
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w_gu = moe_synth.weights(shape, "gate_up", s, experts=experts, device=dev).cpu().numpy()
+    w_d = moe_synth.weights(shape, "down", s, experts=experts, device=dev).cpu().numpy()
+    E, I, H = shape.E, shape.I, shape.H
+    p_gu = np.zeros((E, 2 * I, H // 2), np.uint8)
+    a_gu = np.zeros((E, 2 * I * H // 64), np.float32)
+    p_d = np.zeros((E, H, I // 2), np.uint8)
+    a_d = np.zeros((E, H * I // 64), np.float32)
+    for i, e in enumerate(experts):
+        p, a = oracle.quantize_blockwise(w_gu[i])
+        p_gu[e], a_gu[e] = p, a.reshape(-1)
+        p, a = oracle.quantize_blockwise(w_d[i])
+        p_d[e], a_d[e] = p, a.reshape(-1)
+    stack = oracle.ExpertStack(p_gu, a_gu, p_d, a_d)
+    t0 = time.perf_counter()
+    oracle.moe_layer(X, lg, stack, shape.k, shape.renormalize, tokens=toks)
+    dt = time.perf_counter() - t0
+    return n_tokens, dt
+
+
+def cpu_cores():
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except AttributeError:
+        aff = os.cpu_count()
+    threads = aff
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            threads = max(int(d.get("num_threads", 1)) for d in info)
+    except Exception:
+        pass
+    return os.cpu_count(), aff, threads
+
+
+def run_reference(args, shape, T, layers):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    n_tok = 2
+    for _ in range(args.warmup):
+        oracle_sample(shape, T, args.seed, n_tok)
+    total_tok, total_t, start = 0, 0.0, 0
+    for _ in range(args.steps):
+        n, dt = oracle_sample(shape, T, args.seed, n_tok, start_token=start)
+        total_tok += n
+        total_t += dt
+        start += n_tok
+    value = total_tok / total_t
+    ncpu, aff, threads = cpu_cores()
+    line = {
+        "impl": "reference", "metric": "MoE layer tokens/s", "value": value,
+        "unit": "tokens/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.config, "T": T, "layers": layers, "E": shape.E,
+                   "k": shape.k, "hidden": shape.H, "intermediate": shape.I},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n_tok} tokens of layer 0 per step, experts dequantized "
+                                   f"afresh each step; host cpu_count={ncpu}, affinity={aff}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    args = parse_args()
+    shape, T, layers = CONFIGS[args.config]
+    T = args.tokens or T
+    layers = args.layers or layers
+    if args.impl == "reference":
+        run_reference(args, shape, T, layers)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    world, rank, local = dist_setup()
+    import bit_mixture_experts_route_b200 as moe
+    moe.load()
+    wl = Workload(shape, T, layers, args.seed + rank)
+    hbm, tf_burst, tf_sust, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- warm-up
+    for _ in range(max(args.warmup, 3)):
+        wl.step(args.algo)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events around every gate_up launch
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in range(layers)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for s in range(args.steps):
+            wl.step(args.algo, evs[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_step = T * layers          # layer-tokens: T tokens through each layer
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    gu_ms = [e[0].elapsed_time(e[1]) for st in evs for e in st]
+    gu_avg_ms = sum(gu_ms) / len(gu_ms)
+
+    d = wl.distinct_experts()
+    d_avg = sum(d) / len(d)
+    gu_bytes = sum(wl.gate_up_bytes(x) for x in d) / len(d)
+    gu_flops = wl.gate_up_flops()
+    prefill = T * shape.k >= 16 * shape.E
+    if prefill:
+        achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
+        peak = tf_burst
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "grouped NF4 gate_up GEMM + SwiGLU",
+                "per_launch": f"{gu_flops:.4g} FLOP (2*T*k*H*2I)",
+                "peak_source": f"{peak_kind} bf16 dense"}
+    else:
+        achieved = gu_bytes / (gu_avg_ms / 1e3) / 1e9
+        peak = hbm
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "grouped NF4 gate_up GEMV + SwiGLU",
+                "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*0.5625 "
+                              f"+ X + Hbuf)",
+                "peak_source": f"{peak_kind} HBM copy"}
+
+    # ---- graphed variant of the same step (CUDA graph of all launches)
+    graphed = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            wl.step(args.algo)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            wl.step(args.algo)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        gs.record()
+        for _ in range(args.steps):
+            g.replay()
+        ge.record()
+        torch.cuda.synchronize()
+        gms = max_over_ranks(gs.elapsed_time(ge), world)
+        graphed = {"value": world * tokens_per_step * args.steps / (gms / 1e3),
+                   "ms_per_step": gms / args.steps}
+        del g
+    except Exception as exc:  # noqa: BLE001
+        graphed = {"error": str(exc)[:200]}
+
+    # ---- end to end through the one-call C API with host buffers
+    X_h = wl.X.cpu().pin_memory()
+    L_h = wl.logits.cpu().pin_memory()
+    Y_h = torch.empty((T, shape.H), dtype=torch.float32).pin_memory()
+    X_d, L_d = torch.empty_like(wl.X), torch.empty_like(wl.logits)
+
+    def e2e_step():
+        X_d.copy_(X_h, non_blocking=True)
+        L_d.copy_(L_h, non_blocking=True)
+        for layer in range(layers):
+            moe.layer_forward(X_d, L_d[layer], shape.k, shape.renormalize, *wl.stacks[layer],
+                              workspace=wl.lws, out=wl.Y)
+        Y_h.copy_(wl.Y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    es.record()
+    for _ in range(args.steps):
+        e2e_step()
+    ee.record()
+    torch.cuda.synchronize()
+    ems = max_over_ranks(es.elapsed_time(ee), world)
+    e2e = {"value": world * tokens_per_step * args.steps / (ems / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": X_h.numel() * 2 + L_h.numel() * 4,
+           "d2h_bytes_per_step": Y_h.numel() * 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ncpu, aff, threads = cpu_cores()
+        n_tok = 16 if not prefill else 4
+        n, dt = oracle_sample(shape, T, args.seed, n_tok)
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} tokens of layer 0 of this workload (NF4 experts dequantized, "
+                         f"per-token fp64 expert MLPs); host cpu_count={ncpu}, "
+                         f"affinity={aff}; {dt:.1f} s"}
+
+    launches_per_layer = 5  # route_tile, permute_scatter, gate_up, down, combine
+    line = {
+        "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": args.config, "T": T, "layers": layers, "E": shape.E,
+                   "k": shape.k, "hidden": shape.H, "intermediate": shape.I,
+                   "renormalize": shape.renormalize, "routing": shape.routing,
+                   "value_counts": "layer-tokens: T tokens through each of the layers",
+                   "l2": f"inputs larger than L2: {layers} layers x "
+                         f"{shape.E * shape.nf4_bytes_per_expert / 1e6:.0f} MB NF4 weights",
+                   "distinct_experts_per_layer": d_avg, "algo": args.algo,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "graphed": graphed,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_layer * layers * args.steps,
+        "clocks": clk.summary(),
+        "gate_up_ms_avg": gu_avg_ms,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

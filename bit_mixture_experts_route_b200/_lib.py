@@ -1,0 +1,229 @@
+"""ctypes binding of libmoenf4.so: argument marshalling only.
+
+Every function here takes torch CUDA tensors, checks dtype / shape /
+contiguity, allocates outputs with torch when the caller does not pass them,
+and calls the C entry point of the same name on the current CUDA stream.
+All arithmetic runs in the library's kernels; there is no fallback.  If the
+shared library is missing, importing any op raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoenf4.so")
+
+MOE_OK = 0
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED",
+          3: "MOE_ERR_UNSUPPORTED", 4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA"}
+DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+EPI = {"none": 0, "swiglu": 1}
+ALGO = {"auto": 0, "gemv": 1, "tc": 2}
+DEVERR_NONFINITE, DEVERR_BAD_OFFSETS, DEVERR_BAD_INDEX, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+# Every exported symbol with (restype, argtypes); the header declares them.
+_P, _I, _Z, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+SIGNATURES = {
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_abi_version": (_I, []),
+    "moe_nf4_levels": (_I, [_P]),
+    "moe_nf4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _S]),
+    "moe_nf4_dequantize": (_I, [_P, _P, _I, _I, _I, _P, _I, _S]),
+    "moe_route_permute_workspace_size": (_I, [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_route_permute": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _S]),
+    "moe_nf4_grouped_gemm": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P,
+                                  _I, _I, _P, _S]),
+    "moe_swiglu": (_I, [_P, _I, _I, _I, _P, _I, _S]),
+    "moe_unpermute_combine": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _S]),
+    "moe_layer_workspace_size": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_layer_forward": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
+                               _P, _S]),
+}
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+def load() -> ctypes.CDLL:
+    """Load libmoenf4.so (once) and bind every exported signature."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise MoEError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m bit_mixture_experts_route_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(f"{what}: {STATUS.get(status, status)}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise MoEError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise MoEError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise MoEError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise MoEError(f"{name} must have {ndim} dims")
+
+
+def nf4_levels():
+    buf = (ctypes.c_float * 16)()
+    _check(load().moe_nf4_levels(ctypes.cast(buf, ctypes.c_void_p)), "moe_nf4_levels")
+    return list(buf)
+
+
+def nf4_quantize(W, packed=None, absmax=None, dev_err=None):
+    """``W fp32 [E, N, K]`` -> ``(packed u8 [E, N, K/2], absmax fp32 [E, N*K/64])``."""
+    _need(W, torch.float32, "W", 3)
+    E, N, K = W.shape
+    if packed is None:
+        packed = torch.empty((E, N, K // 2), dtype=torch.uint8, device=W.device)
+    if absmax is None:
+        absmax = torch.empty((E, N * K // 64), dtype=torch.float32, device=W.device)
+    _check(load().moe_nf4_quantize(_ptr(W), E, N, K, 64, _ptr(packed), _ptr(absmax),
+                                   _ptr(dev_err), _stream(W.device)), "moe_nf4_quantize")
+    return packed, absmax
+
+
+def nf4_dequantize(packed, absmax, out_dtype=torch.float32):
+    _need(packed, torch.uint8, "packed", 3)
+    E, N, half = packed.shape
+    out = torch.empty((E, N, 2 * half), dtype=out_dtype, device=packed.device)
+    _check(load().moe_nf4_dequantize(_ptr(packed), _ptr(absmax), E, N, 2 * half, _ptr(out),
+                                     DT[out_dtype], _stream(packed.device)),
+           "moe_nf4_dequantize")
+    return out
+
+
+def route_permute_workspace_size(T, E, k):
+    n = ctypes.c_size_t()
+    _check(load().moe_route_permute_workspace_size(T, E, k, ctypes.byref(n)),
+           "moe_route_permute_workspace_size")
+    return n.value
+
+
+def route_permute(logits, k, renormalize=True, workspace=None, out=None):
+    """``logits fp32 [T, E]`` -> dict of topk_idx, topk_w, expert_offsets,
+    sorted_rows, inv_perm (device tensors)."""
+    _need(logits, torch.float32, "logits", 2)
+    T, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = {
+            "topk_idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "topk_w": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "expert_offsets": torch.empty((E + 1,), dtype=torch.int32, device=dev),
+            "sorted_rows": torch.empty((T * k,), dtype=torch.int32, device=dev),
+            "inv_perm": torch.empty((T * k,), dtype=torch.int32, device=dev),
+        }
+    nbytes = route_permute_workspace_size(T, E, k)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=dev)
+    _check(load().moe_route_permute(
+        _ptr(logits), T, E, k, 1 if renormalize else 0, _ptr(out["topk_idx"]),
+        _ptr(out["topk_w"]), _ptr(out["expert_offsets"]), _ptr(out["sorted_rows"]),
+        _ptr(out["inv_perm"]), _ptr(workspace), workspace.numel(), _stream(dev)),
+        "moe_route_permute")
+    return out
+
+
+def nf4_grouped_gemm(A, packed, absmax, expert_offsets, M_total, gather=None, k=1,
+                     epilogue="none", out_dtype=torch.float32, algo="auto", out=None,
+                     dev_err=None):
+    """Grouped NF4 GEMM over all experts in one launch (see the header)."""
+    if A.dtype not in (torch.bfloat16, torch.float16):
+        raise MoEError("A must be bf16 or fp16")
+    _need(A, A.dtype, "A", 2)
+    _need(packed, torch.uint8, "packed", 3)
+    _need(absmax, torch.float32, "absmax")
+    _need(expert_offsets, torch.int32, "expert_offsets", 1)
+    E, N, half = packed.shape
+    K = 2 * half
+    if A.shape[1] != K:
+        raise MoEError("A's columns must equal the weights' K")
+    if gather is not None:
+        _need(gather, torch.int32, "gather", 1)
+    n_out = N // 2 if epilogue == "swiglu" else N
+    if out is None:
+        out = torch.empty((M_total, n_out), dtype=out_dtype, device=A.device)
+    _check(load().moe_nf4_grouped_gemm(
+        _ptr(A), DT[A.dtype], A.shape[0], _ptr(gather), k, _ptr(packed), _ptr(absmax),
+        _ptr(expert_offsets), E, N, K, M_total, EPI[epilogue], _ptr(out), DT[out.dtype],
+        ALGO[algo], _ptr(dev_err), _stream(A.device)), "moe_nf4_grouped_gemm")
+    return out
+
+
+def swiglu(gu, h_dtype=torch.float32, out=None):
+    _need(gu, gu.dtype, "gu", 2)
+    M, two_i = gu.shape
+    if out is None:
+        out = torch.empty((M, two_i // 2), dtype=h_dtype, device=gu.device)
+    _check(load().moe_swiglu(_ptr(gu), DT[gu.dtype], M, two_i // 2, _ptr(out), DT[out.dtype],
+                             _stream(gu.device)), "moe_swiglu")
+    return out
+
+
+def unpermute_combine(Yp, inv_perm, topk_w, y_dtype=torch.float32, out=None):
+    _need(Yp, Yp.dtype, "Yp", 2)
+    _need(inv_perm, torch.int32, "inv_perm")
+    _need(topk_w, torch.float32, "topk_w", 2)
+    T, k = topk_w.shape
+    H = Yp.shape[1]
+    if out is None:
+        out = torch.empty((T, H), dtype=y_dtype, device=Yp.device)
+    _check(load().moe_unpermute_combine(_ptr(Yp), DT[Yp.dtype], _ptr(inv_perm), _ptr(topk_w),
+                                        T, k, H, _ptr(out), DT[out.dtype], _stream(Yp.device)),
+           "moe_unpermute_combine")
+    return out
+
+
+def layer_workspace_size(T, E, k, H, I):
+    n = ctypes.c_size_t()
+    _check(load().moe_layer_workspace_size(T, E, k, H, I, ctypes.byref(n)),
+           "moe_layer_workspace_size")
+    return n.value
+
+
+def layer_forward(X, logits, k, renormalize, packed_gu, absmax_gu, packed_d, absmax_d,
+                  workspace=None, out=None, dev_err=None):
+    """The whole layer through one C call: ``Y fp32 [T, H]``."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(logits, torch.float32, "logits", 2)
+    T, H = X.shape
+    E = logits.shape[1]
+    I = packed_d.shape[2] * 2
+    nbytes = layer_workspace_size(T, E, k, H, I)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=X.device)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=X.device)
+    _check(load().moe_layer_forward(
+        _ptr(X), _ptr(logits), T, E, k, 1 if renormalize else 0, H, I, _ptr(packed_gu),
+        _ptr(absmax_gu), _ptr(packed_d), _ptr(absmax_d), _ptr(out), _ptr(workspace),
+        workspace.numel(), _ptr(dev_err), _stream(X.device)), "moe_layer_forward")
+    return out

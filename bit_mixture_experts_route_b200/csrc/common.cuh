@@ -1,0 +1,134 @@
+// Shared device helpers of the NF4 MoE library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_nf4.h"
+
+namespace moe {
+
+constexpr int kBlock = 64;  // NF4 block size along K
+
+// The sixteen NF4 levels (fp32, ascending), as published with QLoRA's
+// NormalFloat data type and shipped in the bitsandbytes layout the pages'
+// kernel consumes unchanged ("grouped-nf4-gemm & experts-4bit", first and
+// third bullets).  Code 7 is exactly 0; codes 0 and 15 are exactly -1, +1.
+#define MOE_NF4_LEVEL_LIST                                                   \
+  -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f, \
+      -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f,  \
+      0.0f, 0.07958029955625534f, 0.16093020141124725f,                     \
+      0.24611230194568634f, 0.33791524171829224f, 0.44070982933044434f,     \
+      0.5626170039176941f, 0.7229568362236023f, 1.0f
+
+__device__ __forceinline__ void set_dev_err(int32_t* dev_err, int bits) {
+  if (dev_err) atomicOr(reinterpret_cast<int*>(dev_err), bits);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Loads that bypass L1 allocation for streamed-once data (weights).
+__device__ __forceinline__ uint2 ldg_stream_u2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint4 ldg_stream_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Two bf16 (packed in a u32, element 0 in the low half) -> two fp16.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  float lo = __uint_as_float(v << 16);
+  float hi = __uint_as_float(v & 0xffff0000u);
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// silu(g) * u with silu(g) = g / (1 + exp(-g)), IEEE division.
+__device__ __forceinline__ float swiglu_f32(float g, float u) {
+  return __fdiv_rn(g, 1.0f + expf(-g)) * u;
+}
+
+}  // namespace moe
+
+// Host-side launchers implemented in the kernel files, called by api.cu.
+namespace moe_launch {
+cudaError_t nf4_quantize(const float* W, int64_t rows, int K, uint8_t* packed,
+                         float* absmax, int32_t* dev_err, cudaStream_t s);
+cudaError_t nf4_dequantize(const uint8_t* packed, const float* absmax,
+                           int64_t rows, int K, void* out, moe_dtype_t dt,
+                           cudaStream_t s);
+size_t route_workspace_bytes(int T, int E, int k);
+cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
+                          int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                          int32_t* sorted_rows, int32_t* inv_perm, void* ws,
+                          cudaStream_t s);
+cudaError_t grouped_gemm_gemv(const void* A, moe_dtype_t a_dt, int A_rows,
+                              const int32_t* gather, int k,
+                              const uint8_t* packed, const float* absmax,
+                              const int32_t* offsets, int E, int N, int K,
+                              int M_total, moe_epilogue_t epi, void* out,
+                              moe_dtype_t out_dt, int32_t* dev_err,
+                              cudaStream_t s);
+cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows,
+                            const int32_t* gather, int k,
+                            const uint8_t* packed, const float* absmax,
+                            const int32_t* offsets, int E, int N, int K,
+                            int M_total, moe_epilogue_t epi, void* out,
+                            moe_dtype_t out_dt, int32_t* dev_err,
+                            cudaStream_t s);
+bool grouped_gemm_tc_supported(int N, int K, moe_epilogue_t epi);
+cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h,
+                   moe_dtype_t h_dt, cudaStream_t s);
+cudaError_t unpermute_combine(const void* Yp, moe_dtype_t yp_dt,
+                              const int32_t* inv_perm, const float* topk_w,
+                              int T, int k, int H, void* Y, moe_dtype_t y_dt,
+                              cudaStream_t s);
+}  // namespace moe_launch

@@ -1,0 +1,137 @@
+// Standalone SwiGLU and the routing-weighted unpermute/combine.
+//
+// Both are HBM-bound streaming kernels with 16-byte vector accesses.
+//   swiglu:  h[m, i] = silu(gu[m, i]) * gu[m, I + i]
+//   combine: Y[t, :] = sum_{j<k} w[t, j] * Yp[inv_perm[t*k + j], :], summed in
+//            j order in fp32 (deterministic).
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+template <typename T>
+struct Vec4 {
+  T v[4];
+};
+
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&f)[4]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = to_f32<T>(h[i]);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store4(T* p, const float (&f)[4]) {
+  if constexpr (sizeof(T) == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  } else {
+    Vec4<T> o;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o.v[i] = from_f32<T>(f[i]);
+    *reinterpret_cast<Vec4<T>*>(p) = o;
+  }
+}
+
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(256) swiglu_kernel(const InT* __restrict__ gu, int M, int I,
+                                                     OutT* __restrict__ h) {
+  const int64_t per_row = I / 4;
+  const int64_t total = (int64_t)M * per_row;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += stride) {
+    const int64_t m = q / per_row, c = (q % per_row) * 4;
+    float g[4], u[4], o[4];
+    load4(gu + m * 2 * I + c, g);
+    load4(gu + m * 2 * I + I + c, u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = swiglu_f32(g[i], u[i]);
+    store4(h + m * I + c, o);
+  }
+}
+
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(256) combine_kernel(const InT* __restrict__ Yp,
+                                                      const int32_t* __restrict__ inv_perm,
+                                                      const float* __restrict__ w, int T,
+                                                      int k, int H, OutT* __restrict__ Y) {
+  // One CTA-row of threads per token; each thread owns 4 consecutive columns.
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  const int total = T * k;
+  for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4; c < H; c += gridDim.y * blockDim.x * 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int p = inv_perm[(size_t)t * k + j];
+      if (p < 0 || p >= total) continue;
+      const float wj = w[(size_t)t * k + j];
+      float y[4];
+      load4(Yp + (size_t)p * H + c, y);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj, y[i], acc[i]);
+    }
+    store4(Y + (size_t)t * H + c, acc);
+  }
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <typename InT>
+cudaError_t swiglu_out(const InT* gu, int M, int I, void* h, moe_dtype_t h_dt, cudaStream_t s) {
+  const int64_t total = (int64_t)M * (I / 4);
+  int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
+  if (grid < 1) grid = 1;
+  if (h_dt == MOE_DT_F32) swiglu_kernel<<<grid, 256, 0, s>>>(gu, M, I, (float*)h);
+  else if (h_dt == MOE_DT_F16) swiglu_kernel<<<grid, 256, 0, s>>>(gu, M, I, (__half*)h);
+  else swiglu_kernel<<<grid, 256, 0, s>>>(gu, M, I, (__nv_bfloat16*)h);
+  return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t combine_out(const InT* Yp, const int32_t* inv_perm, const float* w, int T, int k,
+                        int H, void* Y, moe_dtype_t y_dt, cudaStream_t s) {
+  const int threads = 256;
+  const int ychunks = std::max(1, std::min((H / 4 + threads - 1) / threads, 8));
+  const dim3 grid(T, ychunks);
+  if (y_dt == MOE_DT_F32) combine_kernel<<<grid, threads, 0, s>>>(Yp, inv_perm, w, T, k, H, (float*)Y);
+  else if (y_dt == MOE_DT_F16) combine_kernel<<<grid, threads, 0, s>>>(Yp, inv_perm, w, T, k, H, (__half*)Y);
+  else combine_kernel<<<grid, threads, 0, s>>>(Yp, inv_perm, w, T, k, H, (__nv_bfloat16*)Y);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace moe
+
+namespace moe_launch {
+
+cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h, moe_dtype_t h_dt,
+                   cudaStream_t s) {
+  if (M == 0) return cudaSuccess;
+  if (gu_dt == MOE_DT_F32) return moe::swiglu_out((const float*)gu, M, I, h, h_dt, s);
+  if (gu_dt == MOE_DT_F16) return moe::swiglu_out((const __half*)gu, M, I, h, h_dt, s);
+  return moe::swiglu_out((const __nv_bfloat16*)gu, M, I, h, h_dt, s);
+}
+
+cudaError_t unpermute_combine(const void* Yp, moe_dtype_t yp_dt, const int32_t* inv_perm,
+                              const float* topk_w, int T, int k, int H, void* Y,
+                              moe_dtype_t y_dt, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (yp_dt == MOE_DT_F32)
+    return moe::combine_out((const float*)Yp, inv_perm, topk_w, T, k, H, Y, y_dt, s);
+  if (yp_dt == MOE_DT_F16)
+    return moe::combine_out((const __half*)Yp, inv_perm, topk_w, T, k, H, Y, y_dt, s);
+  return moe::combine_out((const __nv_bfloat16*)Yp, inv_perm, topk_w, T, k, H, Y, y_dt, s);
+}
+
+}  // namespace moe_launch

@@ -1,0 +1,247 @@
+// Top-k softmax routing and the stable token->expert permutation.
+//
+// The router of "grouped-nf4-gemm & experts-4bit" (jordananderson-pages
+// .pages.dev, second bullet) feeds a kernel that covers all active experts
+// in one launch (first bullet); that launch reads each expert's routed rows
+// as one contiguous segment, which this file builds:
+//   expert_offsets[E+1]  segment starts (exclusive scan of per-expert counts)
+//   sorted_rows[T*k]     flat ids t*k+j ordered by expert, then by flat id
+//   inv_perm[T*k]        position of each flat id
+//
+// Two launches, both deterministic (no atomics whose order matters):
+//  1. route_tile_kernel, one CTA per tile of 64 tokens: one warp per token
+//     selects the top-k with 64-bit keys (ordered logit, ~expert) so ties go
+//     to the lower expert and every lane agrees even on NaN, computes the
+//     softmax weights, then warp 0 ranks the tile's routed rows stably with
+//     __match_any_sync and writes the tile's per-expert counts.
+//  2. permute_scatter_kernel, one CTA per tile: sums the tile counts into
+//     expert totals and the tile's prefix, scans the totals into offsets and
+//     scatters each flat id to offsets[e] + prefix + rank.
+#include <climits>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTileTok = 64;  // tokens per routing tile / CTA
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint32_t ordered_bits(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);  // -0 -> +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unordered_bits(uint32_t o) {
+  const uint32_t u = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
+  return __uint_as_float(u);
+}
+
+template <int NPER>
+__global__ void __launch_bounds__(kThreads) route_tile_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int renorm,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int32_t* __restrict__ rank, int32_t* __restrict__ tile_counts) {
+  __shared__ int s_eid[kTileTok * 32];
+  __shared__ int s_cnt[1024];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tile = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += kThreads) s_cnt[e] = 0;
+
+  for (int tt = warp; tt < kTileTok; tt += kThreads / 32) {
+    const int t = tile * kTileTok + tt;
+    if (t >= T) break;
+    const float* row = logits + (size_t)t * E;
+    uint64_t key[NPER];
+#pragma unroll
+    for (int i = 0; i < NPER; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = (e < E) ? ((uint64_t)ordered_bits(row[e]) << 32) | (uint32_t)(~e) : 0ull;
+    }
+    uint32_t taken = 0;
+    uint64_t mine = 0;  // lane j keeps the j-th selected key
+    uint64_t first = 0;
+    for (int j = 0; j < k; ++j) {
+      uint64_t best = 0;
+#pragma unroll
+      for (int i = 0; i < NPER; ++i)
+        if (!((taken >> i) & 1u) && key[i] > best) best = key[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+        best = other > best ? other : best;
+      }
+      const int e = (int)(~(uint32_t)best);
+      if (e >= 0 && e < E && (e & 31) == lane) taken |= 1u << (e >> 5);
+      if (j == lane) mine = best;
+      if (j == 0) first = best;
+    }
+    // softmax: max logit = first selected
+    const float mx = unordered_bits((uint32_t)(first >> 32));
+    float ex = 0.0f;
+    if (lane < k) ex = expf(unordered_bits((uint32_t)(mine >> 32)) - mx);
+    float denom;
+    if (renorm) {
+      denom = warp_sum(ex);
+    } else {
+      float part = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NPER; ++i)
+        if (lane + 32 * i < E) part += expf(unordered_bits((uint32_t)(key[i] >> 32)) - mx);
+      denom = warp_sum(part);
+    }
+    if (lane < k) {
+      const int e = (int)(~(uint32_t)mine);
+      topk_idx[(size_t)t * k + lane] = e;
+      topk_w[(size_t)t * k + lane] = __fdiv_rn(ex, denom);
+      s_eid[tt * k + lane] = e;
+    }
+  }
+  __syncthreads();
+
+  // Stable rank of every routed row of the tile within its expert: one warp
+  // walks the tile in flat order, 32 rows at a time.
+  const int ntok = min(kTileTok, T - tile * kTileTok);
+  const int n = ntok * k;
+  const size_t fbase = (size_t)tile * kTileTok * k;
+  if (warp == 0) {
+    for (int base = 0; base < n; base += 32) {
+      const int f = base + lane;
+      int e = (f < n) ? s_eid[f] : -1;
+      const bool valid = (e >= 0 && e < E);
+      const int keyv = valid ? e : (1 << 20) + lane;  // unique for invalid lanes
+      const unsigned peers = __match_any_sync(0xffffffffu, keyv);
+      const int r = __popc(peers & lanemask_lt());
+      const int c0 = valid ? s_cnt[e] : 0;
+      __syncwarp();
+      if (valid && (peers >> lane) == 1u) s_cnt[e] = c0 + __popc(peers);  // last lane of group
+      __syncwarp();
+      if (f < n) rank[fbase + f] = valid ? c0 + r : -1;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kThreads) tile_counts[(size_t)tile * E + e] = s_cnt[e];
+}
+
+// Exclusive scan of s[0..n) in place for n <= 1024 with kThreads threads.
+__device__ void block_exclusive_scan(int* s, int n, int* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kPer = 1024 / kThreads;  // 4 elements per thread
+  int v[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int idx = threadIdx.x * kPer + i;
+    v[i] = idx < n ? s[idx] : 0;
+    sum += v[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kThreads / 32 ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kThreads / 32) s_warp[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  int run = incl - sum + (warp ? s_warp[warp - 1] : 0);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int idx = threadIdx.x * kPer + i;
+    if (idx < n) s[idx] = run;
+    run += v[i];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kThreads) permute_scatter_kernel(
+    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ rank,
+    const int32_t* __restrict__ tile_counts, int T, int E, int k, int ntiles,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
+    int32_t* __restrict__ inv_perm) {
+  __shared__ int s_off[1024];
+  __shared__ int s_before[1024];
+  __shared__ int s_warp[kThreads / 32];
+  const int tile = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    int tot = 0, before = 0;
+    for (int b = 0; b < ntiles; ++b) {
+      const int c = tile_counts[(size_t)b * E + e];
+      before += (b < tile) ? c : 0;
+      tot += c;
+    }
+    s_off[e] = tot;
+    s_before[e] = before;
+  }
+  __syncthreads();
+  block_exclusive_scan(s_off, E, s_warp);
+  if (tile == 0) {
+    for (int e = threadIdx.x; e < E; e += kThreads) offsets[e] = s_off[e];
+    if (threadIdx.x == 0) offsets[E] = T * k;
+  }
+  for (int e = threadIdx.x; e < E; e += kThreads) s_before[e] += s_off[e];
+  __syncthreads();
+  const int ntok = min(kTileTok, T - tile * kTileTok);
+  const int n = ntok * k;
+  const size_t fbase = (size_t)tile * kTileTok * k;
+  const int total = T * k;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const size_t f = fbase + i;
+    const int e = topk_idx[f];
+    const int r = rank[f];
+    if (e < 0 || e >= E || r < 0) continue;
+    const int pos = s_before[e] + r;
+    if (pos < 0 || pos >= total) continue;
+    sorted_rows[pos] = (int32_t)f;
+    inv_perm[f] = pos;
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+namespace moe_launch {
+
+static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+size_t route_workspace_bytes(int T, int E, int k) {
+  const size_t ntiles = (T + moe::kTileTok - 1) / moe::kTileTok;
+  return align256((size_t)T * k * 4) + align256(ntiles * E * 4);
+}
+
+cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
+                          int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                          int32_t* sorted_rows, int32_t* inv_perm, void* ws,
+                          cudaStream_t s) {
+  if (T == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
+  const int ntiles = (T + moe::kTileTok - 1) / moe::kTileTok;
+  int32_t* rank = reinterpret_cast<int32_t*>(ws);
+  int32_t* tile_counts =
+      reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + align256((size_t)T * k * 4));
+#define MOE_ROUTE_LAUNCH(NP)                                                          \
+  moe::route_tile_kernel<NP><<<ntiles, moe::kThreads, 0, s>>>(logits, T, E, k, renorm, \
+                                                              topk_idx, topk_w, rank,  \
+                                                              tile_counts)
+  if (E <= 32) MOE_ROUTE_LAUNCH(1);
+  else if (E <= 64) MOE_ROUTE_LAUNCH(2);
+  else if (E <= 128) MOE_ROUTE_LAUNCH(4);
+  else if (E <= 256) MOE_ROUTE_LAUNCH(8);
+  else if (E <= 512) MOE_ROUTE_LAUNCH(16);
+  else MOE_ROUTE_LAUNCH(32);
+#undef MOE_ROUTE_LAUNCH
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  moe::permute_scatter_kernel<<<ntiles, moe::kThreads, 0, s>>>(
+      topk_idx, rank, tile_counts, T, E, k, ntiles, offsets, sorted_rows, inv_perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe_launch

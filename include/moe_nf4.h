@@ -1,0 +1,240 @@
+/*
+ * moe_nf4.h -- C ABI of the B200 (sm_100a) NF4 grouped mixture-of-experts
+ * library (libmoenf4.so).
+ *
+ * The library runs one mixture-of-experts layer directly on 4-bit NF4 expert
+ * weights: top-k routing and a token->expert permutation, one grouped GEMM
+ * launch over all active experts for gate_up with SiLU(gate)*up fused in its
+ * epilogue, a grouped down projection, and a routing-weighted combine.  The
+ * NF4 codebook and per-block absmax are decoded in registers inside the GEMM;
+ * no dequantized weight copy is ever written to memory.  The method is the
+ * one described in "grouped-nf4-gemm & experts-4bit" (jordananderson-pages
+ * .pages.dev), first bullet, and in the "grouped-nf4-gemm" bullet of the
+ * pjordanandrsn GitHub profile page.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All pointers are DEVICE pointers unless a parameter says otherwise; the
+ *   caller allocates and owns every buffer (inputs, outputs, workspace).  The
+ *   library keeps no mutable global state between calls.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every call only enqueues work: it is asynchronous and
+ *   stream-ordered, and never synchronizes the device.
+ * - Matrices are dense and row-major.  Sizes are element counts.
+ * - Synchronous argument errors return at once and enqueue nothing.
+ *   A launch failure returns MOE_ERR_CUDA.  Contract violations that only
+ *   the device can see (non-finite weights, inconsistent expert offsets,
+ *   an expert index out of range) set a bit in the caller's device word
+ *   `dev_err` (int32, may be NULL) and the affected work is skipped; the
+ *   caller reads the word when it chooses.  No kernel traps or asserts.
+ * - sm_100a only: calls on another architecture return MOE_ERR_UNSUPPORTED.
+ *
+ * NF4 weight layout (the fused 3-D expert parameter of "4-bit
+ * Mixture-of-Experts fine-tuning on small GPUs", jordananderson.work, first
+ * bullet, quantized as in "grouped-nf4-gemm & experts-4bit", first bullet):
+ * - a stack of E experts, each an [N, K] out x in matrix, K % 64 == 0;
+ * - packed  uint8 [E, N, K/2]: element 2j of a row in the HIGH nibble of
+ *   byte j, element 2j+1 in the low nibble;
+ * - absmax  fp32  [E, N*K/64]: one scale per 64 consecutive elements of a
+ *   row; weight = NF4_LEVEL[code] * absmax.
+ * gate_up stacks are [E, 2I, H] with rows [0, I) the gate and [I, 2I) the
+ * up projection; down stacks are [E, H, I].
+ */
+#ifndef MOE_NF4_H
+#define MOE_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_NF4_ABI_VERSION 1
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size or enum value       */
+  MOE_ERR_MISALIGNED = 2,  /* a pointer is not 16-byte aligned           */
+  MOE_ERR_UNSUPPORTED = 3, /* shape or device this build does not cover  */
+  MOE_ERR_WORKSPACE = 4,   /* workspace missing or too small             */
+  MOE_ERR_CUDA = 5         /* a CUDA launch or runtime call failed       */
+} moe_status_t;
+
+typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1, MOE_DT_F16 = 2 } moe_dtype_t;
+
+typedef enum { MOE_EPI_NONE = 0, MOE_EPI_SWIGLU = 1 } moe_epilogue_t;
+
+/* Grouped-GEMM kernel choice.  AUTO picks GEMV for small row counts and the
+ * tensor-memory (tcgen05) kernel otherwise; the others force one path. */
+typedef enum {
+  MOE_ALGO_AUTO = 0,
+  MOE_ALGO_GEMV = 1, /* decode: streams weights, warp MMA per 16 rows      */
+  MOE_ALGO_TC = 2    /* prefill: tcgen05.mma with TMEM accumulators        */
+} moe_algo_t;
+
+/* Bits the kernels OR into the caller's device error word. */
+#define MOE_DEVERR_NONFINITE 0x1   /* quantize saw a NaN or Inf weight      */
+#define MOE_DEVERR_BAD_OFFSETS 0x2 /* expert_offsets not monotone / total   */
+#define MOE_DEVERR_BAD_INDEX 0x4   /* a row or expert index out of range    */
+#define MOE_DEVERR_TIMEOUT 0x8     /* a bounded wait inside a kernel expired */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status_t status);
+
+/* MOE_NF4_ABI_VERSION of the loaded library. */
+int moe_abi_version(void);
+
+/* Copies the library's 16 NF4 levels (fp32, ascending, code c -> level c)
+ * into HOST memory `levels_out[16]`.  Host-only, no CUDA call. */
+moe_status_t moe_nf4_levels(float* levels_out);
+
+/*
+ * moe_nf4_quantize -- blockwise NF4 quantization of a fused expert stack.
+ * ("4-bit Mixture-of-Experts fine-tuning on small GPUs", jordananderson.work,
+ * second bullet: the primitive that quantizes the fused expert stack.)
+ *
+ *   W       fp32  [E, N, K]    input weights (device, read only)
+ *   E, N, K >= 1, K % 64 == 0
+ *   blocksize must be 64
+ *   packed  uint8 [E, N, K/2]  output codes (device)
+ *   absmax  fp32  [E, N*K/64]  output scales (device)
+ *   dev_err int32 device word or NULL; MOE_DEVERR_NONFINITE is set if any
+ *           weight is NaN/Inf (its block's codes are then unspecified).
+ * Per 64-block: a = max|x|; a == 0 -> every code 7; else n = x / a (IEEE
+ * fp32 division) and code = #{i : n > fl32(L_i + L_{i+1}) * 0.5}, i.e. the
+ * nearest level with ties to the lower code.  Deterministic, bit-exact.
+ * W, packed and absmax must be 16-byte aligned.
+ */
+moe_status_t moe_nf4_quantize(const float* W, int E, int N, int K,
+                              int blocksize, uint8_t* packed, float* absmax,
+                              int32_t* dev_err, void* stream);
+
+/*
+ * Inverse of the quantizer for inspection and tests: out[E, N, K] =
+ * L[code] * absmax, the exact product rounded once to `out_dtype`.
+ */
+moe_status_t moe_nf4_dequantize(const uint8_t* packed, const float* absmax,
+                                int E, int N, int K, void* out,
+                                moe_dtype_t out_dtype, void* stream);
+
+/*
+ * Workspace bytes moe_route_permute needs for (T, E, k).  `bytes` is a HOST
+ * pointer.  Host-only, no CUDA call.
+ */
+moe_status_t moe_route_permute_workspace_size(int T, int E, int k,
+                                              size_t* bytes);
+
+/*
+ * moe_route_permute -- top-k softmax routing and the token->expert
+ * permutation.  (The router of "grouped-nf4-gemm & experts-4bit", second
+ * bullet; the per-expert row segments one grouped launch needs, first
+ * bullet.)
+ *
+ *   logits         fp32  [T, E]   router logits (device)
+ *   T >= 0; 1 <= E <= 1024; 1 <= k <= min(E, 32)
+ *   renormalize    1: weights = softmax over the k chosen logits;
+ *                  0: weights = softmax over all E logits, taken at the k
+ *   topk_idx       int32 [T, k]   chosen experts, descending logit, equal
+ *                                 logits -> lower expert index first
+ *   topk_w         fp32  [T, k]   routing weights
+ *   expert_offsets int32 [E+1]    segment starts; offsets[E] == T*k
+ *   sorted_rows    int32 [T*k]    flat id t*k+j at each permuted position,
+ *                                 stable: by expert, then by flat id
+ *   inv_perm       int32 [T*k]    permuted position of each flat id
+ *   workspace      device scratch of moe_route_permute_workspace_size bytes
+ * Indices, offsets and the permutation are deterministic and bit-exact;
+ * the weights are fp32 (expf, fixed reduction order).  Logits must be
+ * finite.  All pointers 16-byte aligned.
+ */
+moe_status_t moe_route_permute(const float* logits, int T, int E, int k,
+                               int renormalize, int32_t* topk_idx,
+                               float* topk_w, int32_t* expert_offsets,
+                               int32_t* sorted_rows, int32_t* inv_perm,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * moe_nf4_grouped_gemm -- one launch over all experts:
+ *   out[p, :] = W[e(p)] . A[r(p), :]   for p in [0, M_total)
+ * where e(p) is the expert whose segment [offsets[e], offsets[e+1]) holds p
+ * and r(p) = gather[p] / k when `gather` is given (the routed token of the
+ * permuted row), else p.  The NF4 weights are decoded in registers.
+ * ("grouped-nf4-gemm & experts-4bit", first bullet: one launch for all active
+ * experts, codebook decoded inside the GEMM, no dequantize-to-bf16 round
+ * trip.)
+ *
+ *   A        [A_rows, K] BF16 or F16 activations; with `gather` A holds the
+ *            T tokens (A_rows = T), without it one row per position
+ *            (A_rows >= M_total, checked on the host)
+ *   gather   int32 [M_total] or NULL; k = the routing top-k (used with
+ *            gather only).  A gathered id f must satisfy 0 <= f < M_total
+ *            and f / k < A_rows, else MOE_DEVERR_BAD_INDEX is set and the
+ *            row is computed as zeros
+ *   packed   uint8 [E, N, K/2], absmax fp32 [E, N*K/64]
+ *   expert_offsets int32 [E+1], monotone, offsets[E] == M_total (checked on
+ *            the device: violation -> MOE_DEVERR_BAD_OFFSETS, no output)
+ *   N % 64 == 0 (for SWIGLU N = 2I); K % 64 == 0
+ *   epilogue NONE:   out [M_total, N]
+ *            SWIGLU: out [M_total, N/2] = silu(g) * u with g the first N/2
+ *                    outputs (gate rows) and u the last N/2 (up rows)
+ *   out_dtype F32, BF16 or F16 (rounded once from the fp32 accumulator)
+ *   algo     MOE_ALGO_AUTO / _GEMV / _TC
+ * Accumulation is fp32; weights enter the tensor cores as fp16 (the exact
+ * fp16 rounding of each level, or of level*absmax), activations as fp16.
+ * All pointers 16-byte aligned.
+ */
+moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype,
+                                  int A_rows, const int32_t* gather, int k,
+                                  const uint8_t* packed, const float* absmax,
+                                  const int32_t* expert_offsets, int E, int N,
+                                  int K, int M_total, moe_epilogue_t epilogue,
+                                  void* out, moe_dtype_t out_dtype,
+                                  moe_algo_t algo, int32_t* dev_err,
+                                  void* stream);
+
+/*
+ * moe_swiglu -- standalone h[m, i] = silu(gu[m, i]) * gu[m, I + i],
+ * silu(g) = g / (1 + exp(-g)), for gu [M, 2I] (F32, BF16 or F16) into
+ * h [M, I] of h_dtype.  The fused path never calls this; it exists for
+ * callers that keep gate_up outputs.  I % 4 == 0, pointers 16-byte aligned.
+ */
+moe_status_t moe_swiglu(const void* gu, moe_dtype_t gu_dtype, int M, int I,
+                        void* h, moe_dtype_t h_dtype, void* stream);
+
+/*
+ * moe_unpermute_combine -- Y[t, :] = sum_{j<k} topk_w[t, j] *
+ * Yp[inv_perm[t*k + j], :], summed in j order in fp32.
+ *   Yp [T*k, H] of yp_dtype (F32, BF16, F16), Y [T, H] of y_dtype.
+ *   H % 4 == 0, pointers 16-byte aligned.
+ */
+moe_status_t moe_unpermute_combine(const void* Yp, moe_dtype_t yp_dtype,
+                                   const int32_t* inv_perm,
+                                   const float* topk_w, int T, int k, int H,
+                                   void* Y, moe_dtype_t y_dtype,
+                                   void* stream);
+
+/*
+ * Whole layer in one call (route -> permute -> gate_up+SwiGLU -> down ->
+ * combine), each step the entry point above, all on `stream`.
+ *   X bf16 [T, H]; logits fp32 [T, E]; gate_up stack [E, 2I, H];
+ *   down stack [E, H, I]; Y fp32 [T, H].
+ *   workspace: moe_layer_workspace_size bytes; it holds the routing outputs
+ *   and the fp16 intermediates [T*k, I] and [T*k, H].
+ */
+moe_status_t moe_layer_workspace_size(int T, int E, int k, int H, int I,
+                                      size_t* bytes);
+moe_status_t moe_layer_forward(const void* X, const float* logits, int T,
+                               int E, int k, int renormalize, int H, int I,
+                               const uint8_t* packed_gu,
+                               const float* absmax_gu,
+                               const uint8_t* packed_d, const float* absmax_d,
+                               float* Y, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_err,
+                               void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_NF4_H */

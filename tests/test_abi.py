@@ -1,0 +1,121 @@
+"""The C-ABI library loads and exports what include/moe_nf4.h declares (CPU).
+
+No compute call is made: the host-only entry points (status strings, levels,
+workspace sizes) are exercised, and argument validation is checked on calls
+that must be rejected before any CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_mixture_experts_route_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from bit_mixture_experts_route_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_five_path_calls():
+    names = _declared()
+    for n in ("moe_nf4_quantize", "moe_route_permute", "moe_nf4_grouped_gemm", "moe_swiglu",
+              "moe_unpermute_combine"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.moe_abi_version() == 1
+    for code, name in _lib.STATUS.items():
+        assert lib.moe_status_string(code).decode() == name
+
+
+def test_library_levels_equal_oracle_levels_bitwise(lib):
+    got = np.array(_lib.nf4_levels(), dtype=np.float32)
+    assert np.array_equal(got.view(np.int32), oracle.nf4_levels().view(np.int32))
+
+
+def test_route_workspace_size(lib):
+    n = _lib.route_permute_workspace_size(4096, 128, 8)
+    assert n >= 4096 * 8 * 4 + 64 * 128 * 4
+    with pytest.raises(_lib.MoEError):
+        _lib.route_permute_workspace_size(16, 8, 9)   # k > E
+    with pytest.raises(_lib.MoEError):
+        _lib.route_permute_workspace_size(16, 2048, 8)  # E > 1024
+
+
+def test_layer_workspace_size(lib):
+    n = _lib.layer_workspace_size(64, 64, 8, 2048, 1024)
+    assert n >= 64 * 8 * (1024 + 2048) * 2
+
+
+# Fake, never-dereferenced device addresses: validation must reject these
+# calls before touching CUDA.
+ALIGNED = ctypes.c_void_p(0x7000_0000)
+MISALIGNED = ctypes.c_void_p(0x7000_0004)
+
+
+def test_quantize_rejects_bad_arguments(lib):
+    q = lib.moe_nf4_quantize
+    assert q(ALIGNED, 1, 64, 100, 64, ALIGNED, ALIGNED, None, None) == 1   # K % 64
+    assert q(ALIGNED, 1, 64, 128, 32, ALIGNED, ALIGNED, None, None) == 1   # blocksize
+    assert q(None, 1, 64, 128, 64, ALIGNED, ALIGNED, None, None) == 1      # null W
+    assert q(MISALIGNED, 1, 64, 128, 64, ALIGNED, ALIGNED, None, None) == 2
+
+
+def test_grouped_gemm_rejects_bad_arguments(lib):
+    g = lib.moe_nf4_grouped_gemm
+    args = dict(A=ALIGNED, adt=1, arows=32, gather=ALIGNED, k=8, packed=ALIGNED, absmax=ALIGNED,
+                off=ALIGNED, E=8, N=1024, K=256, M=32, epi=1, out=ALIGNED, odt=0, algo=0,
+                err=None, s=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return g(*a.values())
+
+    assert call(adt=0) == 1            # fp32 activations are not accepted
+    assert call(K=100) == 1            # K % 64
+    assert call(N=100) == 1            # N % 64
+    assert call(epi=7) == 1
+    assert call(algo=9) == 1
+    assert call(E=0) == 1
+    assert call(packed=None) == 1
+    assert call(out=MISALIGNED) == 2
+    assert call(gather=None, arows=10) == 1   # without gather A needs M_total rows
+
+
+def test_route_permute_rejects_small_workspace(lib):
+    r = lib.moe_route_permute
+    assert r(ALIGNED, 16, 8, 2, 1, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 8,
+             None) == 4
+    assert r(ALIGNED, 16, 8, 9, 1, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+             1 << 20, None) == 1
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/libmoenf4.so")
+    with pytest.raises(_lib.MoEError):
+        _lib.load()
