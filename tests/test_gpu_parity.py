@@ -196,7 +196,10 @@ def test_grouped_gemm_output_dtypes(out_dtype):
                                out_dtype=out_dtype)
     pr, ar = oracle.quantize_blockwise(W.numpy())
     ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
-    rel, mae = assert_close(_np(out.float()), ref, str(out_dtype))
+    # A 16-bit output carries its own rounding (bf16: up to 2^-9 relative),
+    # so it is compared with the oracle's value rounded once to that type.
+    ref_rounded = torch.from_numpy(ref).to(out_dtype).double().numpy()
+    assert_close(_np(out.float()), ref_rounded, str(out_dtype))
     assert out.dtype == out_dtype
 
 
