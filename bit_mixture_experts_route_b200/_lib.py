@@ -37,6 +37,7 @@ SIGNATURES = {
     "moe_route_permute": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _S]),
     "moe_nf4_grouped_gemm": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                   _I, _I, _P, _S]),
+    "moe_permute_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _S]),
     "moe_swiglu": (_I, [_P, _I, _I, _I, _P, _I, _S]),
     "moe_unpermute_combine": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _S]),
     "moe_layer_workspace_size": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
@@ -175,6 +176,22 @@ def nf4_grouped_gemm(A, packed, absmax, expert_offsets, M_total, gather=None, k=
         _ptr(A), DT[A.dtype], A.shape[0], _ptr(gather), k, _ptr(packed), _ptr(absmax),
         _ptr(expert_offsets), E, N, K, M_total, EPI[epilogue], _ptr(out), DT[out.dtype],
         ALGO[algo], _ptr(dev_err), _stream(A.device)), "moe_nf4_grouped_gemm")
+    return out
+
+
+def permute_rows(X, sorted_rows, k, M_total=None, out=None, dev_err=None):
+    """``Xp[p] = fp16(X[sorted_rows[p] // k])`` -> ``fp16 [M_total, K]``."""
+    if X.dtype not in (torch.bfloat16, torch.float16):
+        raise MoEError("X must be bf16 or fp16")
+    _need(X, X.dtype, "X", 2)
+    _need(sorted_rows, torch.int32, "sorted_rows", 1)
+    T, K = X.shape
+    M = sorted_rows.numel() if M_total is None else M_total
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.float16, device=X.device)
+    _check(load().moe_permute_rows(_ptr(X), DT[X.dtype], T, K, _ptr(sorted_rows), k, M,
+                                   _ptr(out), _ptr(dev_err), _stream(X.device)),
+           "moe_permute_rows")
     return out
 
 

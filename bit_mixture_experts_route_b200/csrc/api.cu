@@ -122,7 +122,8 @@ moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows
   if (moe_status_t st = check_device()) return st;
   if (M_total == 0) return MOE_OK;
   const cudaStream_t s = (cudaStream_t)stream;
-  const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue);
+  const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue) && !gather &&
+                     a_dtype == MOE_DT_F16;
   bool use_tc;
   if (algo == MOE_ALGO_TC) {
     if (!tc_ok) return MOE_ERR_UNSUPPORTED;
@@ -142,6 +143,21 @@ moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows
   return from_cuda(moe_launch::grouped_gemm_gemv(A, a_dtype, A_rows, gather, k, packed, absmax,
                                                  expert_offsets, E, N, K, M_total, epilogue,
                                                  out, out_dtype, dev_err, s));
+}
+
+moe_status_t moe_permute_rows(const void* X, moe_dtype_t x_dtype, int T, int K,
+                              const int32_t* sorted_rows, int k, int M_total, void* Xp,
+                              int32_t* dev_err, void* stream) {
+  if ((x_dtype != MOE_DT_BF16 && x_dtype != MOE_DT_F16) || T < 0 || K < 8 || K % 8 || k < 1 ||
+      M_total < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (M_total > 0 && (!X || !sorted_rows || !Xp)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, sorted_rows, Xp};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(moe_launch::permute_rows(X, x_dtype, T, K, sorted_rows, k, M_total, Xp,
+                                            dev_err, (cudaStream_t)stream));
 }
 
 moe_status_t moe_swiglu(const void* gu, moe_dtype_t gu_dtype, int M, int I, void* h,
@@ -169,8 +185,9 @@ moe_status_t moe_unpermute_combine(const void* Yp, moe_dtype_t yp_dtype, const i
 }
 
 // Layer workspace: [topk_idx | topk_w | offsets | sorted_rows | inv_perm |
-// route scratch | Hbuf fp16 [T*k, I] | Yp fp16 [T*k, H]], each 256-aligned.
-static void layer_layout(int T, int E, int k, int H, int I, size_t off[8]) {
+// route scratch | Hbuf fp16 [T*k, I] | Yp fp16 [T*k, H] | Xp fp16 [T*k, H]],
+// each 256-aligned.
+static void layer_layout(int T, int E, int k, int H, int I, size_t off[9]) {
   const size_t tk = (size_t)T * k;
   off[0] = 0;
   off[1] = off[0] + align256(tk * 4);
@@ -180,14 +197,15 @@ static void layer_layout(int T, int E, int k, int H, int I, size_t off[8]) {
   off[5] = off[4] + align256(tk * 4);
   off[6] = off[5] + align256(moe_launch::route_workspace_bytes(T, E, k));
   off[7] = off[6] + align256(tk * I * 2);
+  off[8] = off[7] + align256(tk * H * 2);
 }
 
 moe_status_t moe_layer_workspace_size(int T, int E, int k, int H, int I, size_t* bytes) {
   if (!bytes || T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32 || H < 1 || I < 1)
     return MOE_ERR_INVALID_ARG;
-  size_t off[8];
+  size_t off[9];
   layer_layout(T, E, k, H, I, off);
-  *bytes = off[7] + align256((size_t)T * k * H * 2);
+  *bytes = off[8] + align256((size_t)T * k * H * 2);
   return MOE_OK;
 }
 
@@ -201,7 +219,7 @@ moe_status_t moe_layer_forward(const void* X, const float* logits, int T, int E,
   if (T == 0) return MOE_OK;
   if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MOE_ERR_MISALIGNED;
-  size_t off[8];
+  size_t off[9];
   layer_layout(T, E, k, H, I, off);
   char* ws = reinterpret_cast<char*>(workspace);
   int32_t* topk_idx = reinterpret_cast<int32_t*>(ws + off[0]);
@@ -216,7 +234,12 @@ moe_status_t moe_layer_forward(const void* X, const float* logits, int T, int E,
   moe_status_t st = moe_route_permute(logits, T, E, k, renormalize, topk_idx, topk_w, offsets,
                                       sorted_rows, inv_perm, rws, off[6] - off[5], stream);
   if (st) return st;
-  st = moe_nf4_grouped_gemm(X, MOE_DT_BF16, T, sorted_rows, k, packed_gu, absmax_gu, offsets, E,
+  // Routed activation rows in expert order, fp16: both grouped kernels read
+  // them without a gather or a conversion in their inner loops.
+  void* xp = ws + off[8];
+  st = moe_permute_rows(X, MOE_DT_BF16, T, H, sorted_rows, k, M, xp, dev_err, stream);
+  if (st) return st;
+  st = moe_nf4_grouped_gemm(xp, MOE_DT_F16, M, nullptr, 1, packed_gu, absmax_gu, offsets, E,
                             2 * I, H, M, MOE_EPI_SWIGLU, hbuf, MOE_DT_F16, MOE_ALGO_AUTO,
                             dev_err, stream);
   if (st) return st;

@@ -1,10 +1,15 @@
 // Shared device helpers of the NF4 MoE library (sm_100a).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <algorithm>
+#include <type_traits>
 
 #include "../../include/moe_nf4.h"
 
@@ -96,6 +101,21 @@ __device__ __forceinline__ float swiglu_f32(float g, float u) {
   return __fdiv_rn(g, 1.0f + expf(-g)) * u;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link-time dependency on libcuda).  Null if the driver lacks it.
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
 }  // namespace moe
 
 // Host-side launchers implemented in the kernel files, called by api.cu.
@@ -117,6 +137,12 @@ cudaError_t grouped_gemm_gemv(const void* A, moe_dtype_t a_dt, int A_rows,
                               int M_total, moe_epilogue_t epi, void* out,
                               moe_dtype_t out_dt, int32_t* dev_err,
                               cudaStream_t s);
+bool grouped_gemm_decode_supported(int N, int K);
+cudaError_t grouped_gemm_decode(const void* A, moe_dtype_t a_dt, int A_rows,
+                                const int32_t* gather, int k, const uint8_t* packed,
+                                const float* absmax, const int32_t* offsets, int E, int N,
+                                int K, int M_total, moe_epilogue_t epi, void* out,
+                                moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);
 cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows,
                             const int32_t* gather, int k,
                             const uint8_t* packed, const float* absmax,
@@ -125,6 +151,8 @@ cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows,
                             moe_dtype_t out_dt, int32_t* dev_err,
                             cudaStream_t s);
 bool grouped_gemm_tc_supported(int N, int K, moe_epilogue_t epi);
+cudaError_t permute_rows(const void* X, moe_dtype_t x_dt, int T, int K, const int32_t* rows,
+                         int k, int M_total, void* Xp, int32_t* dev_err, cudaStream_t s);
 cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h,
                    moe_dtype_t h_dt, cudaStream_t s);
 cudaError_t unpermute_combine(const void* Yp, moe_dtype_t yp_dt,

@@ -4,6 +4,8 @@
 //   swiglu:  h[m, i] = silu(gu[m, i]) * gu[m, I + i]
 //   combine: Y[t, :] = sum_{j<k} w[t, j] * Yp[inv_perm[t*k + j], :], summed in
 //            j order in fp32 (deterministic).
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace moe {
@@ -80,6 +82,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const InT* __restrict__ Yp
   }
 }
 
+// Xp[p, :] = X[sorted_rows[p] / k, :] converted to fp16, one warp per row,
+// 16-byte accesses.  Rows whose id is out of range are zero-filled and flagged.
+template <typename InT>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict__ X, int T, int K,
+                                                           const int32_t* __restrict__ rows, int k,
+                                                           int M_total, __half* __restrict__ Xp,
+                                                           int32_t* dev_err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int p = warp; p < M_total; p += nwarps) {
+    const int f = rows[p];
+    const bool ok = f >= 0 && f < M_total && f / k < T;
+    if (!ok && lane == 0) set_dev_err(dev_err, MOE_DEVERR_BAD_INDEX);
+    const InT* src = X + (size_t)(ok ? f / k : 0) * K;
+    __half* dst = Xp + (size_t)p * K;
+    for (int c = lane * 8; c < K; c += 256) {
+      uint4 o;
+      if (!ok) {
+        o = make_uint4(0, 0, 0, 0);
+      } else if constexpr (sizeof(InT) == 2 && !std::is_same<InT, __half>::value) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src + c);
+        o = make_uint4(bf16x2_to_f16x2(u.x), bf16x2_to_f16x2(u.y), bf16x2_to_f16x2(u.z),
+                       bf16x2_to_f16x2(u.w));
+      } else {
+        o = *reinterpret_cast<const uint4*>(src + c);
+      }
+      *reinterpret_cast<uint4*>(dst + c) = o;
+    }
+  }
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -114,6 +147,20 @@ cudaError_t combine_out(const InT* Yp, const int32_t* inv_perm, const float* w, 
 }  // namespace moe
 
 namespace moe_launch {
+
+cudaError_t permute_rows(const void* X, moe_dtype_t x_dt, int T, int K, const int32_t* rows,
+                         int k, int M_total, void* Xp, int32_t* dev_err, cudaStream_t s) {
+  if (M_total == 0) return cudaSuccess;
+  const int grid = (int)std::min<int64_t>(((int64_t)M_total + 7) / 8,
+                                          (int64_t)moe::sm_count() * 16);
+  if (x_dt == MOE_DT_BF16)
+    moe::permute_rows_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, T, K, rows, k, M_total,
+                                                  (__half*)Xp, dev_err);
+  else
+    moe::permute_rows_kernel<<<grid, 256, 0, s>>>((const __half*)X, T, K, rows, k, M_total,
+                                                  (__half*)Xp, dev_err);
+  return cudaGetLastError();
+}
 
 cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h, moe_dtype_t h_dt,
                    cudaStream_t s) {

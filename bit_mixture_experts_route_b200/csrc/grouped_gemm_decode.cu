@@ -1,0 +1,467 @@
+// Grouped NF4 GEMM, decode path with TMA-staged weights (few rows per
+// expert; HBM-bound).
+//
+// "grouped-nf4-gemm & experts-4bit" (jordananderson-pages.pages.dev), first
+// bullet: one launch for all active experts, the 16-entry codebook decoded in
+// registers, no dequantized weight copy.  At decode sizes the whole cost is
+// streaming the NF4 bytes of every expert that received a token, so the
+// design goal is to keep enough bytes in flight to saturate HBM:
+//
+// * Persistent CTAs (two per SM) walk a list of work items built on the
+//   device from expert_offsets: (expert, 64 weight rows, up to 32 routed rows).
+// * One producer thread streams each item's packed rows through an 8-stage
+//   ring with TMA tile loads (64 rows x 128 bytes = 256 k per stage, 128-byte
+//   swizzle so the consumers' reads are conflict-free) plus the matching
+//   absmax tile; ~72 KB per CTA in flight, independent of registers.
+// * Four consumer warps each own 16 weight rows: per 64-k block a lane reads
+//   8 packed bytes of two rows, maps each byte to an fp16 pair {L[hi], L[lo]}
+//   with one lookup in a per-lane replicated table, and issues
+//   mma.sync.m16n8k16 with the routed rows as the N side (swap-AB); the
+//   block's fp32 absmax scales the block's fp32 partial sums.
+// * The SwiGLU epilogue pairs gate row j and up row I + j in the same lane.
+// Every wait is bounded; on expiry MOE_DEVERR_TIMEOUT is set and all roles
+// leave their loops.
+#include "common.cuh"
+
+namespace moe {
+namespace dec {
+
+constexpr int ROWS = 64;        // weight rows per item
+constexpr int TOK = 32;         // routed rows per item (max)
+constexpr int SK = 256;         // k per stage
+constexpr int SB = SK / 2;      // packed bytes per row per stage
+constexpr int STAGES = 8;
+constexpr int CWARPS = 4;
+constexpr int THREADS = 32 * (CWARPS + 1);
+constexpr uint32_t kSpinLimit = 1u << 24;
+constexpr uint32_t kStageBytes = ROWS * SB + ROWS * 4 * 4;
+
+struct __align__(8) Smem {
+  uint8_t w[STAGES][ROWS * SB];  // 1024-aligned (struct placed at 1024)
+  float a[STAGES][ROWS * 4];
+  uint32_t lut[256 * 32];
+  uint64_t full[STAGES], empty[STAGES];
+  int abort_flag;
+  int nitems;
+  int item_prefix[1025];
+};
+
+__constant__ float c_levels_dec[16] = {MOE_NF4_LEVEL_LIST};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem& sm,
+                                          int32_t* dev_err) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) return false;
+  }
+  *reinterpret_cast<volatile int*>(&sm.abort_flag) = 1;
+  set_dev_err(dev_err, MOE_DEVERR_TIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 16 activations A[row][k0 .. k0+16) as 8 fp16 pairs.
+template <typename AT>
+__device__ __forceinline__ void load_x16(const AT* __restrict__ p, uint32_t (&xf)[8]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  const uint4 u = __ldg(q), v = __ldg(q + 1);
+  if constexpr (std::is_same<AT, __half>::value) {
+    xf[0] = u.x; xf[1] = u.y; xf[2] = u.z; xf[3] = u.w;
+    xf[4] = v.x; xf[5] = v.y; xf[6] = v.z; xf[7] = v.w;
+  } else {
+    xf[0] = bf16x2_to_f16x2(u.x); xf[1] = bf16x2_to_f16x2(u.y);
+    xf[2] = bf16x2_to_f16x2(u.z); xf[3] = bf16x2_to_f16x2(u.w);
+    xf[4] = bf16x2_to_f16x2(v.x); xf[5] = bf16x2_to_f16x2(v.y);
+    xf[6] = bf16x2_to_f16x2(v.z); xf[7] = bf16x2_to_f16x2(v.w);
+  }
+}
+
+struct Item {
+  int expert, rtile, start, cnt;  // routed rows [start, start + cnt)
+};
+
+__device__ __forceinline__ Item item_info(const Smem& sm, const int32_t* offsets, int E,
+                                          int rtiles, int it) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (sm.item_prefix[mid] <= it) lo = mid; else hi = mid;
+  }
+  const int local = it - sm.item_prefix[lo];
+  const int tc = local / rtiles;
+  Item r;
+  r.expert = lo;
+  r.rtile = local - tc * rtiles;
+  const int s = offsets[lo], e = offsets[lo + 1];
+  r.start = s + tc * TOK;
+  r.cnt = min(TOK, e - r.start);
+  return r;
+}
+
+// One item's main loop and epilogue for one consumer warp, NT8 token tiles.
+template <typename AT, int EPI, typename OutT, int NT8>
+__device__ __forceinline__ bool consume_item(
+    Smem& sm, const Item& it, const AT* __restrict__ A, int A_rows,
+    const int32_t* __restrict__ gather, int k, int N, int K, int M_total, OutT* __restrict__ out,
+    int32_t* dev_err, int& stage, uint32_t& phase) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + g : 16 * warp + g;
+  const int rB = (EPI == MOE_EPI_SWIGLU) ? 32 + 8 * warp + g : 16 * warp + g + 8;
+
+  const AT* xrow[NT8];
+  bool xok[NT8];
+#pragma unroll
+  for (int j = 0; j < NT8; ++j) {
+    const int tok = 8 * j + g;
+    xok[j] = tok < it.cnt;
+    int r = 0;
+    if (xok[j]) {
+      const int p = it.start + tok;
+      if (gather) {
+        const int f = gather[p];
+        if (f < 0 || f >= M_total || f / k >= A_rows) {
+          set_dev_err(dev_err, MOE_DEVERR_BAD_INDEX);
+          xok[j] = false;
+        } else {
+          r = f / k;
+        }
+      } else {
+        r = p;
+      }
+    }
+    xrow[j] = A + (size_t)r * K + 16 * t;
+  }
+
+  float acc[NT8][4];
+#pragma unroll
+  for (int j = 0; j < NT8; ++j)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[j][q] = 0.0f;
+
+  const uint32_t* lut = sm.lut + lane;
+  const int KS = K / SK;
+  for (int s = 0; s < KS; ++s) {
+    if (!mbar_wait(&sm.full[stage], phase, sm, dev_err)) return false;
+    const uint8_t* wst = sm.w[stage];
+    const float4 sa = *reinterpret_cast<const float4*>(&sm.a[stage][rA * 4]);
+    const float4 sb = *reinterpret_cast<const float4*>(&sm.a[stage][rB * 4]);
+    const float sav[4] = {sa.x, sa.y, sa.z, sa.w};
+    const float sbv[4] = {sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      uint32_t xf[NT8][8];
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        if (xok[j]) {
+          load_x16<AT>(xrow[j] + (size_t)(s * SK + b * kBlock), xf[j]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xf[j][q] = 0u;
+        }
+      }
+      // byte offset of this lane's 8 bytes in the row, 128-byte swizzled
+      const int off = b * 32 + 8 * t;
+      const uint2 wa = *reinterpret_cast<const uint2*>(
+          wst + rA * SB + ((((off >> 4) ^ (rA & 7)) << 4) | (off & 15)));
+      const uint2 wb = *reinterpret_cast<const uint2*>(
+          wst + rB * SB + ((((off >> 4) ^ (rB & 7)) << 4) | (off & 15)));
+      float tmp[NT8][4];
+#pragma unroll
+      for (int j = 0; j < NT8; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmp[j][q] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t vA = (i < 2) ? wa.x : wa.y;
+        const uint32_t vB = (i < 2) ? wb.x : wb.y;
+        const int sh = (i & 1) * 16;
+        uint32_t af[4];
+        af[0] = lut[((vA >> sh) & 0xffu) << 5];
+        af[1] = lut[((vB >> sh) & 0xffu) << 5];
+        af[2] = lut[((vA >> (sh + 8)) & 0xffu) << 5];
+        af[3] = lut[((vB >> (sh + 8)) & 0xffu) << 5];
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) mma_16816(tmp[j], af, xf[j][2 * i], xf[j][2 * i + 1]);
+      }
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        acc[j][0] = fmaf(sav[b], tmp[j][0], acc[j][0]);
+        acc[j][1] = fmaf(sav[b], tmp[j][1], acc[j][1]);
+        acc[j][2] = fmaf(sbv[b], tmp[j][2], acc[j][2]);
+        acc[j][3] = fmaf(sbv[b], tmp[j][3], acc[j][3]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[stage]);
+    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+  }
+
+  // acc[j][q]: row rA (q < 2) or rB (q >= 2), routed row 8j + 2t + (q & 1)
+#pragma unroll
+  for (int j = 0; j < NT8; ++j) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int tok = 8 * j + 2 * t + q;
+      if (tok >= it.cnt) continue;
+      const size_t p = (size_t)(it.start + tok);
+      if (EPI == MOE_EPI_SWIGLU) {
+        const int I = N / 2;
+        const int col = it.rtile * (ROWS / 2) + 8 * warp + g;
+        out[p * I + col] = from_f32<OutT>(swiglu_f32(acc[j][q], acc[j][q + 2]));
+      } else {
+        const int col = it.rtile * ROWS + 16 * warp + g;
+        out[p * N + col] = from_f32<OutT>(acc[j][q]);
+        out[p * N + col + 8] = from_f32<OutT>(acc[j][q + 2]);
+      }
+    }
+  }
+  return true;
+}
+
+template <typename AT, int EPI, typename OutT>
+__global__ void __launch_bounds__(THREADS, 2) nf4_decode_kernel(
+    const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
+    const AT* __restrict__ A, int A_rows, const int32_t* __restrict__ gather, int k,
+    const int32_t* __restrict__ offsets, int E, int N, int K, int M_total,
+    OutT* __restrict__ out, int32_t* dev_err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rtiles = N / ROWS;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], CWARPS);
+    }
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = threadIdx.x; i < 256 * 32; i += THREADS) {
+    const int b = i >> 5;
+    const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
+                                     __float2half_rn(c_levels_dec[b & 15]));
+    sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  if (warp == CWARPS) {
+    // item_prefix[e] = sum over e' < e of ceil(count / TOK) * rtiles
+    bool bad = offsets[0] != 0 || offsets[E] != M_total;
+    int run = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int c = 0;
+      if (e < E) {
+        c = offsets[e + 1] - offsets[e];
+        if (c < 0) { bad = true; c = 0; }
+      }
+      const int items = ((c + TOK - 1) / TOK) * rtiles;
+      int incl = items;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (e < E) sm.item_prefix[e] = run + incl - items;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      sm.item_prefix[E] = run;
+      sm.nitems = bad ? 0 : run;
+      if (bad) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  const int total = sm.nitems;
+  const int KS = K / SK;
+
+  if (warp == CWARPS) {
+    // ---------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        const Item it = item_info(sm, offsets, E, rtiles, i);
+        int y0, y1;
+        if (EPI == MOE_EPI_SWIGLU) {
+          y0 = it.expert * N + it.rtile * (ROWS / 2);
+          y1 = y0 + N / 2;
+        } else {
+          y0 = it.expert * N + it.rtile * ROWS;
+          y1 = y0 + ROWS / 2;
+        }
+        for (int s = 0; s < KS; ++s) {
+          if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
+          mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+          tma_load_2d(sm.w[stage], &wmap, &sm.full[stage], s * SB, y0);
+          tma_load_2d(sm.w[stage] + (ROWS / 2) * SB, &wmap, &sm.full[stage], s * SB, y1);
+          tma_load_2d(sm.a[stage], &amap, &sm.full[stage], s * 4, y0);
+          tma_load_2d(sm.a[stage] + (ROWS / 2) * 4, &amap, &sm.full[stage], s * 4, y1);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else {
+    // ---------------- consumers
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int i = blockIdx.x; i < total; i += gridDim.x) {
+      const Item it = item_info(sm, offsets, E, rtiles, i);
+      bool ok;
+      if (it.cnt > 24)
+        ok = consume_item<AT, EPI, OutT, 4>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
+                                            dev_err, stage, phase);
+      else if (it.cnt > 16)
+        ok = consume_item<AT, EPI, OutT, 3>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
+                                            dev_err, stage, phase);
+      else if (it.cnt > 8)
+        ok = consume_item<AT, EPI, OutT, 2>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
+                                            dev_err, stage, phase);
+      else
+        ok = consume_item<AT, EPI, OutT, 1>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
+                                            dev_err, stage, phase);
+      if (!ok) break;
+    }
+  }
+  __syncthreads();
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <typename AT, int EPI, typename OutT>
+cudaError_t launch(const void* A, int A_rows, const int32_t* gather, int k,
+                   const uint8_t* packed, const float* absmax, const int32_t* offsets, int E,
+                   int N, int K, int M_total, void* out, int32_t* dev_err, cudaStream_t s) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap wmap, amap;
+  const cuuint32_t estr[2] = {1, 1};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)E * N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t box[2] = {SB, ROWS / 2};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)K / kBlock, (cuuint64_t)E * N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K / kBlock * 4};
+    const cuuint32_t box[2] = {SK / kBlock, ROWS / 2};
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(absmax), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const size_t smem = sizeof(Smem) + 1024;
+  auto kern = nf4_decode_kernel<AT, EPI, OutT>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const int64_t max_items = ((int64_t)M_total / TOK + E) * (N / ROWS);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(2 * sm_count(), max_items));
+  kern<<<grid, THREADS, smem, s>>>(wmap, amap, reinterpret_cast<const AT*>(A), A_rows, gather, k,
+                                   offsets, E, N, K, M_total, reinterpret_cast<OutT*>(out),
+                                   dev_err);
+  return cudaGetLastError();
+}
+
+template <typename AT, int EPI>
+cudaError_t launch_out(const void* A, int A_rows, const int32_t* gather, int k,
+                       const uint8_t* packed, const float* absmax, const int32_t* offsets, int E,
+                       int N, int K, int M_total, void* out, moe_dtype_t out_dt,
+                       int32_t* dev_err, cudaStream_t s) {
+  if (out_dt == MOE_DT_F32)
+    return launch<AT, EPI, float>(A, A_rows, gather, k, packed, absmax, offsets, E, N, K,
+                                  M_total, out, dev_err, s);
+  if (out_dt == MOE_DT_F16)
+    return launch<AT, EPI, __half>(A, A_rows, gather, k, packed, absmax, offsets, E, N, K,
+                                   M_total, out, dev_err, s);
+  return launch<AT, EPI, __nv_bfloat16>(A, A_rows, gather, k, packed, absmax, offsets, E, N, K,
+                                        M_total, out, dev_err, s);
+}
+
+}  // namespace dec
+}  // namespace moe
+
+namespace moe_launch {
+
+bool grouped_gemm_decode_supported(int N, int K) {
+  // absmax rows must be a multiple of 16 bytes for the TMA map: K % 256.
+  return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
+}
+
+cudaError_t grouped_gemm_decode(const void* A, moe_dtype_t a_dt, int A_rows,
+                                const int32_t* gather, int k, const uint8_t* packed,
+                                const float* absmax, const int32_t* offsets, int E, int N, int K,
+                                int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
+                                int32_t* dev_err, cudaStream_t s) {
+  using namespace moe::dec;
+  if (a_dt == MOE_DT_BF16) {
+    return epi == MOE_EPI_SWIGLU
+               ? launch_out<__nv_bfloat16, MOE_EPI_SWIGLU>(A, A_rows, gather, k, packed, absmax,
+                                                           offsets, E, N, K, M_total, out,
+                                                           out_dt, dev_err, s)
+               : launch_out<__nv_bfloat16, MOE_EPI_NONE>(A, A_rows, gather, k, packed, absmax,
+                                                         offsets, E, N, K, M_total, out, out_dt,
+                                                         dev_err, s);
+  }
+  return epi == MOE_EPI_SWIGLU
+             ? launch_out<__half, MOE_EPI_SWIGLU>(A, A_rows, gather, k, packed, absmax, offsets,
+                                                  E, N, K, M_total, out, out_dt, dev_err, s)
+             : launch_out<__half, MOE_EPI_NONE>(A, A_rows, gather, k, packed, absmax, offsets, E,
+                                                N, K, M_total, out, out_dt, dev_err, s);
+}
+
+}  // namespace moe_launch

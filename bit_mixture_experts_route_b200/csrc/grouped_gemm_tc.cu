@@ -1,16 +1,500 @@
-// Grouped NF4 GEMM, prefill path (tcgen05 tensor cores, TMEM accumulators).
-// Not yet available in this build: the dispatcher routes every size to the
-// GEMV kernel.
+// Grouped NF4 GEMM, prefill path: tcgen05 tensor cores, TMEM accumulators.
+//
+// "grouped-nf4-gemm & experts-4bit" (jordananderson-pages.pages.dev), first
+// bullet: one launch for all active experts, the codebook decoded inside the
+// GEMM, no dequantized copy of the weights in memory.  At prefill sizes
+// (hundreds of routed rows per expert) the work is a dense contraction, so
+// this kernel runs it on the 5th-generation tensor cores.
+//
+// Orientation: the MMA's M side is 128 weight rows (A, decoded NF4), its N
+// side up to 256 routed rows of activations (B, fp16), so each decoded weight
+// feeds up to 512 FLOP.  D = A * B^T lands in TMEM as 128 lanes x N fp32
+// columns; two accumulators (2 x 256 columns) let the epilogue of one tile
+// overlap the main loop of the next.
+//
+// Persistent CTAs walk a tile list built on the device from expert_offsets
+// (expert-major, then token tile, then weight-row tile), so no host sync is
+// needed.  Warp roles (320 threads):
+//   warp 0     TMA producer: activation tiles [256 rows x 64 k] (fp16,
+//              128-byte swizzle) into a 3-stage ring
+//   warp 1     TMEM allocator and MMA issuer (one thread):
+//              tcgen05.mma.cta_group::1.kind::f16, 4 x K16 per stage
+//   warps 2-5  decoders, one thread per weight row: 32 packed bytes and one
+//              fp32 absmax per 64-k step, each byte -> fp16 pair {L[hi],
+//              L[lo]} through a per-lane shared table, times fp16(absmax),
+//              stored in the same 128-byte-swizzled K-major layout
+//   warps 6-9  epilogue: tcgen05.ld 32 columns at a time, SwiGLU (gate and
+//              up rows interleaved in the tile, paired with one shuffle) or a
+//              plain store, then release the accumulator.
+// Every mbarrier wait is bounded; on expiry the kernel sets
+// MOE_DEVERR_TIMEOUT, every role leaves its loop, TMEM is freed and the
+// kernel returns.
 #include "common.cuh"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;          // weight rows per tile (MMA M)
+constexpr int BN = 256;          // routed rows per tile (max MMA N)
+constexpr int BK = 64;           // k per stage = one NF4 block
+constexpr int STAGES = 3;
+constexpr int A_STAGE = BM * BK * 2;   // 16 KB
+constexpr int B_STAGE = BN * BK * 2;   // 32 KB
+constexpr int B_BOX_ROWS = 128;        // TMA box: 64 k x 128 rows
+constexpr int THREADS = 320;
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+struct __align__(8) Smem {
+  uint8_t b[STAGES][B_STAGE];  // 1024-aligned (struct placed at 1024)
+  uint8_t a[STAGES][A_STAGE];
+  uint32_t lut[256 * 32];
+  uint64_t full_a[STAGES], full_b[STAGES], empty[STAGES];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int ntiles_total;
+  int tile_prefix[1025];
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false (and the abort flag set) if the phase never completes
+// or another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem& sm,
+                                          int32_t* dev_err) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) return false;
+  }
+  *reinterpret_cast<volatile int*>(&sm.abort_flag) = 1;
+  set_dev_err(dev_err, MOE_DEVERR_TIMEOUT);
+  return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), sm_100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;               // LBO (unused for swizzled K-major)
+  d |= (uint64_t)(1024u >> 4) << 32;     // SBO
+  d |= (uint64_t)1u << 46;               // version
+  d |= (uint64_t)2u << 61;               // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: D fp32, A/B fp16, both K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_f16(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+        "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+        "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__constant__ float c_levels_tc[16] = {MOE_NF4_LEVEL_LIST};
+
+struct TileInfo {
+  int expert, row0, nrows, ntile;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const Smem& sm, const int32_t* offsets, int E,
+                                              int n_tiles, int t) {
+  // expert e with tile_prefix[e] <= t < tile_prefix[e+1]
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (sm.tile_prefix[mid] <= t) lo = mid; else hi = mid;
+  }
+  const int local = t - sm.tile_prefix[lo];
+  const int tt = local / n_tiles;
+  TileInfo ti;
+  ti.expert = lo;
+  ti.ntile = local - tt * n_tiles;
+  const int start = offsets[lo], end = offsets[lo + 1];
+  ti.row0 = start + tt * BN;
+  ti.nrows = min(BN, end - ti.row0);
+  return ti;
+}
+
+template <int EPI, typename OutT>
+__global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
+    const __grid_constant__ CUtensorMap bmap, const uint8_t* __restrict__ packed,
+    const float* __restrict__ absmax, const int32_t* __restrict__ offsets, int E, int N, int K,
+    int M_total, OutT* __restrict__ out, int32_t* dev_err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = N / BM;
+  const int KT = K / BK;
+
+  // ---- setup: barriers, decode table, tile list, TMEM
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full_a[s], 128);
+      mbar_init(&sm.full_b[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.acc_full[b], 1);
+      mbar_init(&sm.acc_empty[b], 128);
+    }
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = threadIdx.x; i < 256 * 32; i += THREADS) {
+    const int b = i >> 5;
+    const __half2 h = __halves2half2(__float2half_rn(c_levels_tc[b >> 4]),
+                                     __float2half_rn(c_levels_tc[b & 15]));
+    sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  if (warp == 0) {
+    // tile_prefix[e] = sum over e' < e of ceil(count / BN) * n_tiles
+    bool bad = offsets[0] != 0 || offsets[E] != M_total;
+    int run = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int c = 0;
+      if (e < E) {
+        c = offsets[e + 1] - offsets[e];
+        if (c < 0) { bad = true; c = 0; }
+      }
+      int tiles = ((c + BN - 1) / BN) * n_tiles;
+      int incl = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (e < E) sm.tile_prefix[e] = run + incl - tiles;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      sm.tile_prefix[E] = run;
+      sm.ntiles_total = bad ? 0 : run;
+      if (bad) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sm.tmem_base;
+  const int total = sm.ntiles_total;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: activation tiles
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = tile_info(sm, offsets, E, n_tiles, t);
+        const int nmma = (ti.nrows + 15) & ~15;
+        const int boxes = (nmma + B_BOX_ROWS - 1) / B_BOX_ROWS;
+        for (int ks = 0; ks < KT; ++ks) {
+          if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
+          mbar_arrive_expect_tx(&sm.full_b[stage], boxes * B_BOX_ROWS * BK * 2);
+          for (int b = 0; b < boxes; ++b)
+            tma_load_2d(sm.b[stage] + b * (B_BOX_ROWS * BK * 2), &bmap, &sm.full_b[stage],
+                        ks * BK, ti.row0 + b * B_BOX_ROWS);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int lt = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+        const TileInfo ti = tile_info(sm, offsets, E, n_tiles, t);
+        const int nmma = (ti.nrows + 15) & ~15;
+        const int acc = lt & 1;
+        if (!(ok = mbar_wait(&sm.acc_empty[acc], ((lt >> 1) & 1) ^ 1, sm, dev_err))) break;
+        tc_fence_after();
+        const uint32_t idesc = idesc_f16(nmma);
+        const uint32_t dcol = tmem_base + acc * BN;
+        for (int ks = 0; ks < KT; ++ks) {
+          if (!(ok = mbar_wait(&sm.full_a[stage], phase, sm, dev_err))) break;
+          if (!(ok = mbar_wait(&sm.full_b[stage], phase, sm, dev_err))) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sm.a[stage]), b0 = smem_u32(sm.b[stage]);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_f16(dcol, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                    (ks | kk) != 0);
+          mma_commit(&sm.empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (ok) mma_commit(&sm.acc_full[acc]);
+      }
+    }
+  } else if (warp < 6) {
+    // ---------------- decoders: thread m owns tile row m
+    const int m = threadIdx.x - 64;
+    const uint32_t* lut = sm.lut + lane;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const TileInfo ti = tile_info(sm, offsets, E, n_tiles, t);
+      int row;
+      if (EPI == MOE_EPI_SWIGLU) {
+        const int j = ti.ntile * (BM / 2) + (m >> 1);
+        row = (m & 1) ? (N / 2 + j) : j;
+      } else {
+        row = ti.ntile * BM + m;
+      }
+      const size_t grow = (size_t)ti.expert * N + row;
+      const uint4* wp = reinterpret_cast<const uint4*>(packed + grow * (size_t)(K / 2));
+      const float* ap = absmax + grow * (size_t)KT;
+      uint4 q0 = ldg_stream_u4(wp), q1 = ldg_stream_u4(wp + 1);
+      float a = __ldg(ap);
+      for (int ks = 0; ks < KT; ++ks) {
+        // prefetch the next 64-k step while this one is decoded
+        uint4 n0 = q0, n1 = q1;
+        float na = a;
+        if (ks + 1 < KT) {
+          n0 = ldg_stream_u4(wp + 2 * (ks + 1));
+          n1 = ldg_stream_u4(wp + 2 * (ks + 1) + 1);
+          na = __ldg(ap + ks + 1);
+        }
+        if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
+        const __half2 ah = __float2half2_rn(a);
+        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        uint8_t* arow = sm.a[stage] + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t w = words[c];
+          uint32_t h[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t raw = lut[((w >> (8 * i)) & 0xffu) << 5];
+            __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&raw), ah);
+            h[i] = *reinterpret_cast<uint32_t*>(&v);
+          }
+          *reinterpret_cast<uint4*>(arow + ((c ^ (m & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+        fence_proxy_async();
+        mbar_arrive(&sm.full_a[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        q0 = n0; q1 = n1; a = na;
+      }
+    }
+  } else {
+    // ---------------- epilogue: warp q reads TMEM lanes 32q .. 32q+31
+    const int q = warp & 3;
+    const int m = 32 * q + lane;
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    bool ok = true;
+    int lt = 0;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+      const TileInfo ti = tile_info(sm, offsets, E, n_tiles, t);
+      const int acc = lt & 1;
+      if (!(ok = mbar_wait(&sm.acc_full[acc], (lt >> 1) & 1, sm, dev_err))) break;
+      tc_fence_after();
+      const int ncols = (ti.nrows + 15) & ~15;
+      for (int c0 = 0; c0 < ncols; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + lane_addr + acc * BN + c0, v);
+        if (EPI == MOE_EPI_SWIGLU) {
+          const int I = N / 2;
+          const int j = ti.ntile * (BM / 2) + (m >> 1);
+          const bool up = m & 1;
+          // even lane (gate) finishes columns [0,16), odd lane (up) [16,32)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float mine = __uint_as_float(v[i]);
+            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+            const bool owner = up ? (i >= 16) : (i < 16);
+            const int r = c0 + i;
+            if (owner && r < ti.nrows) {
+              const float g = up ? other : mine, u = up ? mine : other;
+              out[(size_t)(ti.row0 + r) * I + j] = from_f32<OutT>(swiglu_f32(g, u));
+            }
+          }
+        } else {
+          const int n = ti.ntile * BM + m;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int r = c0 + i;
+            if (r < ti.nrows)
+              out[(size_t)(ti.row0 + r) * N + n] = from_f32<OutT>(__uint_as_float(v[i]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS));
+  }
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <int EPI, typename OutT>
+cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
+                   const int32_t* offsets, int E, int N, int K, int M_total, void* out,
+                   int32_t* dev_err, cudaStream_t s) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M_total};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {BK, B_BOX_ROWS};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem) + 1024;
+  auto kern = nf4_tc_kernel<EPI, OutT>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  // Upper bound on tiles: every expert's rows rounded up to BN, plus one
+  // partial tile per expert; the kernel derives the exact list itself.
+  const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / BM);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
+  kern<<<grid, THREADS, smem, s>>>(map, packed, absmax, offsets, E, N, K, M_total,
+                                   reinterpret_cast<OutT*>(out), dev_err);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace moe
 
 namespace moe_launch {
 
-bool grouped_gemm_tc_supported(int, int, moe_epilogue_t) { return false; }
+bool grouped_gemm_tc_supported(int N, int K, moe_epilogue_t epi) {
+  (void)epi;
+  return N % moe::tc::BM == 0 && K % moe::tc::BK == 0 && K >= moe::tc::BK;
+}
 
-cudaError_t grouped_gemm_tc(const void*, moe_dtype_t, int, const int32_t*, int, const uint8_t*,
-                            const float*, const int32_t*, int, int, int, int, moe_epilogue_t,
-                            void*, moe_dtype_t, int32_t*, cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows, const int32_t* gather,
+                            int k, const uint8_t* packed, const float* absmax,
+                            const int32_t* offsets, int E, int N, int K, int M_total,
+                            moe_epilogue_t epi, void* out, moe_dtype_t out_dt, int32_t* dev_err,
+                            cudaStream_t s) {
+  (void)k;
+  if (gather || a_dt != MOE_DT_F16 || A_rows < M_total) return cudaErrorNotSupported;
+  using namespace moe::tc;
+  if (epi == MOE_EPI_SWIGLU) {
+    if (out_dt == MOE_DT_F16)
+      return launch<MOE_EPI_SWIGLU, __half>(A, packed, absmax, offsets, E, N, K, M_total, out,
+                                            dev_err, s);
+    if (out_dt == MOE_DT_BF16)
+      return launch<MOE_EPI_SWIGLU, __nv_bfloat16>(A, packed, absmax, offsets, E, N, K,
+                                                   M_total, out, dev_err, s);
+    return launch<MOE_EPI_SWIGLU, float>(A, packed, absmax, offsets, E, N, K, M_total, out,
+                                         dev_err, s);
+  }
+  if (out_dt == MOE_DT_F16)
+    return launch<MOE_EPI_NONE, __half>(A, packed, absmax, offsets, E, N, K, M_total, out,
+                                        dev_err, s);
+  if (out_dt == MOE_DT_BF16)
+    return launch<MOE_EPI_NONE, __nv_bfloat16>(A, packed, absmax, offsets, E, N, K, M_total,
+                                               out, dev_err, s);
+  return launch<MOE_EPI_NONE, float>(A, packed, absmax, offsets, E, N, K, M_total, out,
+                                     dev_err, s);
 }
 
 }  // namespace moe_launch

@@ -180,8 +180,13 @@ moe_status_t moe_route_permute(const float* logits, int T, int E, int k,
  *                    outputs (gate rows) and u the last N/2 (up rows)
  *   out_dtype F32, BF16 or F16 (rounded once from the fp32 accumulator)
  *   algo     MOE_ALGO_AUTO / _GEMV / _TC
- * Accumulation is fp32; weights enter the tensor cores as fp16 (the exact
- * fp16 rounding of each level, or of level*absmax), activations as fp16.
+ * Accumulation is fp32; activations enter the tensor cores as fp16.
+ * GEMV kernel: weights enter as the fp16 rounding of each level, the fp32
+ * absmax multiplies each 64-element block's fp32 partial sum.
+ * TC kernel (tcgen05): weights enter as fp16(fp16(level) * fp16(absmax));
+ * it needs gather == NULL and F16 A (rows already permuted, e.g. by
+ * moe_permute_rows), N % 128 == 0, absmax < 65504.  AUTO uses it when those
+ * hold and M_total >= 16 * E.
  * All pointers 16-byte aligned.
  */
 moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype,
@@ -192,6 +197,21 @@ moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype,
                                   void* out, moe_dtype_t out_dtype,
                                   moe_algo_t algo, int32_t* dev_err,
                                   void* stream);
+
+/*
+ * moe_permute_rows -- gathers the routed activation rows into permuted
+ * order, converted to fp16: Xp[p, :] = fp16(X[sorted_rows[p] / k, :]) for
+ * p < M_total.  This is the activation side of the permutation (the
+ * permuted rows one grouped launch reads as contiguous per-expert
+ * segments, "grouped-nf4-gemm & experts-4bit", first bullet); the tensor-core
+ * grouped GEMM reads its activations this way, through TMA.
+ *   X   [T, K] BF16 or F16; sorted_rows int32 [M_total]; Xp fp16 [M_total, K]
+ *   K % 8 == 0; ids with f < 0, f >= M_total or f / k >= T give zero rows
+ *   and MOE_DEVERR_BAD_INDEX.  Pointers 16-byte aligned.
+ */
+moe_status_t moe_permute_rows(const void* X, moe_dtype_t x_dtype, int T, int K,
+                              const int32_t* sorted_rows, int k, int M_total,
+                              void* Xp, int32_t* dev_err, void* stream);
 
 /*
  * moe_swiglu -- standalone h[m, i] = silu(gu[m, i]) * gu[m, I + i],
@@ -220,7 +240,8 @@ moe_status_t moe_unpermute_combine(const void* Yp, moe_dtype_t yp_dtype,
  *   X bf16 [T, H]; logits fp32 [T, E]; gate_up stack [E, 2I, H];
  *   down stack [E, H, I]; Y fp32 [T, H].
  *   workspace: moe_layer_workspace_size bytes; it holds the routing outputs
- *   and the fp16 intermediates [T*k, I] and [T*k, H].
+ *   and the fp16 intermediates [T*k, H] (permuted X, tensor-core path
+ *   only), [T*k, I] and [T*k, H].
  */
 moe_status_t moe_layer_workspace_size(int T, int E, int k, int H, int I,
                                       size_t* bytes);

@@ -1,0 +1,112 @@
+"""GPU parity of the tensor-core (tcgen05) grouped NF4 GEMM and of the
+activation permutation that feeds it, against the CPU oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import moe_synth
+import oracle
+from parity_util import LazyOracleStack, assert_close, gpu_stack
+
+pytestmark = pytest.mark.gpu
+
+moe = pytest.importorskip("bit_mixture_experts_route_b200")
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def test_permute_rows_exact():
+    g = torch.Generator().manual_seed(1)
+    T, K, k = 37, 320, 3
+    X = torch.randn((T, K), generator=g).to(torch.bfloat16)
+    rows = torch.randperm(T * k, generator=g).to(torch.int32)
+    Xp = torch.empty((T * k, K), dtype=torch.float16, device="cuda")
+    lib = moe.load()
+    from bit_mixture_experts_route_b200._lib import _ptr, _stream
+    st = lib.moe_permute_rows(_ptr(X.cuda()), 1, T, K, _ptr(rows.cuda()), k, T * k, _ptr(Xp),
+                              None, _stream())
+    assert st == 0
+    ref = X[rows.long() // k].to(torch.float16)   # bf16 -> fp16 is exact here
+    assert torch.equal(Xp.cpu(), ref)
+
+
+def _ragged(E, counts):
+    off = np.zeros(E + 1, dtype=np.int32)
+    off[1:] = np.cumsum(counts)
+    return off
+
+
+@pytest.mark.parametrize("epi", ["none", "swiglu"])
+@pytest.mark.parametrize("counts", [
+    [1, 0, 15, 16, 17, 300],          # partial N tiles, an empty expert, two token tiles
+    [0, 0, 513, 0, 2, 256],           # three token tiles, exact 256 tile
+])
+def test_tc_grouped_gemm_ragged(epi, counts):
+    E = len(counts)
+    counts = np.array(counts)
+    off = _ragged(E, counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(int(counts.sum()))
+    N, K = (512, 256) if epi == "swiglu" else (256, 384)
+    W = torch.randn((E, N, K), generator=g) * 0.05
+    X = (torch.randn((M, K), generator=g)).to(torch.float16)
+    p, a = moe.nf4_quantize(W.cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
+                               out_dtype=torch.float32, algo="tc", dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    pr, ar = oracle.quantize_blockwise(W.numpy())
+    ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
+    if epi == "swiglu":
+        ref = oracle.swiglu(ref)
+    assert_close(_np(out), ref, f"tc {epi}")
+
+
+def test_tc_matches_gemv_closely():
+    E, N, K = 4, 256, 512
+    counts = np.array([40, 300, 0, 97])
+    off = _ragged(E, counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(9)
+    W = torch.randn((E, N, K), generator=g) * 0.05
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    p, a = moe.nf4_quantize(W.cuda())
+    offd = torch.from_numpy(off).cuda()
+    y_tc = moe.nf4_grouped_gemm(X.cuda(), p, a, offd, M, algo="tc")
+    y_gv = moe.nf4_grouped_gemm(X.cuda(), p, a, offd, M, algo="gemv")
+    rel = (y_tc - y_gv).abs().max() / y_gv.abs().max()
+    assert rel < 5e-3
+
+
+def test_tc_flags_bad_offsets():
+    E, N, K = 2, 128, 64
+    p = torch.zeros((E, N, K // 2), dtype=torch.uint8, device="cuda")
+    a = torch.ones((E, N * K // 64), dtype=torch.float32, device="cuda")
+    X = torch.ones((8, K), dtype=torch.float16, device="cuda")
+    bad = torch.tensor([0, 9, 8], dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.nf4_grouped_gemm(X, p, a, bad, 8, algo="tc", dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & moe.DEVERR_BAD_OFFSETS
+
+
+def test_layer_qwen3_prefill_tc_sampled():
+    shape, T, seed = moe_synth.QWEN3_30B, 4096, 2
+    stack_gpu, weights = gpu_stack(shape, seed)
+    stack = LazyOracleStack.shared(stack_gpu, weights)
+    X = moe_synth.activations(T, shape.H, seed)
+    lg = moe_synth.logits(shape, T, seed)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y = moe.layer_forward(X.cuda(), lg.cuda(), shape.k, shape.renormalize, *stack_gpu,
+                          dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rng = np.random.default_rng(1)
+    toks = sorted(rng.choice(T, size=48, replace=False).tolist())
+    ref = oracle.moe_layer(X.float().numpy(), lg.numpy(), stack, shape.k, shape.renormalize,
+                           tokens=toks)
+    assert_close(_np(Y)[toks], ref, "qwen3 prefill (tensor cores)")
