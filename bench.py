@@ -187,6 +187,7 @@ class Workload:
         }
         self.rws = torch.empty((max(moe.route_permute_workspace_size(T, E, k), 256),),
                                dtype=torch.uint8, device=dev)
+        self.Xp = torch.empty((M, H), dtype=torch.float16, device=dev)
         self.Hbuf = torch.empty((M, I), dtype=torch.float16, device=dev)
         self.Yp = torch.empty((M, H), dtype=torch.float16, device=dev)
         self.Y = torch.empty((T, H), dtype=torch.float32, device=dev)
@@ -199,10 +200,10 @@ class Workload:
         r = moe.route_permute(self.logits[layer], sh.k, sh.renormalize, workspace=self.rws,
                               out=self.route)
         M = T * sh.k
+        moe.permute_rows(self.X, r["sorted_rows"], sh.k, out=self.Xp)
         if ev is not None:
             ev[0].record()
-        moe.nf4_grouped_gemm(self.X, p_gu, a_gu, r["expert_offsets"], M,
-                             gather=r["sorted_rows"], k=sh.k, epilogue="swiglu",
+        moe.nf4_grouped_gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, epilogue="swiglu",
                              out=self.Hbuf, algo=algo)
         if ev is not None:
             ev[1].record()
@@ -454,7 +455,7 @@ def main():
                          f"per-token fp64 expert MLPs); host cpu_count={ncpu}, "
                          f"affinity={aff}; {dt:.1f} s"}
 
-    launches_per_layer = 5  # route_tile, permute_scatter, gate_up, down, combine
+    launches_per_layer = 6  # route_tile, permute_scatter, permute_rows, gate_up, down, combine
     line = {
         "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

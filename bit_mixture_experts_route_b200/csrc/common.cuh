@@ -138,8 +138,7 @@ cudaError_t grouped_gemm_gemv(const void* A, moe_dtype_t a_dt, int A_rows,
                               moe_dtype_t out_dt, int32_t* dev_err,
                               cudaStream_t s);
 bool grouped_gemm_decode_supported(int N, int K);
-cudaError_t grouped_gemm_decode(const void* A, moe_dtype_t a_dt, int A_rows,
-                                const int32_t* gather, int k, const uint8_t* packed,
+cudaError_t grouped_gemm_decode(const void* A, int A_rows, const uint8_t* packed,
                                 const float* absmax, const int32_t* offsets, int E, int N,
                                 int K, int M_total, moe_epilogue_t epi, void* out,
                                 moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);

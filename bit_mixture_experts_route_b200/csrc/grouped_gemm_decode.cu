@@ -7,13 +7,15 @@
 // streaming the NF4 bytes of every expert that received a token, so the
 // design goal is to keep enough bytes in flight to saturate HBM:
 //
-// * Persistent CTAs (two per SM) walk a list of work items built on the
-//   device from expert_offsets: (expert, 64 weight rows, up to 32 routed rows).
-// * One producer thread streams each item's packed rows through an 8-stage
-//   ring with TMA tile loads (64 rows x 128 bytes = 256 k per stage, 128-byte
-//   swizzle so the consumers' reads are conflict-free) plus the matching
-//   absmax tile; ~72 KB per CTA in flight, independent of registers.
-// * Four consumer warps each own 16 weight rows: per 64-k block a lane reads
+// * Persistent CTAs (one per SM) walk a list of work items built on the
+//   device from expert_offsets: (expert, 128 weight rows, up to 32 routed
+//   rows).
+// * One producer thread streams each item through a 5-stage ring with TMA
+//   tile loads, 256 k per stage: the packed rows (128 x 128 bytes), their
+//   absmax (128 x 4 fp32) and the routed activation rows (fp16, 8-row boxes
+//   of 64 k); 128-byte swizzle keeps the consumers' shared reads
+//   conflict-free.  Up to ~170 KB in flight per SM, independent of registers.
+// * Eight consumer warps each own 16 weight rows: per 64-k block a lane reads
 //   8 packed bytes of two rows, maps each byte to an fp16 pair {L[hi], L[lo]}
 //   with one lookup in a per-lane replicated table, and issues
 //   mma.sync.m16n8k16 with the routed rows as the N side (swap-AB); the
@@ -26,18 +28,21 @@
 namespace moe {
 namespace dec {
 
-constexpr int ROWS = 64;        // weight rows per item
+constexpr int ROWS = 128;       // weight rows per item
 constexpr int TOK = 32;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int SB = SK / 2;      // packed bytes per row per stage
-constexpr int STAGES = 8;
-constexpr int CWARPS = 4;
+constexpr int STAGES = 5;
+constexpr int CWARPS = 8;
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
-constexpr uint32_t kStageBytes = ROWS * SB + ROWS * 4 * 4;
+constexpr uint32_t kWBytes = ROWS * SB + ROWS * 4 * 4;   // packed + absmax per stage
+constexpr int XBOX = 8 * 64 * 2;                         // one 8-row x 64-k fp16 box
+constexpr int XKBOX = (TOK / 8) * XBOX;                  // 32 rows x 64 k
 
 struct __align__(8) Smem {
   uint8_t w[STAGES][ROWS * SB];  // 1024-aligned (struct placed at 1024)
+  uint8_t x[STAGES][4 * XKBOX];  // [64-k block][32 rows][128 B], swizzled
   float a[STAGES][ROWS * 4];
   uint32_t lut[256 * 32];
   uint64_t full[STAGES], empty[STAGES];
@@ -101,20 +106,16 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// 16 activations A[row][k0 .. k0+16) as 8 fp16 pairs.
-template <typename AT>
-__device__ __forceinline__ void load_x16(const AT* __restrict__ p, uint32_t (&xf)[8]) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-  const uint4 u = __ldg(q), v = __ldg(q + 1);
-  if constexpr (std::is_same<AT, __half>::value) {
-    xf[0] = u.x; xf[1] = u.y; xf[2] = u.z; xf[3] = u.w;
-    xf[4] = v.x; xf[5] = v.y; xf[6] = v.z; xf[7] = v.w;
-  } else {
-    xf[0] = bf16x2_to_f16x2(u.x); xf[1] = bf16x2_to_f16x2(u.y);
-    xf[2] = bf16x2_to_f16x2(u.z); xf[3] = bf16x2_to_f16x2(u.w);
-    xf[4] = bf16x2_to_f16x2(v.x); xf[5] = bf16x2_to_f16x2(v.y);
-    xf[6] = bf16x2_to_f16x2(v.z); xf[7] = bf16x2_to_f16x2(v.w);
-  }
+// This lane's 16 activations of routed row `r` (0..31) in 64-k block `b` of
+// a stage, as 8 fp16 pairs: bytes [32t, 32t + 32) of the row's swizzled
+// 128-byte line.
+__device__ __forceinline__ void lds_x16(const uint8_t* xs, int b, int r, int t,
+                                        uint32_t (&xf)[8]) {
+  const uint8_t* line = xs + b * XKBOX + r * 128;
+  const uint4 u = *reinterpret_cast<const uint4*>(line + (((2 * t) ^ (r & 7)) << 4));
+  const uint4 v = *reinterpret_cast<const uint4*>(line + (((2 * t + 1) ^ (r & 7)) << 4));
+  xf[0] = u.x; xf[1] = u.y; xf[2] = u.z; xf[3] = u.w;
+  xf[4] = v.x; xf[5] = v.y; xf[6] = v.z; xf[7] = v.w;
 }
 
 struct Item {
@@ -140,39 +141,14 @@ __device__ __forceinline__ Item item_info(const Smem& sm, const int32_t* offsets
 }
 
 // One item's main loop and epilogue for one consumer warp, NT8 token tiles.
-template <typename AT, int EPI, typename OutT, int NT8>
-__device__ __forceinline__ bool consume_item(
-    Smem& sm, const Item& it, const AT* __restrict__ A, int A_rows,
-    const int32_t* __restrict__ gather, int k, int N, int K, int M_total, OutT* __restrict__ out,
-    int32_t* dev_err, int& stage, uint32_t& phase) {
+template <int EPI, typename OutT, int NT8>
+__device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, int K,
+                                             OutT* __restrict__ out, int32_t* dev_err,
+                                             int& stage, uint32_t& phase) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + g : 16 * warp + g;
-  const int rB = (EPI == MOE_EPI_SWIGLU) ? 32 + 8 * warp + g : 16 * warp + g + 8;
-
-  const AT* xrow[NT8];
-  bool xok[NT8];
-#pragma unroll
-  for (int j = 0; j < NT8; ++j) {
-    const int tok = 8 * j + g;
-    xok[j] = tok < it.cnt;
-    int r = 0;
-    if (xok[j]) {
-      const int p = it.start + tok;
-      if (gather) {
-        const int f = gather[p];
-        if (f < 0 || f >= M_total || f / k >= A_rows) {
-          set_dev_err(dev_err, MOE_DEVERR_BAD_INDEX);
-          xok[j] = false;
-        } else {
-          r = f / k;
-        }
-      } else {
-        r = p;
-      }
-    }
-    xrow[j] = A + (size_t)r * K + 16 * t;
-  }
+  const int rB = (EPI == MOE_EPI_SWIGLU) ? ROWS / 2 + 8 * warp + g : 16 * warp + g + 8;
 
   float acc[NT8][4];
 #pragma unroll
@@ -185,6 +161,7 @@ __device__ __forceinline__ bool consume_item(
   for (int s = 0; s < KS; ++s) {
     if (!mbar_wait(&sm.full[stage], phase, sm, dev_err)) return false;
     const uint8_t* wst = sm.w[stage];
+    const uint8_t* xst = sm.x[stage];
     const float4 sa = *reinterpret_cast<const float4*>(&sm.a[stage][rA * 4]);
     const float4 sb = *reinterpret_cast<const float4*>(&sm.a[stage][rB * 4]);
     const float sav[4] = {sa.x, sa.y, sa.z, sa.w};
@@ -193,14 +170,7 @@ __device__ __forceinline__ bool consume_item(
     for (int b = 0; b < 4; ++b) {
       uint32_t xf[NT8][8];
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) {
-        if (xok[j]) {
-          load_x16<AT>(xrow[j] + (size_t)(s * SK + b * kBlock), xf[j]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) xf[j][q] = 0u;
-        }
-      }
+      for (int j = 0; j < NT8; ++j) lds_x16(xst, b, 8 * j + g, t, xf[j]);
       // byte offset of this lane's 8 bytes in the row, 128-byte swizzled
       const int off = b * 32 + 8 * t;
       const uint2 wa = *reinterpret_cast<const uint2*>(
@@ -260,12 +230,11 @@ __device__ __forceinline__ bool consume_item(
   return true;
 }
 
-template <typename AT, int EPI, typename OutT>
-__global__ void __launch_bounds__(THREADS, 2) nf4_decode_kernel(
+template <int EPI, typename OutT>
+__global__ void __maxnreg__(224) nf4_decode_kernel(
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
-    const AT* __restrict__ A, int A_rows, const int32_t* __restrict__ gather, int k,
-    const int32_t* __restrict__ offsets, int E, int N, int K, int M_total,
-    OutT* __restrict__ out, int32_t* dev_err) {
+    const __grid_constant__ CUtensorMap xmap, const int32_t* __restrict__ offsets, int E, int N,
+    int K, int M_total, OutT* __restrict__ out, int32_t* dev_err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -334,13 +303,18 @@ __global__ void __launch_bounds__(THREADS, 2) nf4_decode_kernel(
           y0 = it.expert * N + it.rtile * ROWS;
           y1 = y0 + ROWS / 2;
         }
+        const int nr8 = (it.cnt + 7) / 8;
         for (int s = 0; s < KS; ++s) {
           if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
-          mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+          mbar_arrive_expect_tx(&sm.full[stage], kWBytes + nr8 * 4 * XBOX);
           tma_load_2d(sm.w[stage], &wmap, &sm.full[stage], s * SB, y0);
           tma_load_2d(sm.w[stage] + (ROWS / 2) * SB, &wmap, &sm.full[stage], s * SB, y1);
           tma_load_2d(sm.a[stage], &amap, &sm.full[stage], s * 4, y0);
           tma_load_2d(sm.a[stage] + (ROWS / 2) * 4, &amap, &sm.full[stage], s * 4, y1);
+          for (int b = 0; b < 4; ++b)
+            for (int r = 0; r < nr8; ++r)
+              tma_load_2d(sm.x[stage] + b * XKBOX + r * XBOX, &xmap, &sm.full[stage],
+                          s * SK + b * kBlock, it.start + 8 * r);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -353,17 +327,13 @@ __global__ void __launch_bounds__(THREADS, 2) nf4_decode_kernel(
       const Item it = item_info(sm, offsets, E, rtiles, i);
       bool ok;
       if (it.cnt > 24)
-        ok = consume_item<AT, EPI, OutT, 4>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
-                                            dev_err, stage, phase);
+        ok = consume_item<EPI, OutT, 4>(sm, it, N, K, out, dev_err, stage, phase);
       else if (it.cnt > 16)
-        ok = consume_item<AT, EPI, OutT, 3>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
-                                            dev_err, stage, phase);
+        ok = consume_item<EPI, OutT, 3>(sm, it, N, K, out, dev_err, stage, phase);
       else if (it.cnt > 8)
-        ok = consume_item<AT, EPI, OutT, 2>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
-                                            dev_err, stage, phase);
+        ok = consume_item<EPI, OutT, 2>(sm, it, N, K, out, dev_err, stage, phase);
       else
-        ok = consume_item<AT, EPI, OutT, 1>(sm, it, A, A_rows, gather, k, N, K, M_total, out,
-                                            dev_err, stage, phase);
+        ok = consume_item<EPI, OutT, 1>(sm, it, N, K, out, dev_err, stage, phase);
       if (!ok) break;
     }
   }
@@ -377,13 +347,13 @@ int sm_count() {
   return sms;
 }
 
-template <typename AT, int EPI, typename OutT>
-cudaError_t launch(const void* A, int A_rows, const int32_t* gather, int k,
-                   const uint8_t* packed, const float* absmax, const int32_t* offsets, int E,
-                   int N, int K, int M_total, void* out, int32_t* dev_err, cudaStream_t s) {
+template <int EPI, typename OutT>
+cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
+                   const int32_t* offsets, int E, int N, int K, int M_total, void* out,
+                   int32_t* dev_err, cudaStream_t s) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap wmap, amap;
+  CUtensorMap wmap, amap, xmap;
   const cuuint32_t estr[2] = {1, 1};
   {
     const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)E * N};
@@ -404,32 +374,40 @@ cudaError_t launch(const void* A, int A_rows, const int32_t* gather, int k,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)A_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {kBlock, 8};
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   const size_t smem = sizeof(Smem) + 1024;
-  auto kern = nf4_decode_kernel<AT, EPI, OutT>;
+  auto kern = nf4_decode_kernel<EPI, OutT>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int64_t max_items = ((int64_t)M_total / TOK + E) * (N / ROWS);
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(2 * sm_count(), max_items));
-  kern<<<grid, THREADS, smem, s>>>(wmap, amap, reinterpret_cast<const AT*>(A), A_rows, gather, k,
-                                   offsets, E, N, K, M_total, reinterpret_cast<OutT*>(out),
-                                   dev_err);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_items));
+  kern<<<grid, THREADS, smem, s>>>(wmap, amap, xmap, offsets, E, N, K, M_total,
+                                   reinterpret_cast<OutT*>(out), dev_err);
   return cudaGetLastError();
 }
 
-template <typename AT, int EPI>
-cudaError_t launch_out(const void* A, int A_rows, const int32_t* gather, int k,
-                       const uint8_t* packed, const float* absmax, const int32_t* offsets, int E,
-                       int N, int K, int M_total, void* out, moe_dtype_t out_dt,
-                       int32_t* dev_err, cudaStream_t s) {
+template <int EPI>
+cudaError_t launch_out(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
+                       const int32_t* offsets, int E, int N, int K, int M_total, void* out,
+                       moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s) {
   if (out_dt == MOE_DT_F32)
-    return launch<AT, EPI, float>(A, A_rows, gather, k, packed, absmax, offsets, E, N, K,
-                                  M_total, out, dev_err, s);
+    return launch<EPI, float>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
+                              dev_err, s);
   if (out_dt == MOE_DT_F16)
-    return launch<AT, EPI, __half>(A, A_rows, gather, k, packed, absmax, offsets, E, N, K,
-                                   M_total, out, dev_err, s);
-  return launch<AT, EPI, __nv_bfloat16>(A, A_rows, gather, k, packed, absmax, offsets, E, N, K,
-                                        M_total, out, dev_err, s);
+    return launch<EPI, __half>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
+                               dev_err, s);
+  return launch<EPI, __nv_bfloat16>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
+                                    dev_err, s);
 }
 
 }  // namespace dec
@@ -442,26 +420,17 @@ bool grouped_gemm_decode_supported(int N, int K) {
   return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
 }
 
-cudaError_t grouped_gemm_decode(const void* A, moe_dtype_t a_dt, int A_rows,
-                                const int32_t* gather, int k, const uint8_t* packed,
+// Activations must be fp16 rows in permuted order (no gather).
+cudaError_t grouped_gemm_decode(const void* A, int A_rows, const uint8_t* packed,
                                 const float* absmax, const int32_t* offsets, int E, int N, int K,
                                 int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
                                 int32_t* dev_err, cudaStream_t s) {
   using namespace moe::dec;
-  if (a_dt == MOE_DT_BF16) {
-    return epi == MOE_EPI_SWIGLU
-               ? launch_out<__nv_bfloat16, MOE_EPI_SWIGLU>(A, A_rows, gather, k, packed, absmax,
-                                                           offsets, E, N, K, M_total, out,
-                                                           out_dt, dev_err, s)
-               : launch_out<__nv_bfloat16, MOE_EPI_NONE>(A, A_rows, gather, k, packed, absmax,
-                                                         offsets, E, N, K, M_total, out, out_dt,
-                                                         dev_err, s);
-  }
   return epi == MOE_EPI_SWIGLU
-             ? launch_out<__half, MOE_EPI_SWIGLU>(A, A_rows, gather, k, packed, absmax, offsets,
-                                                  E, N, K, M_total, out, out_dt, dev_err, s)
-             : launch_out<__half, MOE_EPI_NONE>(A, A_rows, gather, k, packed, absmax, offsets, E,
-                                                N, K, M_total, out, out_dt, dev_err, s);
+             ? launch_out<MOE_EPI_SWIGLU>(A, A_rows, packed, absmax, offsets, E, N, K, M_total,
+                                          out, out_dt, dev_err, s)
+             : launch_out<MOE_EPI_NONE>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
+                                        out_dt, dev_err, s);
 }
 
 }  // namespace moe_launch

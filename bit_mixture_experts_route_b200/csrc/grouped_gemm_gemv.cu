@@ -1,6 +1,7 @@
 // Grouped NF4 GEMM, decode path, general-shape kernel (few routed rows per
-// expert; HBM-bound).  Shapes with K % 256 == 0 go to the TMA-staged kernel in
-// grouped_gemm_decode.cu; this one covers the rest with direct loads.
+// expert; HBM-bound).  Permuted fp16 activations with K % 256 == 0 go to the
+// TMA-staged kernel in grouped_gemm_decode.cu; this one covers the rest
+// (gathered or bf16 activations, other K) with direct loads.
 //
 // "grouped-nf4-gemm & experts-4bit" (jordananderson-pages.pages.dev), first
 // bullet: one launch for all active experts, the 16-entry codebook decoded in
@@ -283,9 +284,9 @@ cudaError_t grouped_gemm_gemv(const void* A, moe_dtype_t a_dt, int A_rows, const
                               moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
                               int32_t* dev_err, cudaStream_t s) {
   if (M_total == 0) return cudaSuccess;
-  if (grouped_gemm_decode_supported(N, K))
-    return grouped_gemm_decode(A, a_dt, A_rows, gather, k, packed, absmax, offsets, E, N, K,
-                               M_total, epi, out, out_dt, dev_err, s);
+  if (!gather && a_dt == MOE_DT_F16 && grouped_gemm_decode_supported(N, K))
+    return grouped_gemm_decode(A, A_rows, packed, absmax, offsets, E, N, K, M_total, epi, out,
+                               out_dt, dev_err, s);
   using namespace moe;
   if (a_dt == MOE_DT_BF16) {
     return epi == MOE_EPI_SWIGLU

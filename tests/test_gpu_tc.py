@@ -23,14 +23,15 @@ def test_permute_rows_exact():
     T, K, k = 37, 320, 3
     X = torch.randn((T, K), generator=g).to(torch.bfloat16)
     rows = torch.randperm(T * k, generator=g).to(torch.int32)
-    Xp = torch.empty((T * k, K), dtype=torch.float16, device="cuda")
-    lib = moe.load()
-    from bit_mixture_experts_route_b200._lib import _ptr, _stream
-    st = lib.moe_permute_rows(_ptr(X.cuda()), 1, T, K, _ptr(rows.cuda()), k, T * k, _ptr(Xp),
-                              None, _stream())
-    assert st == 0
+    Xp = moe.permute_rows(X.cuda(), rows.cuda(), k)
     ref = X[rows.long() // k].to(torch.float16)   # bf16 -> fp16 is exact here
     assert torch.equal(Xp.cpu(), ref)
+    bad = rows.clone()
+    bad[5] = T * k + 3
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Xb = moe.permute_rows(X.cuda(), bad.cuda(), k, dev_err=err)
+    assert int(err.item()) & moe.DEVERR_BAD_INDEX
+    assert torch.all(Xb[5] == 0)
 
 
 def _ragged(E, counts):
