@@ -30,6 +30,7 @@ _P, _I, _Z, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
 SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_abi_version": (_I, []),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_nf4_levels": (_I, [_P]),
     "moe_nf4_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _S]),
     "moe_nf4_dequantize": (_I, [_P, _P, _I, _I, _I, _P, _I, _S]),
@@ -70,7 +71,10 @@ def load() -> ctypes.CDLL:
 
 def _check(status: int, what: str):
     if status != MOE_OK:
-        raise MoEError(f"{what}: {STATUS.get(status, status)}")
+        detail = ""
+        if status == 5:
+            detail = f" ({load().moe_last_cuda_error().decode()})"
+        raise MoEError(f"{what}: {STATUS.get(status, status)}{detail}")
 
 
 def _ptr(t):

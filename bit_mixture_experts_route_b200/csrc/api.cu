@@ -18,7 +18,14 @@ moe_status_t check_device() {
   return (major == 10 && minor == 0) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
-moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+// The CUDA error behind the calling thread's most recent MOE_ERR_CUDA.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+moe_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  t_last_cuda_error = e;
+  return MOE_ERR_CUDA;
+}
 
 bool valid_dtype(moe_dtype_t d) { return d == MOE_DT_F32 || d == MOE_DT_BF16 || d == MOE_DT_F16; }
 
@@ -41,6 +48,10 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 int moe_abi_version(void) { return MOE_NF4_ABI_VERSION; }
+
+const char* moe_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
 
 moe_status_t moe_nf4_levels(float* levels_out) {
   if (!levels_out) return MOE_ERR_INVALID_ARG;

@@ -8,13 +8,13 @@
 // design goal is to keep enough bytes in flight to saturate HBM:
 //
 // * Persistent CTAs (one per SM) walk a list of work items built on the
-//   device from expert_offsets: (expert, 128 weight rows, up to 32 routed
-//   rows).
-// * One producer thread streams each item through a 5-stage ring with TMA
+//   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
+//   rows; an expert with more routed rows yields one item per 16).
+// * One producer thread streams each item through a 6-stage ring with TMA
 //   tile loads, 256 k per stage: the packed rows (128 x 128 bytes), their
 //   absmax (128 x 4 fp32) and the routed activation rows (fp16, 8-row boxes
 //   of 64 k); 128-byte swizzle keeps the consumers' shared reads
-//   conflict-free.  Up to ~170 KB in flight per SM, independent of registers.
+//   conflict-free.  Up to ~150 KB in flight per SM, independent of registers.
 // * Eight consumer warps each own 16 weight rows: per 64-k block a lane reads
 //   8 packed bytes of two rows, maps each byte to an fp16 pair {L[hi], L[lo]}
 //   with one lookup in a per-lane replicated table, and issues
@@ -29,20 +29,20 @@ namespace moe {
 namespace dec {
 
 constexpr int ROWS = 128;       // weight rows per item
-constexpr int TOK = 32;         // routed rows per item (max)
+constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int SB = SK / 2;      // packed bytes per row per stage
-constexpr int STAGES = 5;
+constexpr int STAGES = 6;
 constexpr int CWARPS = 8;
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr uint32_t kWBytes = ROWS * SB + ROWS * 4 * 4;   // packed + absmax per stage
 constexpr int XBOX = 8 * 64 * 2;                         // one 8-row x 64-k fp16 box
-constexpr int XKBOX = (TOK / 8) * XBOX;                  // 32 rows x 64 k
+constexpr int XKBOX = (TOK / 8) * XBOX;                  // 16 rows x 64 k
 
 struct __align__(8) Smem {
   uint8_t w[STAGES][ROWS * SB];  // 1024-aligned (struct placed at 1024)
-  uint8_t x[STAGES][4 * XKBOX];  // [64-k block][32 rows][128 B], swizzled
+  uint8_t x[STAGES][4 * XKBOX];  // [64-k block][16 rows][128 B], swizzled
   float a[STAGES][ROWS * 4];
   uint32_t lut[256 * 32];
   uint64_t full[STAGES], empty[STAGES];
@@ -106,7 +106,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// This lane's 16 activations of routed row `r` (0..31) in 64-k block `b` of
+// This lane's 16 activations of routed row `r` (0..15) in 64-k block `b` of
 // a stage, as 8 fp16 pairs: bytes [32t, 32t + 32) of the row's swizzled
 // 128-byte line.
 __device__ __forceinline__ void lds_x16(const uint8_t* xs, int b, int r, int t,
@@ -231,7 +231,7 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
 }
 
 template <int EPI, typename OutT>
-__global__ void __maxnreg__(224) nf4_decode_kernel(
+__global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
     const __grid_constant__ CUtensorMap xmap, const int32_t* __restrict__ offsets, int E, int N,
     int K, int M_total, OutT* __restrict__ out, int32_t* dev_err) {
@@ -326,11 +326,7 @@ __global__ void __maxnreg__(224) nf4_decode_kernel(
     for (int i = blockIdx.x; i < total; i += gridDim.x) {
       const Item it = item_info(sm, offsets, E, rtiles, i);
       bool ok;
-      if (it.cnt > 24)
-        ok = consume_item<EPI, OutT, 4>(sm, it, N, K, out, dev_err, stage, phase);
-      else if (it.cnt > 16)
-        ok = consume_item<EPI, OutT, 3>(sm, it, N, K, out, dev_err, stage, phase);
-      else if (it.cnt > 8)
+      if (it.cnt > 8)
         ok = consume_item<EPI, OutT, 2>(sm, it, N, K, out, dev_err, stage, phase);
       else
         ok = consume_item<EPI, OutT, 1>(sm, it, N, K, out, dev_err, stage, phase);

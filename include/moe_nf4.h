@@ -85,6 +85,10 @@ const char* moe_status_string(moe_status_t status);
 /* MOE_NF4_ABI_VERSION of the loaded library. */
 int moe_abi_version(void);
 
+/* Text of the CUDA error behind the calling host thread's most recent
+ * MOE_ERR_CUDA ("no error" if none); a static string, never NULL. */
+const char* moe_last_cuda_error(void);
+
 /* Copies the library's 16 NF4 levels (fp32, ascending, code c -> level c)
  * into HOST memory `levels_out[16]`.  Host-only, no CUDA call. */
 moe_status_t moe_nf4_levels(float* levels_out);
