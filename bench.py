@@ -146,12 +146,19 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host float over all ranks (on the process group's device)."""
     if world <= 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(seed, rank):
+    """Each replica draws its own token batch and weights (weak scaling)."""
+    return seed + 7919 * rank
 
 
 # ----------------------------------------------------------------- workload
@@ -335,7 +342,7 @@ def main():
     world, rank, local = dist_setup()
     import bit_mixture_experts_route_b200 as moe
     moe.load()
-    wl = Workload(shape, T, layers, args.seed + rank)
+    wl = Workload(shape, T, layers, rank_seed(args.seed, rank))
     hbm, tf_burst, tf_sust, peak_kind = load_peaks()
     stream = torch.cuda.current_stream()
 

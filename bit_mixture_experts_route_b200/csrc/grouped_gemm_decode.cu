@@ -186,12 +186,13 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
       for (int i = 0; i < 4; ++i) {
         const uint32_t vA = (i < 2) ? wa.x : wa.y;
         const uint32_t vB = (i < 2) ? wb.x : wb.y;
-        const int sh = (i & 1) * 16;
+        const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
+        // byte -> table entry (byte * 32 + lane): one byte_perm and one shift-add
         uint32_t af[4];
-        af[0] = lut[((vA >> sh) & 0xffu) << 5];
-        af[1] = lut[((vB >> sh) & 0xffu) << 5];
-        af[2] = lut[((vA >> (sh + 8)) & 0xffu) << 5];
-        af[3] = lut[((vB >> (sh + 8)) & 0xffu) << 5];
+        af[0] = lut[__byte_perm(vA, 0, 0x4440u | lo) << 5];
+        af[1] = lut[__byte_perm(vB, 0, 0x4440u | lo) << 5];
+        af[2] = lut[__byte_perm(vA, 0, 0x4440u | (lo + 1)) << 5];
+        af[3] = lut[__byte_perm(vB, 0, 0x4440u | (lo + 1)) << 5];
 #pragma unroll
         for (int j = 0; j < NT8; ++j) mma_16816(tmp[j], af, xf[j][2 * i], xf[j][2 * i + 1]);
       }

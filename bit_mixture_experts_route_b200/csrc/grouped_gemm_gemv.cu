@@ -151,12 +151,12 @@ __device__ __forceinline__ void gemv_chunk(
         // bytes 2i and 2i+1 of this lane's 8 bytes of each row
         const uint32_t wA = (i < 2) ? wa[u].x : wa[u].y;
         const uint32_t wB = (i < 2) ? wb[u].x : wb[u].y;
-        const int sh = (i & 1) * 16;
+        const uint32_t lo = (i & 1) * 2;
         uint32_t a[4];
-        a[0] = lut[((wA >> sh) & 0xffu) * 32 + lane];
-        a[1] = lut[((wB >> sh) & 0xffu) * 32 + lane];
-        a[2] = lut[((wA >> (sh + 8)) & 0xffu) * 32 + lane];
-        a[3] = lut[((wB >> (sh + 8)) & 0xffu) * 32 + lane];
+        a[0] = lut[__byte_perm(wA, 0, 0x4440u | lo) * 32 + lane];
+        a[1] = lut[__byte_perm(wB, 0, 0x4440u | lo) * 32 + lane];
+        a[2] = lut[__byte_perm(wA, 0, 0x4440u | (lo + 1)) * 32 + lane];
+        a[3] = lut[__byte_perm(wB, 0, 0x4440u | (lo + 1)) * 32 + lane];
 #pragma unroll
         for (int j = 0; j < NT8; ++j) mma_f16_16816(tmp[j], a, xf[j][2 * i], xf[j][2 * i + 1]);
       }

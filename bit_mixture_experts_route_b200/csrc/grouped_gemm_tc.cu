@@ -14,18 +14,21 @@
 //
 // Persistent CTAs walk a tile list built on the device from expert_offsets
 // (expert-major, then token tile, then weight-row tile), so no host sync is
-// needed.  Warp roles (320 threads):
-//   warp 0     TMA producer: activation tiles [256 rows x 64 k] (fp16,
-//              128-byte swizzle) into a 3-stage ring
-//   warp 1     TMEM allocator and MMA issuer (one thread):
-//              tcgen05.mma.cta_group::1.kind::f16, 4 x K16 per stage
-//   warps 2-5  decoders, one thread per weight row: 32 packed bytes and one
-//              fp32 absmax per 64-k step, each byte -> fp16 pair {L[hi],
-//              L[lo]} through a per-lane shared table, times fp16(absmax),
-//              stored in the same 128-byte-swizzled K-major layout
-//   warps 6-9  epilogue: tcgen05.ld 32 columns at a time, SwiGLU (gate and
-//              up rows interleaved in the tile, paired with one shuffle) or a
-//              plain store, then release the accumulator.
+// needed.  Warp roles (480 threads):
+//   warp 0      TMA producer: activation tiles [256 rows x 64 k] (fp16,
+//               128-byte swizzle) into a 3-stage ring
+//   warp 1      TMEM allocator and MMA issuer (one thread):
+//               tcgen05.mma.cta_group::1.kind::f16, 4 x K16 per stage
+//   warp 2      TMA producer: the tile's packed NF4 rows [128 rows x 32 B]
+//               per 64-k step into an 8-stage ring
+//   warps 3-10  decoders, two threads per weight row (32 k each): packed
+//               bytes from the ring, absmax prefetched 8 steps ahead, each
+//               byte -> fp16 pair {L[hi], L[lo]} through a per-lane shared
+//               table, times fp16(absmax), stored in the 128-byte-swizzled
+//               K-major layout the MMA reads
+//   warps 11-14 epilogue: tcgen05.ld 32 columns at a time, SwiGLU (gate and
+//               up rows interleaved in the tile, paired with one shuffle) or a
+//               plain store, then release the accumulator.
 // Every mbarrier wait is bounded; on expiry the kernel sets
 // MOE_DEVERR_TIMEOUT, every role leaves its loop, TMEM is freed and the
 // kernel returns.
@@ -41,15 +44,21 @@ constexpr int STAGES = 3;
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BN * BK * 2;   // 32 KB
 constexpr int B_BOX_ROWS = 128;        // TMA box: 64 k x 128 rows
-constexpr int THREADS = 320;
+constexpr int RSTAGES = 8;             // raw NF4 ring: 128 rows x 32 bytes each
+constexpr int RAW_STAGE = BM * BK / 2;
+constexpr int DEC_WARPS = 8;           // two threads per weight row
+constexpr int W_BPROD = 0, W_MMA = 1, W_RPROD = 2, W_DEC = 3, W_EPI = W_DEC + DEC_WARPS;
+constexpr int THREADS = 32 * (W_EPI + 4);
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t kSpinLimit = 1u << 24;
 
 struct __align__(8) Smem {
   uint8_t b[STAGES][B_STAGE];  // 1024-aligned (struct placed at 1024)
   uint8_t a[STAGES][A_STAGE];
+  uint8_t raw[RSTAGES][RAW_STAGE];
   uint32_t lut[256 * 32];
   uint64_t full_a[STAGES], full_b[STAGES], empty[STAGES];
+  uint64_t raw_full[RSTAGES], raw_empty[RSTAGES];
   uint64_t acc_full[2], acc_empty[2];
   uint32_t tmem_base;
   int abort_flag;
@@ -195,7 +204,7 @@ __device__ __forceinline__ TileInfo tile_info(const Smem& sm, const int32_t* off
 
 template <int EPI, typename OutT>
 __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
-    const __grid_constant__ CUtensorMap bmap, const uint8_t* __restrict__ packed,
+    const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
     const float* __restrict__ absmax, const int32_t* __restrict__ offsets, int E, int N, int K,
     int M_total, OutT* __restrict__ out, int32_t* dev_err) {
   extern __shared__ uint8_t smem_raw[];
@@ -208,9 +217,13 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   // ---- setup: barriers, decode table, tile list, TMEM
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full_a[s], 128);
+      mbar_init(&sm.full_a[s], DEC_WARPS);
       mbar_init(&sm.full_b[s], 1);
       mbar_init(&sm.empty[s], 1);
+    }
+    for (int s = 0; s < RSTAGES; ++s) {
+      mbar_init(&sm.raw_full[s], 1);
+      mbar_init(&sm.raw_empty[s], DEC_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
@@ -225,7 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
                                      __float2half_rn(c_levels_tc[b & 15]));
     sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
   }
-  if (warp == 0) {
+  if (warp == W_BPROD) {
     // tile_prefix[e] = sum over e' < e of ceil(count / BN) * n_tiles
     bool bad = offsets[0] != 0 || offsets[E] != M_total;
     int run = 0;
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       if (bad) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
     }
   }
-  if (warp == 1) {
+  if (warp == W_MMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&sm.tmem_base)),
                  "r"(TMEM_COLS));
@@ -265,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   const uint32_t tmem_base = sm.tmem_base;
   const int total = sm.ntiles_total;
 
-  if (warp == 0) {
+  if (warp == W_BPROD) {
     // ---------------- TMA producer: activation tiles
     if (lane == 0) {
       int stage = 0;
@@ -285,7 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == W_MMA) {
     // ---------------- MMA issuer
     if (lane == 0) {
       int stage = 0;
@@ -315,12 +328,42 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         if (ok) mma_commit(&sm.acc_full[acc]);
       }
     }
-  } else if (warp < 6) {
-    // ---------------- decoders: thread m owns tile row m
-    const int m = threadIdx.x - 64;
+  } else if (warp == W_RPROD) {
+    // ---------------- TMA producer: packed NF4 rows of the tile
+    if (lane == 0) {
+      int rs = 0;
+      uint32_t rphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = tile_info(sm, offsets, E, n_tiles, t);
+        int y0, y1;  // first weight row of each 64-row box
+        if (EPI == MOE_EPI_SWIGLU) {
+          y0 = ti.expert * N + ti.ntile * (BM / 2);  // gate rows
+          y1 = y0 + N / 2;                           // matching up rows
+        } else {
+          y0 = ti.expert * N + ti.ntile * BM;
+          y1 = y0 + BM / 2;
+        }
+        for (int ks = 0; ks < KT; ++ks) {
+          if (!(ok = mbar_wait(&sm.raw_empty[rs], rphase ^ 1, sm, dev_err))) break;
+          mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE);
+          tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], ks * (BK / 2), y0);
+          tma_load_2d(sm.raw[rs] + (BM / 2) * (BK / 2), &wmap, &sm.raw_full[rs], ks * (BK / 2), y1);
+          if (++rs == RSTAGES) { rs = 0; rphase ^= 1; }
+        }
+      }
+    }
+  } else if (warp < W_EPI) {
+    // ---------------- decoders: thread pair (m, h) owns half h of tile row m
+    const int i = threadIdx.x - 32 * W_DEC;
+    const int m = i & (BM - 1), h = i >> 7;
+    // row of the raw tile holding tile row m (SwiGLU tiles interleave gate
+    // and up rows: even m = gate j, odd m = up j; the raw tile holds the 64
+    // gate rows, then the 64 up rows)
+    const int rrow = (EPI == MOE_EPI_SWIGLU) ? ((m & 1) ? BM / 2 + (m >> 1) : (m >> 1)) : m;
     const uint32_t* lut = sm.lut + lane;
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, rs = 0;
+    uint32_t phase = 0, rphase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const TileInfo ti = tile_info(sm, offsets, E, n_tiles, t);
@@ -331,45 +374,51 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       } else {
         row = ti.ntile * BM + m;
       }
-      const size_t grow = (size_t)ti.expert * N + row;
-      const uint4* wp = reinterpret_cast<const uint4*>(packed + grow * (size_t)(K / 2));
-      const float* ap = absmax + grow * (size_t)KT;
-      uint4 q0 = ldg_stream_u4(wp), q1 = ldg_stream_u4(wp + 1);
-      float a = __ldg(ap);
-      for (int ks = 0; ks < KT; ++ks) {
-        // prefetch the next 64-k step while this one is decoded
-        uint4 n0 = q0, n1 = q1;
-        float na = a;
-        if (ks + 1 < KT) {
-          n0 = ldg_stream_u4(wp + 2 * (ks + 1));
-          n1 = ldg_stream_u4(wp + 2 * (ks + 1) + 1);
-          na = __ldg(ap + ks + 1);
-        }
-        if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
-        const __half2 ah = __float2half2_rn(a);
-        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        uint8_t* arow = sm.a[stage] + (m >> 3) * 1024 + (m & 7) * 128;
+      const float* ap = absmax + ((size_t)ti.expert * N + row) * (size_t)KT;
+      float a8[8], n8[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t w = words[c];
-          uint32_t h[4];
+      for (int u = 0; u < 8; ++u) a8[u] = (u < KT) ? __ldg(ap + u) : 0.0f;
+      for (int ks0 = 0; ks0 < KT && ok; ks0 += 8) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t raw = lut[((w >> (8 * i)) & 0xffu) << 5];
-            __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&raw), ah);
-            h[i] = *reinterpret_cast<uint32_t*>(&v);
+        for (int u = 0; u < 8; ++u) n8[u] = (ks0 + 8 + u < KT) ? __ldg(ap + ks0 + 8 + u) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (ks0 + u >= KT) break;
+          if (!(ok = mbar_wait(&sm.raw_full[rs], rphase, sm, dev_err))) break;
+          const uint4 q = *reinterpret_cast<const uint4*>(sm.raw[rs] + rrow * (BK / 2) + h * 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.raw_empty[rs]);
+          if (++rs == RSTAGES) { rs = 0; rphase ^= 1; }
+          if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
+          const __half2 ah = __float2half2_rn(a8[u]);
+          const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+          uint8_t* arow = sm.a[stage] + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t w = words[c];
+            uint32_t hv[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const uint32_t raw = lut[__byte_perm(w, 0, 0x4440u | b) << 5];
+              __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&raw), ah);
+              hv[b] = *reinterpret_cast<uint32_t*>(&v);
+            }
+            const int chunk = 4 * h + c;
+            *reinterpret_cast<uint4*>(arow + ((chunk ^ (m & 7)) << 4)) =
+                make_uint4(hv[0], hv[1], hv[2], hv[3]);
           }
-          *reinterpret_cast<uint4*>(arow + ((c ^ (m & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.full_a[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
-        fence_proxy_async();
-        mbar_arrive(&sm.full_a[stage]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        q0 = n0; q1 = n1; a = na;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a8[u] = n8[u];
       }
     }
   } else {
     // ---------------- epilogue: warp q reads TMEM lanes 32q .. 32q+31
-    const int q = warp & 3;
+    const int q = warp & 3;  // four consecutive warps cover every lane quarter
     const int m = 32 * q + lane;
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     bool ok = true;
@@ -416,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == W_MMA) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(TMEM_COLS));
@@ -436,15 +485,29 @@ cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
                    int32_t* dev_err, cudaStream_t s) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M_total};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {BK, B_BOX_ROWS};
+  CUtensorMap map, wmap;
   const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box,
-          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M_total};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {BK, B_BOX_ROWS};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // packed rows as a 2-D byte tensor [E*N, K/2]; box = 32 bytes x 64 rows
+    const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)E * N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t box[2] = {BK / 2, BM / 2};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   const size_t smem = sizeof(Smem) + 1024;
   auto kern = nf4_tc_kernel<EPI, OutT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -454,7 +517,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
   // partial tile per expert; the kernel derives the exact list itself.
   const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / BM);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-  kern<<<grid, THREADS, smem, s>>>(map, packed, absmax, offsets, E, N, K, M_total,
+  kern<<<grid, THREADS, smem, s>>>(map, wmap, absmax, offsets, E, N, K, M_total,
                                    reinterpret_cast<OutT*>(out), dev_err);
   return cudaGetLastError();
 }
