@@ -334,6 +334,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
       if (!ok) break;
     }
   }
+  __syncwarp();  // the producer lane rejoins its warp before the CTA barrier
   __syncthreads();
 }
 

@@ -217,13 +217,13 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   // ---- setup: barriers, decode table, tile list, TMEM
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full_a[s], DEC_WARPS);
+      mbar_init(&sm.full_a[s], 32 * DEC_WARPS);
       mbar_init(&sm.full_b[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
     for (int s = 0; s < RSTAGES; ++s) {
       mbar_init(&sm.raw_full[s], 1);
-      mbar_init(&sm.raw_empty[s], DEC_WARPS);
+      mbar_init(&sm.raw_empty[s], 32 * DEC_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
@@ -386,9 +386,6 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
           if (ks0 + u >= KT) break;
           if (!(ok = mbar_wait(&sm.raw_full[rs], rphase, sm, dev_err))) break;
           const uint4 q = *reinterpret_cast<const uint4*>(sm.raw[rs] + rrow * (BK / 2) + h * 16);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.raw_empty[rs]);
-          if (++rs == RSTAGES) { rs = 0; rphase ^= 1; }
           if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
           const __half2 ah = __float2half2_rn(a8[u]);
           const uint32_t words[4] = {q.x, q.y, q.z, q.w};
@@ -407,10 +404,15 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
             *reinterpret_cast<uint4*>(arow + ((chunk ^ (m & 7)) << 4)) =
                 make_uint4(hv[0], hv[1], hv[2], hv[3]);
           }
+          // every writer makes its stores visible to the tensor core, then arrives
           fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.full_a[stage]);
+          mbar_arrive(&sm.full_a[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          // Release the raw slot only now that its bytes have been decoded: a
+          // release right after the shared load let the next TMA refill land
+          // before the load had read the slot.
+          mbar_arrive(&sm.raw_empty[rs]);
+          if (++rs == RSTAGES) { rs = 0; rphase ^= 1; }
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) a8[u] = n8[u];
@@ -463,6 +465,9 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     }
   }
 
+  // single-lane roles (producers, MMA issuer) rejoin their warp before the
+  // CTA-wide barrier
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == W_MMA) {
