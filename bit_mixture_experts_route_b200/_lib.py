@@ -36,6 +36,7 @@ SIGNATURES = {
     "moe_nf4_dequantize": (_I, [_P, _P, _I, _I, _I, _P, _I, _S]),
     "moe_route_permute_workspace_size": (_I, [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_route_permute": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _S]),
+    "moe_route_permute_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _S]),
     "moe_nf4_grouped_gemm": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                   _I, _I, _P, _S]),
     "moe_permute_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _S]),

@@ -110,6 +110,25 @@ moe_status_t moe_route_permute(const float* logits, int T, int E, int k, int ren
                                              workspace, (cudaStream_t)stream));
 }
 
+moe_status_t moe_route_permute_noalloc(const float* logits, int T, int E, int k,
+                                       int renormalize, int32_t* topk_idx, float* topk_w,
+                                       int32_t* expert_offsets, int32_t* sorted_rows,
+                                       int32_t* inv_perm, void* stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_idx || !topk_w || !sorted_rows || !inv_perm))
+    return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {logits, topk_idx, topk_w, expert_offsets, sorted_rows, inv_perm};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (!moe_launch::route_noalloc_fits(T, E, k)) return MOE_ERR_WORKSPACE;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(moe_launch::route_permute_noalloc(logits, T, E, k, renormalize ? 1 : 0,
+                                                     topk_idx, topk_w, expert_offsets,
+                                                     sorted_rows, inv_perm,
+                                                     (cudaStream_t)stream));
+}
+
 moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows,
                                   const int32_t* gather, int k, const uint8_t* packed, const float* absmax,
                                   const int32_t* expert_offsets, int E, int N, int K,

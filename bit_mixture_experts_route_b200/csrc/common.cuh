@@ -126,6 +126,10 @@ cudaError_t nf4_dequantize(const uint8_t* packed, const float* absmax,
                            int64_t rows, int K, void* out, moe_dtype_t dt,
                            cudaStream_t s);
 size_t route_workspace_bytes(int T, int E, int k);
+bool route_noalloc_fits(int T, int E, int k);
+cudaError_t route_permute_noalloc(const float* logits, int T, int E, int k, int renorm,
+                                  int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                                  int32_t* sorted_rows, int32_t* inv_perm, cudaStream_t s);
 cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
                           int32_t* topk_idx, float* topk_w, int32_t* offsets,
                           int32_t* sorted_rows, int32_t* inv_perm, void* ws,

@@ -18,6 +18,7 @@
 //     expert totals and the tile's prefix, scans the totals into offsets and
 //     scatters each flat id to offsets[e] + prefix + rank.
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -242,6 +243,63 @@ cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
   moe::permute_scatter_kernel<<<ntiles, moe::kThreads, 0, s>>>(
       topk_idx, rank, tile_counts, T, E, k, ntiles, offsets, sorted_rows, inv_perm);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Routing without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they route:
+// a host framework that owns every byte of device memory through its own
+// allocator and forbids side allocations, or a latency-critical serving loop
+// in which cudaMalloc (which may synchronize the device) is not acceptable.
+// For them the routing scratch (per-row ranks and per-tile expert counts)
+// lives in one fixed-size array in this library's device memory instead.
+// Every GPU that loads the library holds this array until the process exits.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+__device__ __align__(256) unsigned char g_route_scratch[MOE_ROUTE_NOALLOC_SCRATCH_BYTES];
+
+// The array's device address on each device, looked up once per device.  In
+// host code `g_route_scratch` only names a host-side stand-in, so the kernel
+// must be given the address that cudaGetSymbolAddress reports.
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+
+cudaError_t scratch_for_current_device(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_route_scratch);  // current device = dev
+    if (err != cudaSuccess) return err;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+bool route_noalloc_fits(int T, int E, int k) {
+  return route_workspace_bytes(T, E, k) <= (size_t)MOE_ROUTE_NOALLOC_SCRATCH_BYTES;
+}
+
+cudaError_t route_permute_noalloc(const float* logits, int T, int E, int k, int renorm,
+                                  int32_t* topk_idx, float* topk_w, int32_t* offsets,
+                                  int32_t* sorted_rows, int32_t* inv_perm, cudaStream_t s) {
+  void* ws = nullptr;
+  cudaError_t err = scratch_for_current_device(&ws);
+  if (err != cudaSuccess) return err;
+  // Nothing in the scratch has to start at zero: the routing kernel writes
+  // every rank and every tile count before the scatter kernel reads them, so
+  // contents left by an earlier call are never observed.
+  return route_permute(logits, T, E, k, renorm, topk_idx, topk_w, offsets, sorted_rows,
+                       inv_perm, ws, s);
 }
 
 }  // namespace moe_launch

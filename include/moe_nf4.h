@@ -159,6 +159,36 @@ moe_status_t moe_route_permute(const float* logits, int T, int E, int k,
                                void* stream);
 
 /*
+ * moe_route_permute_noalloc -- moe_route_permute without a workspace argument.
+ * (The pages have no counterpart: this entry point exists for callers of this
+ * library that cannot allocate device memory where they route, e.g. a host
+ * framework that owns all device memory through its own allocator, or a
+ * latency-critical loop in which cudaMalloc, which may synchronize the
+ * device, is not acceptable.)
+ *
+ * Arguments, outputs and results are those of moe_route_permute.  The scratch
+ * lives in a fixed array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES bytes of device
+ * memory inside the library; every GPU that loads the library holds it until
+ * the process exits.  The call allocates nothing and frees nothing.
+ * - Size limit: moe_route_permute_workspace_size(T, E, k) must not exceed
+ *   MOE_ROUTE_NOALLOC_SCRATCH_BYTES (T*k up to about 200,000 routed rows at
+ *   E = 128); larger problems return MOE_ERR_WORKSPACE and enqueue nothing.
+ * - Set-up: the first call on each device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture on the device.
+ * - Sharing: all calls on a device use the same array, which keeps the last
+ *   call's contents (nothing in it needs to start at zero).  Calls whose
+ *   kernels overlap on the GPU -- on different streams, or from different
+ *   host threads -- race on the array and give wrong results; serialize them.
+ */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (1u << 20)
+moe_status_t moe_route_permute_noalloc(const float* logits, int T, int E, int k,
+                                       int renormalize, int32_t* topk_idx,
+                                       float* topk_w, int32_t* expert_offsets,
+                                       int32_t* sorted_rows, int32_t* inv_perm,
+                                       void* stream);
+
+/*
  * moe_nf4_grouped_gemm -- one launch over all experts:
  *   out[p, :] = W[e(p)] . A[r(p), :]   for p in [0, M_total)
  * where e(p) is the expert whose segment [offsets[e], offsets[e+1]) holds p
