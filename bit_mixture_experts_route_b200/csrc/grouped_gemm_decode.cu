@@ -10,15 +10,12 @@
 // * Persistent CTAs (one per SM) walk a list of work items built on the
 //   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
 //   rows; an expert with more routed rows yields one item per 16).
-// * One producer thread streams each item through two 3-slot rings with TMA
+// * One producer thread streams each item through a 6-stage ring with TMA
 //   tile loads, 256 k per stage: the packed rows (128 x 128 bytes), their
 //   absmax (128 x 4 fp32) and the routed activation rows (fp16, 8-row boxes
 //   of 64 k); 128-byte swizzle keeps the consumers' shared reads
 //   conflict-free.  Up to ~150 KB in flight per SM, independent of registers.
-// * Sixteen consumer warps in two groups: each group owns alternate stages of
-//   the item (its own 3-slot ring), group 1 hands its partial sums to group 0
-//   through shared memory at the end of the item.  In a group, each warp owns
-//   16 weight rows: per 64-k block a lane reads
+// * Eight consumer warps each own 16 weight rows: per 64-k block a lane reads
 //   8 packed bytes of two rows, maps each byte to an fp16 pair {L[hi], L[lo]}
 //   with one lookup in a per-lane replicated table, and issues
 //   mma.sync.m16n8k16 with the routed rows as the N side (swap-AB); the
@@ -35,10 +32,8 @@ constexpr int ROWS = 128;       // weight rows per item
 constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int SB = SK / 2;      // packed bytes per row per stage
-constexpr int GSTAGES = 3;             // ring slots per consumer group
-constexpr int STAGES = 2 * GSTAGES;
-constexpr int RWARPS = 8;              // warps per group: 16 weight rows each
-constexpr int CWARPS = 2 * RWARPS;     // two groups split each item's k range
+constexpr int STAGES = 6;
+constexpr int CWARPS = 8;
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr uint32_t kWBytes = ROWS * SB + ROWS * 4 * 4;   // packed + absmax per stage
@@ -50,7 +45,6 @@ struct __align__(8) Smem {
   uint8_t x[STAGES][4 * XKBOX];  // [64-k block][16 rows][128 B], swizzled
   float a[STAGES][ROWS * 4];
   uint32_t lut[256 * 32];
-  float red[2][RWARPS][32][2 * 4];  // group 1's partial sums, double-buffered
   uint64_t full[STAGES], empty[STAGES];
   int abort_flag;
   int nitems;
@@ -150,10 +144,8 @@ __device__ __forceinline__ Item item_info(const Smem& sm, const int32_t* offsets
 template <int EPI, typename OutT, int NT8>
 __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, int K,
                                              OutT* __restrict__ out, int32_t* dev_err,
-                                             int& slot, uint32_t& phase, int par) {
-  const int G = (threadIdx.x >> 5) / RWARPS;       // consumer group
-  const int warp = (threadIdx.x >> 5) % RWARPS;    // 16-row group within the item
-  const int lane = threadIdx.x & 31;
+                                             int& stage, uint32_t& phase) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + g : 16 * warp + g;
   const int rB = (EPI == MOE_EPI_SWIGLU) ? ROWS / 2 + 8 * warp + g : 16 * warp + g + 8;
@@ -166,13 +158,8 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
 
   const uint32_t* lut = sm.lut + lane;
   const int KS = K / SK;
-  bool failed = false;
-  for (int s = G; s < KS; s += 2) {
-    const int stage = G * GSTAGES + slot;
-    if (!mbar_wait(&sm.full[stage], phase, sm, dev_err)) {
-      failed = true;  // still take part in the barrier below
-      break;
-    }
+  for (int s = 0; s < KS; ++s) {
+    if (!mbar_wait(&sm.full[stage], phase, sm, dev_err)) return false;
     const uint8_t* wst = sm.w[stage];
     const uint8_t* xst = sm.x[stage];
     const float4 sa = *reinterpret_cast<const float4*>(&sm.a[stage][rA * 4]);
@@ -219,36 +206,8 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[stage]);
-    if (++slot == GSTAGES) { slot = 0; phase ^= 1; }
+    if (++stage == STAGES) { stage = 0; phase ^= 1; }
   }
-
-  // Group 1 hands its partial sums to group 0 (double-buffered by item
-  // parity, so one barrier of the 16 consumer warps per item suffices).
-  float* red = &sm.red[par][warp][lane][0];
-  if (G == 1) {
-#pragma unroll
-    for (int j = 0; j < NT8; ++j)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) red[4 * j + q] = acc[j][q];
-  }
-  // Barrier of the 16 consumer warps that also ORs their failure flags, so
-  // that after an expired wait every consumer leaves together (never one
-  // group waiting here for the other).
-  uint32_t any_failed;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(any_failed)
-      : "r"((uint32_t)failed), "n"(32 * CWARPS)
-      : "memory");
-  if (any_failed) return false;
-  if (G == 1) return true;
-#pragma unroll
-  for (int j = 0; j < NT8; ++j)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[j][q] += red[4 * j + q];
 
   // acc[j][q]: row rA (q < 2) or rB (q >= 2), routed row 8j + 2t + (q & 1)
 #pragma unroll
@@ -286,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], RWARPS);
+      mbar_init(&sm.empty[s], CWARPS);
     }
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -332,8 +291,8 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
   if (warp == CWARPS) {
     // ---------------- producer
     if (lane == 0) {
-      int slot[2] = {0, 0};
-      uint32_t phase[2] = {0, 0};
+      int stage = 0;
+      uint32_t phase = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         const Item it = item_info(sm, offsets, E, rtiles, i);
@@ -347,9 +306,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
         }
         const int nr8 = (it.cnt + 7) / 8;
         for (int s = 0; s < KS; ++s) {
-          const int G = s & 1;  // stage s belongs to consumer group s % 2
-          const int stage = G * GSTAGES + slot[G];
-          if (!(ok = mbar_wait(&sm.empty[stage], phase[G] ^ 1, sm, dev_err))) break;
+          if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
           mbar_arrive_expect_tx(&sm.full[stage], kWBytes + nr8 * 4 * XBOX);
           tma_load_2d(sm.w[stage], &wmap, &sm.full[stage], s * SB, y0);
           tma_load_2d(sm.w[stage] + (ROWS / 2) * SB, &wmap, &sm.full[stage], s * SB, y1);
@@ -359,23 +316,22 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
             for (int r = 0; r < nr8; ++r)
               tma_load_2d(sm.x[stage] + b * XKBOX + r * XBOX, &xmap, &sm.full[stage],
                           s * SK + b * kBlock, it.start + 8 * r);
-          if (++slot[G] == GSTAGES) { slot[G] = 0; phase[G] ^= 1; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else {
     // ---------------- consumers
-    int slot = 0;
+    int stage = 0;
     uint32_t phase = 0;
-    int par = 0;
-    for (int i = blockIdx.x; i < total; i += gridDim.x, par ^= 1) {
+    for (int i = blockIdx.x; i < total; i += gridDim.x) {
       const Item it = item_info(sm, offsets, E, rtiles, i);
       bool ok;
       if (it.cnt > 8)
-        ok = consume_item<EPI, OutT, 2>(sm, it, N, K, out, dev_err, slot, phase, par);
+        ok = consume_item<EPI, OutT, 2>(sm, it, N, K, out, dev_err, stage, phase);
       else
-        ok = consume_item<EPI, OutT, 1>(sm, it, N, K, out, dev_err, slot, phase, par);
-      if (!ok) break;  // (only on an expired wait; the kernel then ends)
+        ok = consume_item<EPI, OutT, 1>(sm, it, N, K, out, dev_err, stage, phase);
+      if (!ok) break;
     }
   }
   __syncwarp();  // the producer lane rejoins its warp before the CTA barrier
