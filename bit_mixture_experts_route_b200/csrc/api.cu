@@ -203,7 +203,8 @@ moe_status_t moe_swiglu(const void* gu, moe_dtype_t gu_dtype, int M, int I, void
 moe_status_t moe_unpermute_combine(const void* Yp, moe_dtype_t yp_dtype, const int32_t* inv_perm,
                                    const float* topk_w, int T, int k, int H, void* Y,
                                    moe_dtype_t y_dtype, void* stream) {
-  if (!valid_dtype(yp_dtype) || !valid_dtype(y_dtype) || T < 0 || k < 1 || H < 1 || H % 4)
+  if (!valid_dtype(yp_dtype) || !valid_dtype(y_dtype) || T < 0 || k < 1 || k > 32 || H < 1 ||
+      H % 4)
     return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!Yp || !inv_perm || !topk_w || !Y)) return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {Yp, inv_perm, topk_w, Y};

@@ -64,19 +64,29 @@ __global__ void __launch_bounds__(256) combine_kernel(const InT* __restrict__ Yp
                                                       const float* __restrict__ w, int T,
                                                       int k, int H, OutT* __restrict__ Y) {
   // One CTA-row of threads per token; each thread owns 4 consecutive columns.
+  // The k positions and weights are staged in shared memory first, so the k
+  // row loads of a thread are independent and issue back to back.
+  __shared__ int s_p[32];
+  __shared__ float s_w[32];
   const int t = blockIdx.x;
   if (t >= T) return;
   const int total = T * k;
+  if (threadIdx.x < k) {
+    const int p = inv_perm[(size_t)t * k + threadIdx.x];
+    s_p[threadIdx.x] = (p >= 0 && p < total) ? p : -1;
+    s_w[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+  }
+  __syncthreads();
   for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4; c < H; c += gridDim.y * blockDim.x * 4) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
     for (int j = 0; j < k; ++j) {
-      const int p = inv_perm[(size_t)t * k + j];
-      if (p < 0 || p >= total) continue;
-      const float wj = w[(size_t)t * k + j];
+      const int p = s_p[j];
+      if (p < 0) continue;
       float y[4];
       load4(Yp + (size_t)p * H + c, y);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj, y[i], acc[i]);
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(s_w[j], y[i], acc[i]);
     }
     store4(Y + (size_t)t * H + c, acc);
   }

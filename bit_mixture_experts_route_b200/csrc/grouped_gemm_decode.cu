@@ -166,42 +166,58 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
     const float4 sb = *reinterpret_cast<const float4*>(&sm.a[stage][rB * 4]);
     const float sav[4] = {sa.x, sa.y, sa.z, sa.w};
     const float sbv[4] = {sb.x, sb.y, sb.z, sb.w};
+    // Two 64-k blocks at a time, so two independent MMA chains interleave.
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      uint32_t xf[NT8][8];
+    for (int bp = 0; bp < 2; ++bp) {
+      uint32_t xf[2][NT8][8];
+      uint2 wa[2], wb[2];
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) lds_x16(xst, b, 8 * j + g, t, xf[j]);
-      // byte offset of this lane's 8 bytes in the row, 128-byte swizzled
-      const int off = b * 32 + 8 * t;
-      const uint2 wa = *reinterpret_cast<const uint2*>(
-          wst + rA * SB + ((((off >> 4) ^ (rA & 7)) << 4) | (off & 15)));
-      const uint2 wb = *reinterpret_cast<const uint2*>(
-          wst + rB * SB + ((((off >> 4) ^ (rB & 7)) << 4) | (off & 15)));
-      float tmp[NT8][4];
+      for (int h = 0; h < 2; ++h) {
+        const int b = 2 * bp + h;
 #pragma unroll
-      for (int j = 0; j < NT8; ++j)
+        for (int j = 0; j < NT8; ++j) lds_x16(xst, b, 8 * j + g, t, xf[h][j]);
+        // byte offset of this lane's 8 bytes in the row, 128-byte swizzled
+        const int off = b * 32 + 8 * t;
+        wa[h] = *reinterpret_cast<const uint2*>(
+            wst + rA * SB + ((((off >> 4) ^ (rA & 7)) << 4) | (off & 15)));
+        wb[h] = *reinterpret_cast<const uint2*>(
+            wst + rB * SB + ((((off >> 4) ^ (rB & 7)) << 4) | (off & 15)));
+      }
+      float tmp[2][NT8][4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmp[j][q] = 0.0f;
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int j = 0; j < NT8; ++j)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmp[h][j][q] = 0.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t vA = (i < 2) ? wa.x : wa.y;
-        const uint32_t vB = (i < 2) ? wb.x : wb.y;
         const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
-        // byte -> table entry (byte * 32 + lane): one byte_perm and one shift-add
-        uint32_t af[4];
-        af[0] = lut[__byte_perm(vA, 0, 0x4440u | lo) << 5];
-        af[1] = lut[__byte_perm(vB, 0, 0x4440u | lo) << 5];
-        af[2] = lut[__byte_perm(vA, 0, 0x4440u | (lo + 1)) << 5];
-        af[3] = lut[__byte_perm(vB, 0, 0x4440u | (lo + 1)) << 5];
 #pragma unroll
-        for (int j = 0; j < NT8; ++j) mma_16816(tmp[j], af, xf[j][2 * i], xf[j][2 * i + 1]);
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t vA = (i < 2) ? wa[h].x : wa[h].y;
+          const uint32_t vB = (i < 2) ? wb[h].x : wb[h].y;
+          // byte -> table entry (byte * 32 + lane): one byte_perm and one shift-add
+          uint32_t af[4];
+          af[0] = lut[__byte_perm(vA, 0, 0x4440u | lo) << 5];
+          af[1] = lut[__byte_perm(vB, 0, 0x4440u | lo) << 5];
+          af[2] = lut[__byte_perm(vA, 0, 0x4440u | (lo + 1)) << 5];
+          af[3] = lut[__byte_perm(vB, 0, 0x4440u | (lo + 1)) << 5];
+#pragma unroll
+          for (int j = 0; j < NT8; ++j)
+            mma_16816(tmp[h][j], af, xf[h][j][2 * i], xf[h][j][2 * i + 1]);
+        }
       }
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) {
-        acc[j][0] = fmaf(sav[b], tmp[j][0], acc[j][0]);
-        acc[j][1] = fmaf(sav[b], tmp[j][1], acc[j][1]);
-        acc[j][2] = fmaf(sbv[b], tmp[j][2], acc[j][2]);
-        acc[j][3] = fmaf(sbv[b], tmp[j][3], acc[j][3]);
+      for (int h = 0; h < 2; ++h) {
+        const float s_a = sav[2 * bp + h], s_b = sbv[2 * bp + h];
+#pragma unroll
+        for (int j = 0; j < NT8; ++j) {
+          acc[j][0] = fmaf(s_a, tmp[h][j][0], acc[j][0]);
+          acc[j][1] = fmaf(s_a, tmp[h][j][1], acc[j][1]);
+          acc[j][2] = fmaf(s_b, tmp[h][j][2], acc[j][2]);
+          acc[j][3] = fmaf(s_b, tmp[h][j][3], acc[j][3]);
+        }
       }
     }
     __syncwarp();

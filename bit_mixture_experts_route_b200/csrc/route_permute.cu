@@ -8,10 +8,13 @@
 //   sorted_rows[T*k]     flat ids t*k+j ordered by expert, then by flat id
 //   inv_perm[T*k]        position of each flat id
 //
-// Two launches, both deterministic (no atomics whose order matters):
+// Decode sizes (T*k <= 4096, E <= 256) run in one single-CTA launch
+// (route_small_kernel).  Larger problems take two launches, both
+// deterministic (no atomics whose order matters):
 //  1. route_tile_kernel, one CTA per tile of 64 tokens: one warp per token
 //     selects the top-k with 64-bit keys (ordered logit, ~expert) so ties go
-//     to the lower expert and every lane agrees even on NaN, computes the
+//     to the lower expert and every lane agrees even on NaN (two redux.sync
+//     maxima per selection), computes the
 //     softmax weights, then warp 0 ranks the tile's routed rows stably with
 //     __match_any_sync and writes the tile's per-expert counts.
 //  2. permute_scatter_kernel, one CTA per tile: sums the tile counts into
@@ -37,6 +40,68 @@ __device__ __forceinline__ float unordered_bits(uint32_t o) {
   return __uint_as_float(u);
 }
 
+// Top-k of one token's logits by one warp.  Lane l holds experts l + 32 i
+// as 64-bit keys (order-preserving logit bits << 32 | ~expert; 0 = absent),
+// so the largest key is the largest logit and, among equal logits, the lower
+// expert.  Each of the k rounds takes the warp maximum in two redux.sync
+// steps (high word, then low word among the lanes holding that high word).
+// Lane j < k receives the j-th selected key in `mine`; every lane receives
+// the largest key in `first`.
+template <int NPER>
+__device__ __forceinline__ void warp_topk(const uint64_t (&key)[NPER], int k, int E,
+                                          uint64_t& mine, uint64_t& first) {
+  const int lane = threadIdx.x & 31;
+  uint32_t taken = 0;
+  mine = 0;
+  first = 0;
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = 0;
+#pragma unroll
+    for (int i = 0; i < NPER; ++i)
+      if (!((taken >> i) & 1u) && key[i] > best) best = key[i];
+    const uint32_t hi = (uint32_t)(best >> 32);
+    const uint32_t mh = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t ml = __reduce_max_sync(0xffffffffu, hi == mh ? (uint32_t)best : 0u);
+    const uint64_t sel = ((uint64_t)mh << 32) | ml;
+    const int e = (int)(~ml);
+    if (e >= 0 && e < E && (e & 31) == lane) taken |= 1u << (e >> 5);
+    if (j == lane) mine = sel;
+    if (j == 0) first = sel;
+  }
+}
+
+// Routing weights of the selected experts (softmax over the k selected
+// logits when renormalising, else over all E); lane j < k returns weight j.
+template <int NPER>
+__device__ __forceinline__ float warp_topk_weight(const uint64_t (&key)[NPER], uint64_t mine,
+                                                  uint64_t first, int k, int E, int renorm) {
+  const int lane = threadIdx.x & 31;
+  const float mx = unordered_bits((uint32_t)(first >> 32));
+  float ex = 0.0f;
+  if (lane < k) ex = expf(unordered_bits((uint32_t)(mine >> 32)) - mx);
+  float denom;
+  if (renorm) {
+    denom = warp_sum(ex);
+  } else {
+    float part = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NPER; ++i)
+      if (lane + 32 * i < E) part += expf(unordered_bits((uint32_t)(key[i] >> 32)) - mx);
+    denom = warp_sum(part);
+  }
+  return __fdiv_rn(ex, denom);
+}
+
+template <int NPER>
+__device__ __forceinline__ void load_keys(const float* row, int E, uint64_t (&key)[NPER]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = (e < E) ? ((uint64_t)ordered_bits(row[e]) << 32) | (uint32_t)(~e) : 0ull;
+  }
+}
+
 template <int NPER>
 __global__ void __launch_bounds__(kThreads) route_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
@@ -51,49 +116,15 @@ __global__ void __launch_bounds__(kThreads) route_tile_kernel(
   for (int tt = warp; tt < kTileTok; tt += kThreads / 32) {
     const int t = tile * kTileTok + tt;
     if (t >= T) break;
-    const float* row = logits + (size_t)t * E;
     uint64_t key[NPER];
-#pragma unroll
-    for (int i = 0; i < NPER; ++i) {
-      const int e = lane + 32 * i;
-      key[i] = (e < E) ? ((uint64_t)ordered_bits(row[e]) << 32) | (uint32_t)(~e) : 0ull;
-    }
-    uint32_t taken = 0;
-    uint64_t mine = 0;  // lane j keeps the j-th selected key
-    uint64_t first = 0;
-    for (int j = 0; j < k; ++j) {
-      uint64_t best = 0;
-#pragma unroll
-      for (int i = 0; i < NPER; ++i)
-        if (!((taken >> i) & 1u) && key[i] > best) best = key[i];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-        best = other > best ? other : best;
-      }
-      const int e = (int)(~(uint32_t)best);
-      if (e >= 0 && e < E && (e & 31) == lane) taken |= 1u << (e >> 5);
-      if (j == lane) mine = best;
-      if (j == 0) first = best;
-    }
-    // softmax: max logit = first selected
-    const float mx = unordered_bits((uint32_t)(first >> 32));
-    float ex = 0.0f;
-    if (lane < k) ex = expf(unordered_bits((uint32_t)(mine >> 32)) - mx);
-    float denom;
-    if (renorm) {
-      denom = warp_sum(ex);
-    } else {
-      float part = 0.0f;
-#pragma unroll
-      for (int i = 0; i < NPER; ++i)
-        if (lane + 32 * i < E) part += expf(unordered_bits((uint32_t)(key[i] >> 32)) - mx);
-      denom = warp_sum(part);
-    }
+    load_keys<NPER>(logits + (size_t)t * E, E, key);
+    uint64_t mine, first;
+    warp_topk<NPER>(key, k, E, mine, first);
+    const float w = warp_topk_weight<NPER>(key, mine, first, k, E, renorm);
     if (lane < k) {
       const int e = (int)(~(uint32_t)mine);
       topk_idx[(size_t)t * k + lane] = e;
-      topk_w[(size_t)t * k + lane] = __fdiv_rn(ex, denom);
+      topk_w[(size_t)t * k + lane] = w;
       s_eid[tt * k + lane] = e;
     }
   }
@@ -121,6 +152,112 @@ __global__ void __launch_bounds__(kThreads) route_tile_kernel(
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += kThreads) tile_counts[(size_t)tile * E + e] = s_cnt[e];
+}
+
+// Decode-sized routing in one launch (T*k <= kSmallRows, E <= kSmallE): one
+// CTA of 32 warps routes every token (warp per token), ranks the routed rows
+// stably (each warp walks a contiguous chunk of flat ids with
+// __match_any_sync, keeping per-warp expert counts), scans the counts into
+// expert offsets and scatters.
+constexpr int kSmallRows = 4096;
+constexpr int kSmallE = 256;
+constexpr int kSmallThreads = 1024;
+
+template <int NPER>
+__global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int renorm,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
+    int32_t* __restrict__ inv_perm) {
+  // 16-bit fields: rows, ranks and counts are all < kSmallRows = 4096
+  __shared__ int16_t s_eid[kSmallRows];
+  __shared__ uint16_t s_rank[kSmallRows];
+  __shared__ uint16_t s_wc[32][kSmallE];   // per-warp expert counts, then prefixes
+  __shared__ int s_off[kSmallE + 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 32 * kSmallE; i += kSmallThreads) (&s_wc[0][0])[i] = 0;
+  // (made visible by the __syncthreads after the routing loop)
+
+  for (int t = warp; t < T; t += 32) {
+    uint64_t key[NPER];
+    load_keys<NPER>(logits + (size_t)t * E, E, key);
+    uint64_t mine, first;
+    warp_topk<NPER>(key, k, E, mine, first);
+    const float w = warp_topk_weight<NPER>(key, mine, first, k, E, renorm);
+    if (lane < k) {
+      const int e = (int)(~(uint32_t)mine);
+      topk_idx[(size_t)t * k + lane] = e;
+      topk_w[(size_t)t * k + lane] = w;
+      s_eid[t * k + lane] = (int16_t)((e >= 0 && e < E) ? e : -1);
+    }
+  }
+  __syncthreads();
+
+  // stable rank within each warp's contiguous chunk of flat ids
+  const int n = T * k;
+  const int chunk = (n + 31) / 32;
+  const int f0 = warp * chunk, f1 = min(n, f0 + chunk);
+  for (int base = f0; base < f1; base += 32) {
+    const int f = base + lane;
+    const int e = (f < f1) ? s_eid[f] : -1;
+    const bool valid = e >= 0 && e < E;
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : (1 << 20) + lane);
+    const int r = __popc(peers & lanemask_lt());
+    const int c0 = valid ? s_wc[warp][e] : 0;
+    __syncwarp();
+    if (valid && (peers >> lane) == 1u) s_wc[warp][e] = (uint16_t)(c0 + __popc(peers));
+    __syncwarp();
+    if (f < f1) s_rank[f] = valid ? (uint16_t)(c0 + r) : (uint16_t)0xffffu;
+  }
+  __syncthreads();
+
+  // per expert: exclusive prefix over warps, and the total
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = s_wc[w][e];
+      s_wc[w][e] = (uint16_t)run;
+      run += c;
+    }
+    s_off[e] = run;
+  }
+  __syncthreads();
+  // exclusive scan of the totals by warp 0 (E <= 256: 8 per lane)
+  if (warp == 0) {
+    int v[kSmallE / 32];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kSmallE / 32; ++i) {
+      const int e = lane * (kSmallE / 32) + i;
+      v[i] = e < E ? s_off[e] : 0;
+      sum += v[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < kSmallE / 32; ++i) {
+      const int e = lane * (kSmallE / 32) + i;
+      if (e < E) s_off[e] = run;
+      run += v[i];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += kSmallThreads) offsets[e] = (e < E) ? s_off[e] : n;
+  for (int f = threadIdx.x; f < n; f += kSmallThreads) {
+    const int e = s_eid[f];
+    const int r = s_rank[f];
+    if (e < 0 || e >= E || r == 0xffff) continue;
+    const int pos = s_off[e] + s_wc[f / chunk][e] + r;
+    if (pos < 0 || pos >= n) continue;
+    sorted_rows[pos] = f;
+    inv_perm[f] = pos;
+  }
 }
 
 // Exclusive scan of s[0..n) in place for n <= 1024 with kThreads threads.
@@ -223,6 +360,18 @@ cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
                           int32_t* sorted_rows, int32_t* inv_perm, void* ws,
                           cudaStream_t s) {
   if (T == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
+  if ((int64_t)T * k <= moe::kSmallRows && E <= moe::kSmallE) {
+#define MOE_ROUTE_SMALL(NP)                                                           \
+  moe::route_small_kernel<NP><<<1, moe::kSmallThreads, 0, s>>>(logits, T, E, k, renorm, \
+                                                               topk_idx, topk_w, offsets, \
+                                                               sorted_rows, inv_perm)
+    if (E <= 32) MOE_ROUTE_SMALL(1);
+    else if (E <= 64) MOE_ROUTE_SMALL(2);
+    else if (E <= 128) MOE_ROUTE_SMALL(4);
+    else MOE_ROUTE_SMALL(8);
+#undef MOE_ROUTE_SMALL
+    return cudaGetLastError();
+  }
   const int ntiles = (T + moe::kTileTok - 1) / moe::kTileTok;
   int32_t* rank = reinterpret_cast<int32_t*>(ws);
   int32_t* tile_counts =

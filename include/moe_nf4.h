@@ -260,7 +260,7 @@ moe_status_t moe_swiglu(const void* gu, moe_dtype_t gu_dtype, int M, int I,
  * moe_unpermute_combine -- Y[t, :] = sum_{j<k} topk_w[t, j] *
  * Yp[inv_perm[t*k + j], :], summed in j order in fp32.
  *   Yp [T*k, H] of yp_dtype (F32, BF16, F16), Y [T, H] of y_dtype.
- *   H % 4 == 0, pointers 16-byte aligned.
+ *   1 <= k <= 32, H % 4 == 0, pointers 16-byte aligned.
  */
 moe_status_t moe_unpermute_combine(const void* Yp, moe_dtype_t yp_dtype,
                                    const int32_t* inv_perm,
