@@ -24,6 +24,7 @@ DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EPI = {"none": 0, "swiglu": 1}
 ALGO = {"auto": 0, "gemv": 1, "tc": 2}
 DEVERR_NONFINITE, DEVERR_BAD_OFFSETS, DEVERR_BAD_INDEX, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_LAYOUT = 16
 
 # Every exported symbol with (restype, argtypes); the header declares them.
 _P, _I, _Z, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p

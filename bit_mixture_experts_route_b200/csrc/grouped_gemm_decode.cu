@@ -5,21 +5,27 @@
 // bullet: one launch for all active experts, the 16-entry codebook decoded in
 // registers, no dequantized weight copy.  At decode sizes the whole cost is
 // streaming the NF4 bytes of every expert that received a token, so the
-// design goal is to keep enough bytes in flight to saturate HBM:
+// kernel is built to keep HBM busy with as few instructions per weight as
+// possible:
 //
 // * Persistent CTAs (one per SM) walk a list of work items built on the
 //   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
 //   rows; an expert with more routed rows yields one item per 16).
-// * One producer thread streams each item through a 6-stage ring with TMA
+// * One producer thread streams each item through a 5-stage ring with TMA
 //   tile loads, 256 k per stage: the packed rows (128 x 128 bytes), their
 //   absmax (128 x 4 fp32) and the routed activation rows (fp16, 8-row boxes
-//   of 64 k); 128-byte swizzle keeps the consumers' shared reads
-//   conflict-free.  Up to ~150 KB in flight per SM, independent of registers.
-// * Eight consumer warps each own 16 weight rows: per 64-k block a lane reads
-//   8 packed bytes of two rows, maps each byte to an fp16 pair {L[hi], L[lo]}
-//   with one lookup in a per-lane replicated table, and issues
-//   mma.sync.m16n8k16 with the routed rows as the N side (swap-AB); the
-//   block's fp32 absmax scales the block's fp32 partial sums.
+//   of 64 k), with 128-byte swizzle.
+// * Eight consumer warps each own 16 weight rows and run mma.sync.m16n8k16
+//   with the weights as the M side and the routed rows as N (swap-AB).  A
+//   lane turns each packed byte into an fp16 pair {L[hi], L[lo]} with ONE
+//   byte_perm (which assembles the shared address of the byte's entry in a
+//   per-lane table: 0x10000 | byte << 8 | lane << 2) and one shared load.
+//   The table sits at shared address 64 KB, one 256-byte row per byte value,
+//   so the lookups never conflict.  The four 64-k blocks of a stage run as
+//   four interleaved MMA chains, and each block's fp32 absmax scales its
+//   fp32 partial sums (the only weight rounding is the levels' fp16 one).
+// * MMA row g of a warp maps to weight row sigma(g) = 2(g mod 4) + g div 4,
+//   which makes the swizzled 8-byte reads of the packed rows conflict-free.
 // * The SwiGLU epilogue pairs gate row j and up row I + j in the same lane.
 // Every wait is bounded; on expiry MOE_DEVERR_TIMEOUT is set and all roles
 // leave their loops.
@@ -32,69 +38,97 @@ constexpr int ROWS = 128;       // weight rows per item
 constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int SB = SK / 2;      // packed bytes per row per stage
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int CWARPS = 8;
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
-constexpr uint32_t kWBytes = ROWS * SB + ROWS * 4 * 4;   // packed + absmax per stage
-constexpr int XBOX = 8 * 64 * 2;                         // one 8-row x 64-k fp16 box
-constexpr int XKBOX = (TOK / 8) * XBOX;                  // 16 rows x 64 k
+constexpr int XBOX = 8 * 64 * 2;                 // one 8-row x 64-k fp16 box
+constexpr int XKBOX = (TOK / 8) * XBOX;          // 16 rows x 64 k
+constexpr uint32_t kWBytes = ROWS * SB;          // packed rows per stage
+constexpr uint32_t kXBytes = 4 * XKBOX;          // activations per stage (max)
+constexpr uint32_t kABytes = ROWS * 16;          // absmax per stage
+constexpr uint32_t kStageBytes = kWBytes + kXBytes + kABytes;  // 26 KB, 1 KB multiple
 
-struct __align__(8) Smem {
-  uint8_t w[STAGES][ROWS * SB];  // 1024-aligned (struct placed at 1024)
-  uint8_t x[STAGES][4 * XKBOX];  // [64-k block][16 rows][128 B], swizzled
-  float a[STAGES][ROWS * 4];
-  uint32_t lut[256 * 32];
+// Absolute shared-memory layout.  The dynamic window must start at or below
+// 1 KB (checked at run time).  Stages need 1 KB alignment (128-byte swizzle).
+constexpr uint32_t kStage0 = 1024;                        // stages 0-1
+constexpr uint32_t kMisc = kStage0 + 2 * kStageBytes;     // barriers, item list
+constexpr uint32_t kLut = 65536;                          // table: 256 x 256 B
+constexpr uint32_t kStage2 = 2 * 65536;                   // stages 2-4
+constexpr uint32_t kEnd = kStage2 + (STAGES - 2) * kStageBytes;
+
+__device__ __forceinline__ uint32_t stage_addr(int s) {
+  return s < 2 ? kStage0 + s * kStageBytes : kStage2 + (s - 2) * kStageBytes;
+}
+
+struct Misc {
   uint64_t full[STAGES], empty[STAGES];
   int abort_flag;
   int nitems;
   int item_prefix[1025];
 };
+static_assert(kMisc + sizeof(Misc) <= kLut, "shared layout overlap");
 
 __constant__ float c_levels_dec[16] = {MOE_NF4_LEVEL_LIST};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem& sm,
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Misc& ms,
                                           int32_t* dev_err) {
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) return false;
+    if (*reinterpret_cast<volatile int*>(&ms.abort_flag)) return false;
   }
-  *reinterpret_cast<volatile int*>(&sm.abort_flag) = 1;
+  *reinterpret_cast<volatile int*>(&ms.abort_flag) = 1;
   set_dev_err(dev_err, MOE_DEVERR_TIMEOUT);
   return false;
 }
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
       : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
 }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -105,31 +139,29 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-
-// This lane's 16 activations of routed row `r` (0..15) in 64-k block `b` of
-// a stage, as 8 fp16 pairs: bytes [32t, 32t + 32) of the row's swizzled
-// 128-byte line.
-__device__ __forceinline__ void lds_x16(const uint8_t* xs, int b, int r, int t,
-                                        uint32_t (&xf)[8]) {
-  const uint8_t* line = xs + b * XKBOX + r * 128;
-  const uint4 u = *reinterpret_cast<const uint4*>(line + (((2 * t) ^ (r & 7)) << 4));
-  const uint4 v = *reinterpret_cast<const uint4*>(line + (((2 * t + 1) ^ (r & 7)) << 4));
-  xf[0] = u.x; xf[1] = u.y; xf[2] = u.z; xf[3] = u.w;
-  xf[4] = v.x; xf[5] = v.y; xf[6] = v.z; xf[7] = v.w;
+// Same with a zero accumulator input (first MMA of a block).
+__device__ __forceinline__ void mma_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                            uint32_t b1) {
+  const float z = 0.0f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(z));
 }
 
 struct Item {
   int expert, rtile, start, cnt;  // routed rows [start, start + cnt)
 };
 
-__device__ __forceinline__ Item item_info(const Smem& sm, const int32_t* offsets, int E,
+__device__ __forceinline__ Item item_info(const Misc& ms, const int32_t* offsets, int E,
                                           int rtiles, int it) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (sm.item_prefix[mid] <= it) lo = mid; else hi = mid;
+    if (ms.item_prefix[mid] <= it) lo = mid; else hi = mid;
   }
-  const int local = it - sm.item_prefix[lo];
+  const int local = it - ms.item_prefix[lo];
   const int tc = local / rtiles;
   Item r;
   r.expert = lo;
@@ -142,13 +174,24 @@ __device__ __forceinline__ Item item_info(const Smem& sm, const int32_t* offsets
 
 // One item's main loop and epilogue for one consumer warp, NT8 token tiles.
 template <int EPI, typename OutT, int NT8>
-__device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, int K,
+__device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, int K,
                                              OutT* __restrict__ out, int32_t* dev_err,
                                              int& stage, uint32_t& phase) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + g : 16 * warp + g;
-  const int rB = (EPI == MOE_EPI_SWIGLU) ? ROWS / 2 + 8 * warp + g : 16 * warp + g + 8;
+  const int sg = ((g & 3) << 1) | (g >> 2);  // sigma(g)
+  const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + sg : 16 * warp + sg;
+  const int rB = (EPI == MOE_EPI_SWIGLU) ? ROWS / 2 + 8 * warp + sg : 16 * warp + sg + 8;
+  // byte_perm source: 0x10000 | lane << 2 -> entry address of a byte
+  const uint32_t lb = 0x10000u | ((uint32_t)lane << 2);
+  // this lane's 8 packed bytes of block b in a 128-byte swizzled row whose
+  // row index is congruent to sg (mod 8): chunk (2b + t/2) ^ sg, half t & 1
+  uint32_t woff[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+    woff[b] = ((((2 * b + (t >> 1)) ^ sg) << 4) | ((t & 1) << 3));
+  // activation rows 8j + g: chunks 2t and 2t+1 of the 128-byte line, swizzled
+  const uint32_t xo0 = (uint32_t)(((2 * t) ^ g) << 4), xo1 = (uint32_t)(((2 * t + 1) ^ g) << 4);
 
   float acc[NT8][4];
 #pragma unroll
@@ -156,72 +199,65 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[j][q] = 0.0f;
 
-  const uint32_t* lut = sm.lut + lane;
   const int KS = K / SK;
   for (int s = 0; s < KS; ++s) {
-    if (!mbar_wait(&sm.full[stage], phase, sm, dev_err)) return false;
-    const uint8_t* wst = sm.w[stage];
-    const uint8_t* xst = sm.x[stage];
-    const float4 sa = *reinterpret_cast<const float4*>(&sm.a[stage][rA * 4]);
-    const float4 sb = *reinterpret_cast<const float4*>(&sm.a[stage][rB * 4]);
-    const float sav[4] = {sa.x, sa.y, sa.z, sa.w};
-    const float sbv[4] = {sb.x, sb.y, sb.z, sb.w};
-    // Two 64-k blocks at a time, so two independent MMA chains interleave.
+    const uint32_t base = stage_addr(stage);
+    if (!mbar_wait(smem_u32(&ms.full[stage]), phase, ms, dev_err)) return false;
+    const uint32_t wst = base, xst = base + kWBytes, ast = base + kWBytes + kXBytes;
+    const uint4 sa = lds128(ast + rA * 16), sb = lds128(ast + rB * 16);
+    const float sav[4] = {__uint_as_float(sa.x), __uint_as_float(sa.y), __uint_as_float(sa.z),
+                          __uint_as_float(sa.w)};
+    const float sbv[4] = {__uint_as_float(sb.x), __uint_as_float(sb.y), __uint_as_float(sb.z),
+                          __uint_as_float(sb.w)};
+    uint32_t xf[4][NT8][8];
+    uint2 wa[4], wb[4];
 #pragma unroll
-    for (int bp = 0; bp < 2; ++bp) {
-      uint32_t xf[2][NT8][8];
-      uint2 wa[2], wb[2];
+    for (int b = 0; b < 4; ++b) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int b = 2 * bp + h;
-#pragma unroll
-        for (int j = 0; j < NT8; ++j) lds_x16(xst, b, 8 * j + g, t, xf[h][j]);
-        // byte offset of this lane's 8 bytes in the row, 128-byte swizzled
-        const int off = b * 32 + 8 * t;
-        wa[h] = *reinterpret_cast<const uint2*>(
-            wst + rA * SB + ((((off >> 4) ^ (rA & 7)) << 4) | (off & 15)));
-        wb[h] = *reinterpret_cast<const uint2*>(
-            wst + rB * SB + ((((off >> 4) ^ (rB & 7)) << 4) | (off & 15)));
+      for (int j = 0; j < NT8; ++j) {
+        const uint32_t line = xst + b * XKBOX + (8 * j + g) * 128;
+        const uint4 u = lds128(line + xo0), v = lds128(line + xo1);
+        xf[b][j][0] = u.x; xf[b][j][1] = u.y; xf[b][j][2] = u.z; xf[b][j][3] = u.w;
+        xf[b][j][4] = v.x; xf[b][j][5] = v.y; xf[b][j][6] = v.z; xf[b][j][7] = v.w;
       }
-      float tmp[2][NT8][4];
+      wa[b] = lds64(wst + rA * SB + woff[b]);
+      wb[b] = lds64(wst + rB * SB + woff[b]);
+    }
+    float tmp[4][NT8][4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
+      const uint32_t s0 = 0x7604u | (lo << 4), s1 = 0x7604u | ((lo + 1) << 4);
 #pragma unroll
-        for (int j = 0; j < NT8; ++j)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmp[h][j][q] = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t vA = (i < 2) ? wa[h].x : wa[h].y;
-          const uint32_t vB = (i < 2) ? wb[h].x : wb[h].y;
-          // byte -> table entry (byte * 32 + lane): one byte_perm and one shift-add
-          uint32_t af[4];
-          af[0] = lut[__byte_perm(vA, 0, 0x4440u | lo) << 5];
-          af[1] = lut[__byte_perm(vB, 0, 0x4440u | lo) << 5];
-          af[2] = lut[__byte_perm(vA, 0, 0x4440u | (lo + 1)) << 5];
-          af[3] = lut[__byte_perm(vB, 0, 0x4440u | (lo + 1)) << 5];
-#pragma unroll
-          for (int j = 0; j < NT8; ++j)
-            mma_16816(tmp[h][j], af, xf[h][j][2 * i], xf[h][j][2 * i + 1]);
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float s_a = sav[2 * bp + h], s_b = sbv[2 * bp + h];
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t vA = (i < 2) ? wa[b].x : wa[b].y;
+        const uint32_t vB = (i < 2) ? wb[b].x : wb[b].y;
+        uint32_t af[4];
+        af[0] = lds32(__byte_perm(vA, lb, s0));
+        af[1] = lds32(__byte_perm(vB, lb, s0));
+        af[2] = lds32(__byte_perm(vA, lb, s1));
+        af[3] = lds32(__byte_perm(vB, lb, s1));
 #pragma unroll
         for (int j = 0; j < NT8; ++j) {
-          acc[j][0] = fmaf(s_a, tmp[h][j][0], acc[j][0]);
-          acc[j][1] = fmaf(s_a, tmp[h][j][1], acc[j][1]);
-          acc[j][2] = fmaf(s_b, tmp[h][j][2], acc[j][2]);
-          acc[j][3] = fmaf(s_b, tmp[h][j][3], acc[j][3]);
+          if (i == 0)
+            mma_16816_z(tmp[b][j], af, xf[b][j][0], xf[b][j][1]);
+          else
+            mma_16816(tmp[b][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
         }
       }
     }
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+#pragma unroll
+      for (int j = 0; j < NT8; ++j) {
+        acc[j][0] = fmaf(sav[b], tmp[b][j][0], acc[j][0]);
+        acc[j][1] = fmaf(sav[b], tmp[b][j][1], acc[j][1]);
+        acc[j][2] = fmaf(sbv[b], tmp[b][j][2], acc[j][2]);
+        acc[j][3] = fmaf(sbv[b], tmp[b][j][3], acc[j][3]);
+      }
+    }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.empty[stage]);
+    if (lane == 0) mbar_arrive(smem_u32(&ms.empty[stage]));
     if (++stage == STAGES) { stage = 0; phase ^= 1; }
   }
 
@@ -235,10 +271,10 @@ __device__ __forceinline__ bool consume_item(Smem& sm, const Item& it, int N, in
       const size_t p = (size_t)(it.start + tok);
       if (EPI == MOE_EPI_SWIGLU) {
         const int I = N / 2;
-        const int col = it.rtile * (ROWS / 2) + 8 * warp + g;
+        const int col = it.rtile * (ROWS / 2) + 8 * warp + sg;
         out[p * I + col] = from_f32<OutT>(swiglu_f32(acc[j][q], acc[j][q + 2]));
       } else {
-        const int col = it.rtile * ROWS + 16 * warp + g;
+        const int col = it.rtile * ROWS + 16 * warp + sg;
         out[p * N + col] = from_f32<OutT>(acc[j][q]);
         out[p * N + col + 8] = from_f32<OutT>(acc[j][q + 2]);
       }
@@ -252,32 +288,40 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
     const __grid_constant__ CUtensorMap xmap, const int32_t* __restrict__ offsets, int E, int N,
     int K, int M_total, OutT* __restrict__ out, int32_t* dev_err) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  if (base > kStage0) {  // layout assumption broken: do nothing, say so
+    if (threadIdx.x == 0) set_dev_err(dev_err, MOE_DEVERR_LAYOUT);
+    return;
+  }
+  Misc& ms = *reinterpret_cast<Misc*>(smem_raw + (kMisc - base));
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem_raw + (kLut - base));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rtiles = N / ROWS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], CWARPS);
+      mbar_init(smem_u32(&ms.full[s]), 1);
+      mbar_init(smem_u32(&ms.empty[s]), CWARPS);
     }
-    sm.abort_flag = 0;
+    ms.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // byte b -> {fp16 L[b >> 4] (low half), fp16 L[b & 15] (high half)}, one
+  // 256-byte row per byte value, lane l's copy at 4 l (the upper 128 bytes of
+  // each row are unused)
   for (int i = threadIdx.x; i < 256 * 32; i += THREADS) {
-    const int b = i >> 5;
+    const int b = i >> 5, l = i & 31;
     const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
                                      __float2half_rn(c_levels_dec[b & 15]));
-    sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+    lut[b * 64 + l] = *reinterpret_cast<const uint32_t*>(&h);
   }
   if (warp == CWARPS) {
     // item_prefix[e] = sum over e' < e of ceil(count / TOK) * rtiles
     bool bad = offsets[0] != 0 || offsets[E] != M_total;
     int run = 0;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
+    for (int b0 = 0; b0 < E; b0 += 32) {
+      const int e = b0 + lane;
       int c = 0;
       if (e < E) {
         c = offsets[e + 1] - offsets[e];
@@ -290,18 +334,18 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (e < E) sm.item_prefix[e] = run + incl - items;
+      if (e < E) ms.item_prefix[e] = run + incl - items;
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) {
-      sm.item_prefix[E] = run;
-      sm.nitems = bad ? 0 : run;
+      ms.item_prefix[E] = run;
+      ms.nitems = bad ? 0 : run;
       if (bad) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
     }
   }
   __syncthreads();
-  const int total = sm.nitems;
+  const int total = ms.nitems;
   const int KS = K / SK;
 
   if (warp == CWARPS) {
@@ -311,7 +355,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
       uint32_t phase = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-        const Item it = item_info(sm, offsets, E, rtiles, i);
+        const Item it = item_info(ms, offsets, E, rtiles, i);
         int y0, y1;
         if (EPI == MOE_EPI_SWIGLU) {
           y0 = it.expert * N + it.rtile * (ROWS / 2);
@@ -322,16 +366,18 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
         }
         const int nr8 = (it.cnt + 7) / 8;
         for (int s = 0; s < KS; ++s) {
-          if (!(ok = mbar_wait(&sm.empty[stage], phase ^ 1, sm, dev_err))) break;
-          mbar_arrive_expect_tx(&sm.full[stage], kWBytes + nr8 * 4 * XBOX);
-          tma_load_2d(sm.w[stage], &wmap, &sm.full[stage], s * SB, y0);
-          tma_load_2d(sm.w[stage] + (ROWS / 2) * SB, &wmap, &sm.full[stage], s * SB, y1);
-          tma_load_2d(sm.a[stage], &amap, &sm.full[stage], s * 4, y0);
-          tma_load_2d(sm.a[stage] + (ROWS / 2) * 4, &amap, &sm.full[stage], s * 4, y1);
+          const uint32_t full = smem_u32(&ms.full[stage]);
+          if (!(ok = mbar_wait(smem_u32(&ms.empty[stage]), phase ^ 1, ms, dev_err))) break;
+          const uint32_t sb = stage_addr(stage);
+          mbar_arrive_expect_tx(full, kWBytes + kABytes + nr8 * 4 * XBOX);
+          tma_load_2d(sb, &wmap, full, s * SB, y0);
+          tma_load_2d(sb + (ROWS / 2) * SB, &wmap, full, s * SB, y1);
+          tma_load_2d(sb + kWBytes + kXBytes, &amap, full, s * 4, y0);
+          tma_load_2d(sb + kWBytes + kXBytes + (ROWS / 2) * 16, &amap, full, s * 4, y1);
           for (int b = 0; b < 4; ++b)
             for (int r = 0; r < nr8; ++r)
-              tma_load_2d(sm.x[stage] + b * XKBOX + r * XBOX, &xmap, &sm.full[stage],
-                          s * SK + b * kBlock, it.start + 8 * r);
+              tma_load_2d(sb + kWBytes + b * XKBOX + r * XBOX, &xmap, full, s * SK + b * kBlock,
+                          it.start + 8 * r);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -341,12 +387,12 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
     int stage = 0;
     uint32_t phase = 0;
     for (int i = blockIdx.x; i < total; i += gridDim.x) {
-      const Item it = item_info(sm, offsets, E, rtiles, i);
+      const Item it = item_info(ms, offsets, E, rtiles, i);
       bool ok;
       if (it.cnt > 8)
-        ok = consume_item<EPI, OutT, 2>(sm, it, N, K, out, dev_err, stage, phase);
+        ok = consume_item<EPI, OutT, 2>(ms, it, N, K, out, dev_err, stage, phase);
       else
-        ok = consume_item<EPI, OutT, 1>(sm, it, N, K, out, dev_err, stage, phase);
+        ok = consume_item<EPI, OutT, 1>(ms, it, N, K, out, dev_err, stage, phase);
       if (!ok) break;
     }
   }
@@ -398,7 +444,7 @@ cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t smem = sizeof(Smem) + 1024;
+  const size_t smem = kEnd;  // absolute layout; the window starts at or below 1 KB
   auto kern = nf4_decode_kernel<EPI, OutT>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -78,6 +78,8 @@ typedef enum {
 #define MOE_DEVERR_BAD_OFFSETS 0x2 /* expert_offsets not monotone / total   */
 #define MOE_DEVERR_BAD_INDEX 0x4   /* a row or expert index out of range    */
 #define MOE_DEVERR_TIMEOUT 0x8     /* a bounded wait inside a kernel expired */
+#define MOE_DEVERR_LAYOUT 0x10     /* a kernel's shared-memory layout did not
+                                      fit this device; the call did no work */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_string(moe_status_t status);
