@@ -70,6 +70,26 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def recorded_traffic(kernel_source, workload):
+    """DRAM bytes per launch from profiles/kernel_traffic.txt, or None when the
+    kernel source changed since the capture (sha256 mismatch) or no capture
+    of this workload exists."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "kernel_traffic.txt")
+    src = os.path.join(ROOT, "bit_mixture_experts_route_b200", "csrc", kernel_source)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel_source \
+                    and parts[1] == sha and parts[2] == workload:
+                return float(parts[3])
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
 
@@ -376,11 +396,13 @@ def main():
     gu_bytes = sum(wl.gate_up_bytes(x) for x in d) / len(d)
     gu_flops = wl.gate_up_flops()
     prefill = T * shape.k >= 16 * shape.E
+    workload_key = f"{args.config}:T={T}"
     if prefill:
         achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
         peak = tf_burst
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak,
+                "traffic": recorded_traffic("grouped_gemm_tc.cu", workload_key),
                 "kernel": "grouped NF4 gate_up GEMM + SwiGLU",
                 "per_launch": f"{gu_flops:.4g} FLOP (2*T*k*H*2I)",
                 "peak_source": f"{peak_kind} bf16 dense"}
@@ -388,7 +410,8 @@ def main():
         achieved = gu_bytes / (gu_avg_ms / 1e3) / 1e9
         peak = hbm
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak,
+                "traffic": recorded_traffic("grouped_gemm_decode.cu", workload_key),
                 "kernel": "grouped NF4 gate_up GEMV + SwiGLU",
                 "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*0.5625 "
                               f"+ X + Hbuf)",
@@ -455,7 +478,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ncpu, aff, threads = cpu_cores()
-        n_tok = 16 if not prefill else 4
+        n_tok = min(T, 64) if not prefill else 16
         n, dt = oracle_sample(shape, T, args.seed, n_tok)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} tokens of layer 0 of this workload (NF4 experts dequantized, "
