@@ -161,11 +161,11 @@ moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows
   } else if (algo == MOE_ALGO_GEMV) {
     use_tc = false;
   } else {
-    // The tensor-core kernel decodes every weight once into shared memory
+    // The tensor-core kernel decodes every weight and issues every MMA
     // whatever the token count, so it only wins once experts average enough
     // rows to amortise that; on B200 both kernels take the same time at about
-    // 48 rows per expert on the OLMoE and Qwen3 shapes (gate_up and down).
-    use_tc = tc_ok && (int64_t)M_total >= 48LL * E;
+    // 36 rows per expert on the OLMoE and Qwen3 shapes (gate_up and down).
+    use_tc = tc_ok && (int64_t)M_total >= 36LL * E;
   }
   if (use_tc)
     return from_cuda(moe_launch::grouped_gemm_tc(A, a_dtype, A_rows, gather, k, packed, absmax,

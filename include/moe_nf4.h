@@ -222,7 +222,7 @@ moe_status_t moe_route_permute_noalloc(const float* logits, int T, int E, int k,
  * TC kernel (tcgen05): weights enter as fp16(fp16(level) * fp16(absmax));
  * it needs gather == NULL and F16 A (rows already permuted, e.g. by
  * moe_permute_rows), N % 128 == 0, absmax < 65504.  AUTO uses it when those
- * hold and M_total >= 48 * E.
+ * hold and M_total >= 36 * E.
  * All pointers 16-byte aligned.
  */
 moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype,
