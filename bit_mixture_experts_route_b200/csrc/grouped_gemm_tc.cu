@@ -72,6 +72,7 @@ static_assert(BSTAGES * B_STAGE + RAW_RING * RAW_STAGE + EPI_WARPS * STG_BYTES +
                       2 * 1025 * 4 + 1024 <
                   227 * 1024,
               "shared memory budget");
+static_assert(BSTAGES < RING, "activation slots are released through the TMEM-slot barriers");
 static_assert(RING % GROUPS == 0 && RAW_RING % GROUPS == 0,
               "a group always meets its own slots");
 
@@ -80,9 +81,10 @@ struct __align__(8) Smem {
   uint8_t raw[RAW_RING][RAW_STAGE];
   uint8_t stg[EPI_WARPS][STG_BYTES];
   uint32_t lut[256 * 32];
-  uint64_t full_b[BSTAGES], empty_b[BSTAGES];
   uint64_t raw_full[RAW_RING], raw_empty[RAW_RING];
-  uint64_t a_full[RING], a_empty[RING];
+  // ready[s]: stage s's decoded weights (four decoder-warp arrivals) and its
+  // activation tile (producer arrival + TMA bytes); a_empty[s]: its MMAs done
+  uint64_t ready[RING], a_empty[RING];
   uint64_t acc_full, acc_empty;
   uint32_t tmem_base;
   int abort_flag;
@@ -289,15 +291,13 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   // ---- setup: barriers, offsets, decode table, tile list, TMEM
   if (threadIdx.x == 0) {
     for (int s = 0; s < BSTAGES; ++s) {
-      mbar_init(&sm.full_b[s], 1);
-      mbar_init(&sm.empty_b[s], 1);
     }
     for (int s = 0; s < RAW_RING; ++s) {
       mbar_init(&sm.raw_full[s], 1);
       mbar_init(&sm.raw_empty[s], 4);   // the four warps of the decoding group
     }
     for (int s = 0; s < RING; ++s) {
-      mbar_init(&sm.a_full[s], 4);
+      mbar_init(&sm.ready[s], 4 + 1);
       mbar_init(&sm.a_empty[s], 1);     // MMA completion (tcgen05.commit)
     }
     mbar_init(&sm.acc_full, 1);
@@ -356,20 +356,27 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   if (warp == W_BPROD) {
     // ---------------- TMA producer: activation tiles, stage S of the CTA
     if (lane == 0) {
-      int bs = 0;
-      uint32_t bph = 0;
+      // slot S mod BSTAGES is free once the MMAs of stage S - BSTAGES are
+      // done; their completion is the a_empty barrier of that stage's TMEM
+      // slot (one commit per stage serves both rings)
+      int bs = 0, S = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const TileInfo ti = tile_info(sm, E, n_tiles, t);
         const int nmma = (ti.nrows + 15) & ~15;
         const int boxes = (nmma + B_BOX_ROWS - 1) / B_BOX_ROWS;
-        for (int ks = 0; ks < KT; ++ks) {
-          if (!(ok = mbar_wait(&sm.empty_b[bs], bph ^ 1, sm, dev_err))) break;
-          mbar_arrive_expect_tx(&sm.full_b[bs], boxes * B_BOX_ROWS * BK * 2);
+        for (int ks = 0; ks < KT; ++ks, ++S) {
+          if (S >= BSTAGES) {
+            const int P = S - BSTAGES;
+            if (!(ok = mbar_wait(&sm.a_empty[P % RING], (uint32_t)(P / RING) & 1u, sm, dev_err)))
+              break;
+          }
+          uint64_t* rdy = &sm.ready[S % RING];
+          mbar_arrive_expect_tx(rdy, boxes * B_BOX_ROWS * BK * 2);
           for (int b = 0; b < boxes; ++b)
-            tma_load_2d(sm.b[bs] + b * (B_BOX_ROWS * BK * 2), &bmap, &sm.full_b[bs], ks * BK,
+            tma_load_2d(sm.b[bs] + b * (B_BOX_ROWS * BK * 2), &bmap, rdy, ks * BK,
                         ti.row0 + b * B_BOX_ROWS);
-          if (++bs == BSTAGES) { bs = 0; bph ^= 1; }
+          if (++bs == BSTAGES) bs = 0;
         }
       }
     }
@@ -378,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     if (lane == 0) {
       const uint64_t bdesc0 = sw128_desc(smem_u32(sm.b[0]));
       int bs = 0, as = 0;
-      uint32_t bph = 0, aph = 0;
+      uint32_t aph = 0;
       bool ok = true;
       int lt = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
@@ -390,8 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         const uint32_t idesc = idesc_f16(nmma);
         const uint32_t dcol = tmem_base + ACC_COL;
         for (int ks = 0; ks < KT; ++ks) {
-          if (!(ok = mbar_wait(&sm.a_full[as], aph, sm, dev_err))) break;
-          if (!(ok = mbar_wait(&sm.full_b[bs], bph, sm, dev_err))) break;
+          if (!(ok = mbar_wait(&sm.ready[as], aph, sm, dev_err))) break;
           tc_fence_after();
           // K slice kk: 8 more TMEM columns of A; 32 bytes further into the
           // swizzled activation rows (+2 in the descriptor's address field)
@@ -401,9 +407,8 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
           mma_ts(dcol, acol + 8, bd + 2, idesc, 1u);
           mma_ts(dcol, acol + 16, bd + 4, idesc, 1u);
           mma_ts(dcol, acol + 24, bd + 6, idesc, 1u);
-          mma_commit(&sm.empty_b[bs]);
-          mma_commit(&sm.a_empty[as]);
-          if (++bs == BSTAGES) { bs = 0; bph ^= 1; }
+          mma_commit(&sm.a_empty[as]);  // frees TMEM slot as and activation slot bs
+          if (++bs == BSTAGES) bs = 0;
           if (++as == RING) { as = 0; aph ^= 1; }
         }
         if (ok) mma_commit(&sm.acc_full);
@@ -445,33 +450,36 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     const int rrow = (EPI == MOE_EPI_SWIGLU) ? ((m & 1) ? BM / 2 + (m >> 1) : (m >> 1)) : m;
     const uint32_t* lut = sm.lut + lane;
     const uint32_t tlane = tmem_base + ((uint32_t)(32 * q) << 16);
-    // absmax of own stage S: block ks of this thread's weight row in the tile
-    int c_tl = -1, c_expert = 0, c_ntile = 0;
-    auto absmax_of = [&](int S, float& a) -> bool {
-      const int tl = S / KT, ks = S - tl * KT;
-      const int t = blockIdx.x + tl * gridDim.x;
-      if (t >= total) return false;
-      if (tl != c_tl) {
-        const TileId id = tile_id(sm, E, n_tiles, t);
-        c_tl = tl; c_expert = id.expert; c_ntile = id.ntile;
-      }
+    // absmax of this thread's weight row, block ks of tile t (null past the
+    // CTA's last tile); walked one own stage ahead without divisions
+    auto row_absmax = [&](int t) -> const float* {
+      if (t >= total) return nullptr;
+      const TileId id = tile_id(sm, E, n_tiles, t);
       int row;
       if (EPI == MOE_EPI_SWIGLU) {
-        const int j = c_ntile * (BM / 2) + (m >> 1);
+        const int j = id.ntile * (BM / 2) + (m >> 1);
         row = (m & 1) ? (N / 2 + j) : j;
       } else {
-        row = c_ntile * BM + m;
+        row = id.ntile * BM + m;
       }
-      a = __ldg(absmax + ((size_t)c_expert * N + row) * (size_t)KT + ks);
-      return true;
+      return absmax + ((size_t)id.expert * N + row) * (size_t)KT;
     };
-    float a_cur = 0.0f;
-    bool have = absmax_of(g, a_cur);
+    int n_ks = g, n_t = blockIdx.x;
+    while (n_ks >= KT) { n_ks -= KT; n_t += gridDim.x; }
+    const float* n_row = row_absmax(n_t);
+    float a_cur = n_row ? __ldg(n_row + n_ks) : 0.0f;
+    bool have = n_row != nullptr;
     for (int S = g; have; S += GROUPS) {
       const int slot = S % RING, rslot = S % RAW_RING;
       const uint32_t ph = (uint32_t)(S / RING) & 1u, rph = (uint32_t)(S / RAW_RING) & 1u;
-      float a_next = 0.0f;
-      const bool have_next = absmax_of(S + GROUPS, a_next);  // one stage ahead
+      n_ks += GROUPS;
+      while (n_ks >= KT && n_row) {
+        n_ks -= KT;
+        n_t += gridDim.x;
+        n_row = row_absmax(n_t);
+      }
+      const bool have_next = n_row != nullptr;
+      const float a_next = have_next ? __ldg(n_row + n_ks) : 0.0f;  // one stage ahead
       // warp-uniform outcomes: tcgen05.st below is .aligned
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[rslot], rph, sm, dev_err))) break;
       const uint8_t* rp = sm.raw[rslot] + rrow * (BK / 2);
@@ -499,7 +507,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sm.a_full[slot]);
+        mbar_arrive(&sm.ready[slot]);
         mbar_arrive(&sm.raw_empty[rslot]);  // its bytes are decoded
       }
       a_cur = a_next;
