@@ -67,6 +67,31 @@ def test_tc_grouped_gemm_ragged(epi, counts):
     assert_close(_np(out), ref, f"tc {epi}")
 
 
+@pytest.mark.parametrize("K", [64, 192, 320])
+def test_tc_short_and_odd_k(K):
+    # K / 64 k-stages per tile: 1 (fewer than the four decoder groups), 3 and
+    # 5 (odd, so a group's stages straddle tile boundaries)
+    E, N = 3, 256
+    counts = np.array([5, 0, 40])
+    off = _ragged(E, counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(K)
+    W = torch.randn((E, N, K), generator=g) * 0.05
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    p, a = moe.nf4_quantize(W.cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for epi in ("none", "swiglu"):
+        out = moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
+                                   out_dtype=torch.float32, algo="tc", dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        pr, ar = oracle.quantize_blockwise(W.numpy())
+        ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
+        if epi == "swiglu":
+            ref = oracle.swiglu(ref)
+        assert_close(_np(out), ref, f"tc K={K} {epi}")
+
+
 def test_tc_matches_gemv_closely():
     E, N, K = 4, 256, 512
     counts = np.array([40, 300, 0, 97])
