@@ -519,7 +519,6 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     const int ew = warp - W_EPI;
     const int q = warp & 3;       // consecutive warps cover every lane quarter
     const int hc = ew >> 2;       // which 32 of each 64 columns
-    const int m = 32 * q + lane;
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint8_t* stg = sm.stg[ew];
     // a staged row: 16 outputs (SwiGLU pairs) or 32 (plain) of one token
