@@ -47,7 +47,7 @@ CONFIGS = {
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", choices=sorted(CONFIGS), default="olmoe-decode")
@@ -91,30 +91,40 @@ def recorded_traffic(kernel_source, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks / throttle reasons every 20 ms.  Each sample carries
+    nvidia-smi's own timestamp; only samples taken between mark_start() and
+    mark_end() (the timed region) enter the summary."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.6)  # nvidia-smi's start-up, before the timed region
         except OSError:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *exc):
         self.lines = []
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
@@ -123,25 +133,43 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
+    @staticmethod
+    def _stamp(text):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(text, fmt).timestamp()
+            except ValueError:
+                continue
+        return None
+
     def summary(self):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        outside = 0
         for ln in getattr(self, "lines", []):
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
+                continue
+            ts = self._stamp(parts[0])
+            if self.t0 is not None and ts is not None and not (
+                    self.t0 - 0.02 <= ts <= (self.t1 or ts) + 0.02):
+                outside += 1
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                sm.append(float(parts[2]))
+                smax = float(parts[3])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
+            for nm, val in zip(names, parts[6:10]):
                 if val.lower() == "active":
                     reasons.add(nm)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "samples_outside_timed_region": outside}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "samples_outside_timed_region": outside}
 
 
 def dist_setup():
@@ -378,11 +406,13 @@ def main():
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
+        clk.mark_start()
         start.record(stream)
         for s in range(args.steps):
             wl.step(args.algo, evs[s])
         end.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         barrier(world)
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
     ms_per_step = elapsed_ms / args.steps
@@ -395,7 +425,9 @@ def main():
     d_avg = sum(d) / len(d)
     gu_bytes = sum(wl.gate_up_bytes(x) for x in d) / len(d)
     gu_flops = wl.gate_up_flops()
-    prefill = T * shape.k >= 16 * shape.E
+    # the tensor-core kernel serves the GEMMs from 36 routed rows per expert
+    # on average (the AUTO dispatch rule); below that the decode GEMV does
+    prefill = T * shape.k >= 36 * shape.E
     workload_key = f"{args.config}:T={T}"
     if prefill:
         achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
@@ -481,9 +513,18 @@ def main():
         n_tok = min(T, 64) if not prefill else 16
         n, dt = oracle_sample(shape, T, args.seed, n_tok)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "blas_threads": threads,
                "sample": f"{n} tokens of layer 0 of this workload (NF4 experts dequantized, "
                          f"per-token fp64 expert MLPs); host cpu_count={ncpu}, "
                          f"affinity={aff}; {dt:.1f} s"}
+        try:  # the same oracle on one thread, on a quarter of the tokens
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                n1, dt1 = oracle_sample(shape, T, args.seed, max(2, n_tok // 4))
+            cpu["value_1thread"] = n1 / dt1
+            cpu["sample"] += f"; 1-thread run: {n1} tokens in {dt1:.1f} s"
+        except ImportError:
+            pass
 
     launches_per_layer = 6  # route_tile, permute_scatter, permute_rows, gate_up, down, combine
     line = {

@@ -284,14 +284,37 @@ def test_layer_olmoe_decode(T):
     _layer_parity(moe_synth.OLMOE, T, 0)
 
 
+def test_layer_olmoe_decode_last_layer():
+    # layer 15 of the 16-layer decode stack (its own weights and logits)
+    _layer_parity(moe_synth.OLMOE, 16, 15)
+
+
 def test_layer_qwen3_30b_decode():
     _layer_parity(moe_synth.QWEN3_30B, 64, 1)
 
 
+def test_layer_qwen3_30b_decode_last_layer():
+    # layer 47 of the 48-layer decode stack
+    _layer_parity(moe_synth.QWEN3_30B, 8, 47)
+
+
 def test_layer_qwen3_30b_prefill_sampled():
+    # 256 seeded tokens of 4096 (Zipf routing: 0 to ~1500 rows per expert,
+    # empty experts included; the grouped GEMMs run on the tensor cores)
     rng = np.random.default_rng(0)
-    toks = sorted(rng.choice(4096, size=48, replace=False).tolist())
+    toks = sorted(rng.choice(4096, size=256, replace=False).tolist())
     _layer_parity(moe_synth.QWEN3_30B, 4096, 2, tokens=toks)
+
+
+def test_layer_qwen3_235b_decode():
+    # hidden 4096, moe_intermediate 1536, 0.1 % of the weights at 8 sigma
+    _layer_parity(moe_synth.QWEN3_235B, 1, 3)
+
+
+def test_layer_qwen3_235b_prefill_sampled():
+    rng = np.random.default_rng(1)
+    toks = sorted(rng.choice(2048, size=4, replace=False).tolist())
+    _layer_parity(moe_synth.QWEN3_235B, 2048, 5, tokens=toks)
 
 
 def test_layer_single_expert_dense():
