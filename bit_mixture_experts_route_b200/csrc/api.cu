@@ -10,12 +10,9 @@ namespace {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status_t check_device() {
-  int dev = 0, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return (major == 10 && minor == 0) ? MOE_OK : MOE_ERR_UNSUPPORTED;
+  moe::DeviceInfo d;
+  if (!moe::device_info(&d)) return MOE_ERR_CUDA;
+  return (d.major == 10 && d.minor == 0) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
 // The CUDA error behind the calling thread's most recent MOE_ERR_CUDA.

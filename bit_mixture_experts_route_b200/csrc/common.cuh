@@ -9,7 +9,11 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <string>
 #include <type_traits>
+#include <unordered_map>
 
 #include "../../include/moe_nf4.h"
 
@@ -114,6 +118,98 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   }();
   return fn;
+}
+
+// A tensor map depends only on its arguments (address, sizes, strides, box,
+// swizzle, promotion, fill), so each distinct map is encoded once and reused:
+// a launch then costs a hash lookup instead of a driver call.  Same signature
+// and results as cuTensorMapEncodeTiled.
+inline CUresult encode_tiled_cached(CUtensorMap* out, CUtensorMapDataType dt, cuuint32_t rank,
+                                    void* addr, const cuuint64_t* dims,
+                                    const cuuint64_t* strides, const cuuint32_t* box,
+                                    const cuuint32_t* estr, CUtensorMapInterleave il,
+                                    CUtensorMapSwizzle sw, CUtensorMapL2promotion l2,
+                                    CUtensorMapFloatOOBfill oob) {
+  const auto enc = tensor_map_encoder();
+  if (!enc || rank < 1 || rank > 5) return CUDA_ERROR_NOT_SUPPORTED;
+  uint64_t key[24] = {};
+  int n = 0;
+  key[n++] = (uint64_t)dt;
+  key[n++] = rank;
+  key[n++] = (uint64_t)(uintptr_t)addr;
+  for (cuuint32_t i = 0; i < rank; ++i) key[n++] = dims[i];
+  for (cuuint32_t i = 0; i + 1 < rank; ++i) key[n++] = strides[i];
+  for (cuuint32_t i = 0; i < rank; ++i) key[n++] = ((uint64_t)box[i] << 32) | estr[i];
+  key[n++] = ((uint64_t)il << 48) | ((uint64_t)sw << 32) | ((uint64_t)l2 << 16) | (uint64_t)oob;
+  const std::string k(reinterpret_cast<const char*>(key), n * sizeof(uint64_t));
+  static std::mutex mu;
+  static std::unordered_map<std::string, CUtensorMap> cache;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(k);
+    if (it != cache.end()) {
+      *out = it->second;
+      return CUDA_SUCCESS;
+    }
+  }
+  const CUresult r = enc(out, dt, rank, addr, dims, strides, box, estr, il, sw, l2, oob);
+  if (r == CUDA_SUCCESS) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 4096) cache.clear();
+    cache.emplace(k, *out);
+  }
+  return r;
+}
+
+// Compute capability and SM count of the current device, queried once per
+// device.
+struct DeviceInfo {
+  int major, minor, sms;
+};
+inline bool device_info(DeviceInfo* out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static DeviceInfo info[kMaxDevices];
+  static bool known[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!known[dev]) {
+    DeviceInfo d{};
+    if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    info[dev] = d;
+    known[dev] = true;
+  }
+  *out = info[dev];
+  return true;
+}
+inline int device_sm_count() {
+  DeviceInfo d;
+  return device_info(&d) ? d.sms : 148;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device.
+inline cudaError_t set_max_dynamic_smem_once(const void* kern, int bytes) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;  // device bitmask
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const uint64_t bit = 1ull << (dev & 63);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = done.find(kern);
+    if (it != done.end() && (it->second & bit)) return cudaSuccess;
+  }
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    done[kern] |= bit;
+  }
+  return err;
 }
 
 }  // namespace moe

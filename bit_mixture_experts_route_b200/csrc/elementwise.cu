@@ -123,12 +123,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict
   }
 }
 
-int sm_count() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
+int sm_count() { return device_sm_count(); }
 
 template <typename InT>
 cudaError_t swiglu_out(const InT* gu, int M, int I, void* h, moe_dtype_t h_dt, cudaStream_t s) {

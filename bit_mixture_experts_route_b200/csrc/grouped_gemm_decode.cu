@@ -400,19 +400,14 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
   __syncthreads();
 }
 
-int sm_count() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
+int sm_count() { return device_sm_count(); }
 
 template <int EPI, typename OutT>
 cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
                    const int32_t* offsets, int E, int N, int K, int M_total, void* out,
                    int32_t* dev_err, cudaStream_t s) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  const auto enc = encode_tiled_cached;
   CUtensorMap wmap, amap, xmap;
   const cuuint32_t estr[2] = {1, 1};
   {
@@ -446,8 +441,7 @@ cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float
   }
   const size_t smem = kEnd;  // absolute layout; the window starts at or below 1 KB
   auto kern = nf4_decode_kernel<EPI, OutT>;
-  cudaError_t err =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
   const int64_t max_items = ((int64_t)M_total / TOK + E) * (N / ROWS);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_items));

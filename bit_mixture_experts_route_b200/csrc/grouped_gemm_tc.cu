@@ -599,19 +599,14 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   }
 }
 
-int sm_count() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
+int sm_count() { return device_sm_count(); }
 
 template <int EPI, typename OutT>
 cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
                    const int32_t* offsets, int E, int N, int K, int M_total, void* out,
                    int32_t* dev_err, cudaStream_t s) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  const auto enc = encode_tiled_cached;
   CUtensorMap map, wmap;
   const cuuint32_t estr[2] = {1, 1};
   {
@@ -637,8 +632,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
   }
   const size_t smem = sizeof(Smem) + 1024;
   auto kern = nf4_tc_kernel<EPI, OutT>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
   // Upper bound on tiles: every expert's rows rounded up to BN, plus one
   // partial tile per expert; the kernel derives the exact list itself.

@@ -104,9 +104,7 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
 }
 
 int grid_for(int64_t threads) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   int64_t blocks = (threads + 255) / 256;
   const int64_t cap = (int64_t)sms * 8;
   return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
