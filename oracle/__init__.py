@@ -19,6 +19,10 @@ Sources (web pages on the method, cited by page title and section):
 * The problem statement of this library fixes the rest: blocksize 64, fp32
   absmax, two codes per byte, top-k softmax routing, SiLU(gate)*up, a
   routing-weighted combine.
+* The same pages mention GPTQ-calibrated int4 experts served by an INT4
+  decode GEMV ("grouped-nf4-gemm & experts-4bit", third bullet; "MoE Training
+  on Consumer GPUs", cerinamroth.com/ml, section "Task guides");
+  ``oracle.int4`` states the format readings.
 
 Where the pages are silent the oracle takes one reading, documented at each
 function.  Every function is pinned by tests in ``tests/test_oracle_*.py``
@@ -38,10 +42,17 @@ from .nf4 import (  # noqa: F401
     dequantize_blockwise,
     unpack_codes,
 )
+from .int4 import (  # noqa: F401
+    GROUP as INT4_GROUP,
+    quantize_int4_grouped,
+    dequantize_int4_grouped,
+    int4_scales_zeros,
+)
 from .routing import route_topk, permute_by_expert  # noqa: F401
 from .moe import (  # noqa: F401
     swiglu,
     grouped_gemm,
+    grouped_gemm_int4,
     unpermute_combine,
     moe_layer,
     moe_layer_dense,

@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from .int4 import dequantize_int4_grouped
 from .nf4 import dequantize_blockwise
 from .routing import route_topk, permute_by_expert
 
@@ -73,6 +74,25 @@ def swiglu(gu: np.ndarray) -> np.ndarray:
     return _silu(gu[:, :I]) * gu[:, I:]
 
 
+def _grouped(A, weight_of, N: int, expert_offsets, gather, k: int, rows) -> np.ndarray:
+    """``out[p] = W(e(p)) @ A[r(p)]`` for the positions p of a grouped GEMM;
+    ``weight_of(e)`` returns expert e's dequantized ``[N, K]`` weights."""
+    A = np.asarray(A, dtype=np.float64)
+    offsets = np.asarray(expert_offsets, dtype=np.int64)
+    M_total = int(offsets[-1])
+    positions = np.arange(M_total) if rows is None else np.asarray(rows)
+    out = np.zeros((positions.size, N), dtype=np.float64)
+    experts = np.searchsorted(offsets, positions, side="right") - 1
+    cache = {}
+    for i, p in enumerate(positions):
+        e = int(experts[i])
+        if e not in cache:
+            cache[e] = weight_of(e)
+        r = int(gather[p]) // k if gather is not None else int(p)
+        out[i] = cache[e] @ A[r]
+    return out
+
+
 def grouped_gemm(A: np.ndarray, packed: np.ndarray, absmax: np.ndarray,
                  expert_offsets: np.ndarray, gather=None, k: int = 1,
                  rows=None) -> np.ndarray:
@@ -84,21 +104,19 @@ def grouped_gemm(A: np.ndarray, packed: np.ndarray, absmax: np.ndarray,
     ``rows`` optionally restricts the result to those positions (returned in
     that order).  fp64 result ``[len(rows) or M_total, N]``.
     """
-    A = np.asarray(A, dtype=np.float64)
-    offsets = np.asarray(expert_offsets, dtype=np.int64)
     E, N, half_k = packed.shape
-    M_total = int(offsets[-1])
-    positions = np.arange(M_total) if rows is None else np.asarray(rows)
-    out = np.zeros((positions.size, N), dtype=np.float64)
-    experts = np.searchsorted(offsets, positions, side="right") - 1
-    cache = {}
-    for i, p in enumerate(positions):
-        e = int(experts[i])
-        if e not in cache:
-            cache[e] = dequantize_blockwise(packed[e], absmax[e].reshape(N, -1))
-        r = int(gather[p]) // k if gather is not None else int(p)
-        out[i] = cache[e] @ A[r]
-    return out
+    return _grouped(A, lambda e: dequantize_blockwise(packed[e], absmax[e].reshape(N, -1)), N,
+                    expert_offsets, gather, k, rows)
+
+
+def grouped_gemm_int4(A: np.ndarray, packed: np.ndarray, meta: np.ndarray,
+                      expert_offsets: np.ndarray, gather=None, k: int = 1,
+                      rows=None) -> np.ndarray:
+    """The same grouped GEMM on grouped INT4 weights (``oracle.int4``):
+    ``packed uint8[E, N, K/2]``, ``meta uint32[E, N, K/128]``."""
+    E, N, half_k = packed.shape
+    return _grouped(A, lambda e: dequantize_int4_grouped(packed[e], meta[e]), N, expert_offsets,
+                    gather, k, rows)
 
 
 def unpermute_combine(Yp: np.ndarray, inv_perm: np.ndarray,
