@@ -54,6 +54,8 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=None, help="token batch T")
     p.add_argument("--layers", type=int, default=None)
     p.add_argument("--algo", choices=["auto", "gemv", "tc"], default="auto")
+    p.add_argument("--weights", choices=["nf4", "int4"], default="nf4",
+                   help="expert weight format (int4: grouped GPTQ-style codes, decode GEMV)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
@@ -212,18 +214,20 @@ def rank_seed(seed, rank):
 # ----------------------------------------------------------------- workload
 
 class Workload:
-    def __init__(self, shape, T, layers, seed, device="cuda"):
+    def __init__(self, shape, T, layers, seed, device="cuda", weights="nf4"):
         import bit_mixture_experts_route_b200 as moe
         self.moe = moe
         self.shape, self.T, self.L = shape, T, layers
+        self.int4 = weights == "int4"
+        quantize = moe.int4_quantize if self.int4 else moe.nf4_quantize
         self.stacks = []
         for layer in range(layers):
             s = seed * 1000 + layer
             w = moe_synth.weights(shape, "gate_up", s, device=device)
-            p_gu, a_gu = moe.nf4_quantize(w)
+            p_gu, a_gu = quantize(w)
             del w
             w = moe_synth.weights(shape, "down", s, device=device)
-            p_d, a_d = moe.nf4_quantize(w)
+            p_d, a_d = quantize(w)
             del w
             self.stacks.append((p_gu, a_gu, p_d, a_d))
         torch.cuda.empty_cache()
@@ -249,21 +253,30 @@ class Workload:
         self.lws = torch.empty((max(moe.layer_workspace_size(T, E, k, H, I), 256),),
                                dtype=torch.uint8, device=dev)
 
-    def layer(self, layer, algo="auto", ev=None):
+    def layer(self, layer, algo="auto", ev=None, X=None, logits=None):
         moe, sh, T = self.moe, self.shape, self.T
+        X = self.X if X is None else X
+        logits = self.logits[layer] if logits is None else logits
         p_gu, a_gu, p_d, a_d = self.stacks[layer]
-        r = moe.route_permute(self.logits[layer], sh.k, sh.renormalize, workspace=self.rws,
-                              out=self.route)
+        r = moe.route_permute(logits, sh.k, sh.renormalize, workspace=self.rws, out=self.route)
         M = T * sh.k
-        moe.permute_rows(self.X, r["sorted_rows"], sh.k, out=self.Xp)
+        moe.permute_rows(X, r["sorted_rows"], sh.k, out=self.Xp)
         if ev is not None:
             ev[0].record()
-        moe.nf4_grouped_gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, epilogue="swiglu",
-                             out=self.Hbuf, algo=algo)
+        if self.int4:
+            moe.int4_grouped_gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, epilogue="swiglu",
+                                  out=self.Hbuf)
+        else:
+            moe.nf4_grouped_gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, epilogue="swiglu",
+                                 out=self.Hbuf, algo=algo)
         if ev is not None:
             ev[1].record()
-        moe.nf4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
-                             out=self.Yp, algo=algo)
+        if self.int4:
+            moe.int4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
+                                  out=self.Yp)
+        else:
+            moe.nf4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
+                                 out=self.Yp, algo=algo)
         moe.unpermute_combine(self.Yp, r["inv_perm"], r["topk_w"], out=self.Y)
 
     def step(self, algo="auto", evs=None):
@@ -282,7 +295,9 @@ class Workload:
 
     def gate_up_bytes(self, d):
         sh, T = self.shape, self.T
-        w = d * (2 * sh.I * sh.H) * 0.5625
+        # per weight: 4-bit code + fp32 absmax per 64 (NF4) or fp16 scale and
+        # zero in 4 bytes per 128 (INT4)
+        w = d * (2 * sh.I * sh.H) * (0.53125 if self.int4 else 0.5625)
         return w + T * sh.H * 2 + T * sh.k * sh.I * 2
 
     def layer_bytes(self, d):
@@ -296,10 +311,11 @@ class Workload:
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(shape, T, seed, n_tokens, start_token=0, threads=None):
+def oracle_sample(shape, T, seed, n_tokens, start_token=0, threads=None, weights="nf4"):
     """Time the oracle on ``n_tokens`` tokens of layer 0: dequantize the NF4
-    experts they need and run the per-token expert MLPs.  Weights come from
-    the same generator as the GPU run; quantization is untimed setup."""
+    (or INT4) experts they need and run the per-token expert MLPs.  Weights
+    come from the same generator as the GPU run; quantization is untimed
+    setup."""
     import oracle
     s = seed * 1000
     X = moe_synth.activations(T, shape.H, seed).float().numpy()
@@ -311,6 +327,18 @@ def oracle_sample(shape, T, seed, n_tokens, start_token=0, threads=None):
     w_gu = moe_synth.weights(shape, "gate_up", s, experts=experts, device=dev).cpu().numpy()
     w_d = moe_synth.weights(shape, "down", s, experts=experts, device=dev).cpu().numpy()
     E, I, H = shape.E, shape.I, shape.H
+    if weights == "int4":
+        p_gu = np.zeros((E, 2 * I, H // 2), np.uint8)
+        m_gu = np.zeros((E, 2 * I, H // 128), np.uint32)
+        p_d = np.zeros((E, H, I // 2), np.uint8)
+        m_d = np.zeros((E, H, I // 128), np.uint32)
+        for i, e in enumerate(experts):
+            p_gu[e], m_gu[e] = oracle.quantize_int4_grouped(w_gu[i])
+            p_d[e], m_d[e] = oracle.quantize_int4_grouped(w_d[i])
+        stack = oracle.Int4ExpertStack(p_gu, m_gu, p_d, m_d)
+        t0 = time.perf_counter()
+        oracle.moe_layer(X, lg, stack, shape.k, shape.renormalize, tokens=toks)
+        return n_tokens, time.perf_counter() - t0
     p_gu = np.zeros((E, 2 * I, H // 2), np.uint8)
     a_gu = np.zeros((E, 2 * I * H // 64), np.float32)
     p_d = np.zeros((E, H, I // 2), np.uint8)
@@ -390,7 +418,10 @@ def main():
     world, rank, local = dist_setup()
     import bit_mixture_experts_route_b200 as moe
     moe.load()
-    wl = Workload(shape, T, layers, rank_seed(args.seed, rank))
+    wl = Workload(shape, T, layers, rank_seed(args.seed, rank), weights=args.weights)
+    if args.weights == "int4" and T * shape.k >= 36 * shape.E:
+        raise SystemExit("int4 weights have the decode GEMV path only (fewer than 36 routed "
+                         "rows per expert)")
     hbm, tf_burst, tf_sust, peak_kind = load_peaks()
     stream = torch.cuda.current_stream()
 
@@ -428,7 +459,8 @@ def main():
     # the tensor-core kernel serves the GEMMs from 36 routed rows per expert
     # on average (the AUTO dispatch rule); below that the decode GEMV does
     prefill = T * shape.k >= 36 * shape.E
-    workload_key = f"{args.config}:T={T}"
+    workload_name = args.config + ("/int4" if args.weights == "int4" else "")
+    workload_key = f"{workload_name}:T={T}"
     if prefill:
         achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
         peak = tf_burst
@@ -443,10 +475,12 @@ def main():
         peak = hbm
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak,
-                "traffic": recorded_traffic("grouped_gemm_decode.cu", workload_key),
-                "kernel": "grouped NF4 gate_up GEMV + SwiGLU",
-                "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*0.5625 "
-                              f"+ X + Hbuf)",
+                "traffic": recorded_traffic(
+                    "grouped_gemm_int4.cu" if args.weights == "int4" else "grouped_gemm_decode.cu",
+                    workload_key),
+                "kernel": f"grouped {args.weights.upper()} gate_up GEMV + SwiGLU",
+                "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*"
+                              f"{0.53125 if args.weights == 'int4' else 0.5625} + X + Hbuf)",
                 "peak_source": f"{peak_kind} HBM copy"}
 
     # ---- the same step as one CUDA graph (how a decode server replays it):
@@ -500,8 +534,11 @@ def main():
         X_d.copy_(X_h, non_blocking=True)
         L_d.copy_(L_h, non_blocking=True)
         for layer in range(layers):
-            moe.layer_forward(X_d, L_d[layer], shape.k, shape.renormalize, *wl.stacks[layer],
-                              workspace=wl.lws, out=wl.Y)
+            if wl.int4:  # the five calls through the binding, on the copied inputs
+                wl.layer(layer, args.algo, X=X_d, logits=L_d[layer])
+            else:
+                moe.layer_forward(X_d, L_d[layer], shape.k, shape.renormalize,
+                                  *wl.stacks[layer], workspace=wl.lws, out=wl.Y)
         Y_h.copy_(wl.Y, non_blocking=True)
 
     for _ in range(3):
@@ -523,7 +560,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ncpu, aff, threads = cpu_cores()
         n_tok = min(T, 64) if not prefill else 16
-        n, dt = oracle_sample(shape, T, args.seed, n_tok)
+        n, dt = oracle_sample(shape, T, args.seed, n_tok, weights=args.weights)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "blas_threads": threads,
                "sample": f"{n} tokens of layer 0 of this workload (NF4 experts dequantized, "
@@ -532,7 +569,8 @@ def main():
         try:  # the same oracle on one thread, on a quarter of the tokens
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
-                n1, dt1 = oracle_sample(shape, T, args.seed, max(2, n_tok // 4))
+                n1, dt1 = oracle_sample(shape, T, args.seed, max(2, n_tok // 4),
+                                        weights=args.weights)
             cpu["value_1thread"] = n1 / dt1
             cpu["sample"] += f"; 1-thread run: {n1} tokens in {dt1:.1f} s"
         except ImportError:
@@ -550,9 +588,9 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": args.config, "T": T, "layers": layers, "E": shape.E,
+        "config": {"workload": workload_name, "T": T, "layers": layers, "E": shape.E,
                    "k": shape.k, "hidden": shape.H, "intermediate": shape.I,
-                   "renormalize": shape.renormalize, "routing": shape.routing,
+                   "weights": args.weights, "renormalize": shape.renormalize, "routing": shape.routing,
                    "value_counts": "layer-tokens: T tokens through each of the layers",
                    "l2": f"inputs larger than L2: {layers} layers x "
                          f"{shape.E * shape.nf4_bytes_per_expert / 1e6:.0f} MB NF4 weights",

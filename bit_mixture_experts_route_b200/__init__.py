@@ -18,6 +18,8 @@ from ._lib import (  # noqa: F401
     route_permute_workspace_size,
     route_permute,
     nf4_grouped_gemm,
+    int4_quantize,
+    int4_grouped_gemm,
     permute_rows,
     swiglu,
     unpermute_combine,

@@ -40,6 +40,8 @@ SIGNATURES = {
     "moe_route_permute_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _S]),
     "moe_nf4_grouped_gemm": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                   _I, _I, _P, _S]),
+    "moe_int4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
+    "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
     "moe_permute_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _S]),
     "moe_swiglu": (_I, [_P, _I, _I, _I, _P, _I, _S]),
     "moe_unpermute_combine": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _S]),
@@ -182,6 +184,42 @@ def nf4_grouped_gemm(A, packed, absmax, expert_offsets, M_total, gather=None, k=
         _ptr(A), DT[A.dtype], A.shape[0], _ptr(gather), k, _ptr(packed), _ptr(absmax),
         _ptr(expert_offsets), E, N, K, M_total, EPI[epilogue], _ptr(out), DT[out.dtype],
         ALGO[algo], _ptr(dev_err), _stream(A.device)), "moe_nf4_grouped_gemm")
+    return out
+
+
+def int4_quantize(W, packed=None, meta=None, dev_err=None):
+    """``W fp32 [E, N, K]`` -> ``(packed u8 [E, N, K/2], meta u32-as-int32
+    [E, N, K/128])``: grouped INT4 codes, per 128-group fp16 scale | zero << 16."""
+    _need(W, torch.float32, "W", 3)
+    E, N, K = W.shape
+    if packed is None:
+        packed = torch.empty((E, N, K // 2), dtype=torch.uint8, device=W.device)
+    if meta is None:
+        meta = torch.empty((E, N, K // 128), dtype=torch.int32, device=W.device)
+    _check(load().moe_int4_quantize(_ptr(W), E, N, K, _ptr(packed), _ptr(meta), _ptr(dev_err),
+                                    _stream(W.device)), "moe_int4_quantize")
+    return packed, meta
+
+
+def int4_grouped_gemm(A, packed, meta, expert_offsets, M_total, epilogue="none",
+                      out_dtype=torch.float32, out=None, dev_err=None):
+    """Decode-shaped grouped GEMM on INT4 weights, all experts in one launch
+    (see the header); ``A`` fp16 rows in permuted order."""
+    _need(A, torch.float16, "A", 2)
+    _need(packed, torch.uint8, "packed", 3)
+    _need(meta, torch.int32, "meta", 3)
+    _need(expert_offsets, torch.int32, "expert_offsets", 1)
+    E, N, half = packed.shape
+    K = 2 * half
+    if A.shape[1] != K:
+        raise MoEError("A's columns must equal the weights' K")
+    n_out = N // 2 if epilogue == "swiglu" else N
+    if out is None:
+        out = torch.empty((M_total, n_out), dtype=out_dtype, device=A.device)
+    _check(load().moe_int4_grouped_gemm(
+        _ptr(A), A.shape[0], _ptr(packed), _ptr(meta), _ptr(expert_offsets), E, N, K, M_total,
+        EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
+        "moe_int4_grouped_gemm")
     return out
 
 

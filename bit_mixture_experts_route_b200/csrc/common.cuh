@@ -250,6 +250,13 @@ cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows,
                             moe_dtype_t out_dt, int32_t* dev_err,
                             cudaStream_t s);
 bool grouped_gemm_tc_supported(int N, int K, moe_epilogue_t epi);
+cudaError_t int4_quantize(const float* W, int64_t rows, int K, uint8_t* packed, uint32_t* meta,
+                          int32_t* dev_err, cudaStream_t s);
+bool grouped_gemm_int4_supported(int N, int K);
+cudaError_t grouped_gemm_int4(const void* A, int A_rows, const uint8_t* packed,
+                              const uint32_t* meta, const int32_t* offsets, int E, int N, int K,
+                              int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
+                              int32_t* dev_err, cudaStream_t s);
 cudaError_t permute_rows(const void* X, moe_dtype_t x_dt, int T, int K, const int32_t* rows,
                          int k, int M_total, void* Xp, int32_t* dev_err, cudaStream_t s);
 cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h,

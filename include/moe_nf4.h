@@ -125,6 +125,55 @@ moe_status_t moe_nf4_dequantize(const uint8_t* packed, const float* absmax,
                                 moe_dtype_t out_dtype, void* stream);
 
 /*
+ * moe_int4_quantize -- grouped INT4 quantization of a fused expert stack, the
+ * format of moe_int4_grouped_gemm.  ("grouped-nf4-gemm & experts-4bit",
+ * jordananderson-pages.pages.dev, third bullet: GPTQ-calibrated int4 experts
+ * served by an INT4 decode GEMV.  The pages fix no format; this one follows
+ * the GPTQ checkpoint convention.)
+ *
+ *   W       fp32   [E, N, K]      input weights (device, read only)
+ *   E, N, K >= 1, K % 128 == 0
+ *   packed  uint8  [E, N, K/2]    codes q, two per byte, element 2j of a row in
+ *                                 the high nibble of byte j (device)
+ *   meta    uint32 [E, N, K/128]  per group of 128 along K: fp16 bits of the
+ *                                 scale s | zero z << 16 (device)
+ *   dev_err int32 device word or NULL; MOE_DEVERR_NONFINITE if any weight is
+ *           NaN/Inf (its group's codes are then unspecified).
+ * Per group: lo = min(min x, 0), hi = max(max x, 0), s = fp16(fl32((hi-lo)/15)),
+ * z = clamp(rint(-lo/s), 0, 15), q = clamp(rint(x/s) + z, 0, 15) (IEEE fp32
+ * division, rint to nearest even); stored scale 0 -> z = 0, q = 0.  The value
+ * of a code is (q - z) * s.  Round-to-nearest, deterministic, bit-exact.
+ * W, packed and meta must be 16-byte aligned.
+ */
+moe_status_t moe_int4_quantize(const float* W, int E, int N, int K, uint8_t* packed,
+                               uint32_t* meta, int32_t* dev_err, void* stream);
+
+/*
+ * moe_int4_grouped_gemm -- decode-shaped grouped GEMM on INT4 weights:
+ * out[p] = W[e(p)] @ A[p] for every row p in expert e's segment
+ * [expert_offsets[e], expert_offsets[e+1]), W[e] = (q - z) * s from
+ * (packed, meta) as written by moe_int4_quantize, all experts in one launch.
+ *
+ *   A        fp16 [A_rows >= M_total, K]  routed rows in permuted order
+ *            (e.g. moe_permute_rows output); no gather
+ *   packed   uint8 [E, N, K/2], meta uint32 [E, N, K/128]
+ *   expert_offsets int32 [E+1] (device), monotone, offsets[E] == M_total
+ *   N % 128 == 0, K % 256 == 0, E <= 1024
+ *   epilogue MOE_EPI_NONE: out [M_total, N]; MOE_EPI_SWIGLU: rows [0, N/2)
+ *            are gate and [N/2, N) up, out [M_total, N/2] = silu(g) * u
+ *   out      F32 / F16 / BF16
+ *   dev_err  as moe_nf4_grouped_gemm (BAD_OFFSETS, TIMEOUT, LAYOUT)
+ * The weights enter the MMA as the exact integers q - z (fp16); each 64-k
+ * block's fp32 partial sum is scaled by its group's s.  Streams every
+ * selected expert's bytes once (HBM-bound at decode sizes).
+ * All pointers 16-byte aligned.
+ */
+moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
+                                   const uint32_t* meta, const int32_t* expert_offsets, int E,
+                                   int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
+                                   moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
+
+/*
  * Workspace bytes moe_route_permute needs for (T, E, k).  `bytes` is a HOST
  * pointer.  Host-only, no CUDA call.
  */

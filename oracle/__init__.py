@@ -58,4 +58,5 @@ from .moe import (  # noqa: F401
     moe_layer_dense,
     moe_layer_permuted,
     ExpertStack,
+    Int4ExpertStack,
 )

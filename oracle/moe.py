@@ -63,6 +63,34 @@ class ExpertStack:
         return self._d[e]
 
 
+class Int4ExpertStack:
+    """Grouped INT4 gate_up and down stacks of one layer (``oracle.int4``),
+    dequantized lazily per expert; same interface as ``ExpertStack``.
+
+    ``packed_gu uint8[E, 2I, H/2]``, ``meta_gu uint32[E, 2I, H/128]``,
+    ``packed_d uint8[E, H, I/2]``, ``meta_d uint32[E, H, I/128]``.
+    """
+
+    def __init__(self, packed_gu, meta_gu, packed_d, meta_d):
+        self.packed_gu, self.meta_gu = np.asarray(packed_gu, np.uint8), np.asarray(meta_gu)
+        self.packed_d, self.meta_d = np.asarray(packed_d, np.uint8), np.asarray(meta_d)
+        self.E, two_i, half_h = self.packed_gu.shape
+        self.I = two_i // 2
+        self.H = half_h * 2
+        assert self.packed_d.shape == (self.E, self.H, self.I // 2)
+        self._gu, self._d = {}, {}
+
+    def gate_up(self, e: int) -> np.ndarray:
+        if e not in self._gu:
+            self._gu[e] = dequantize_int4_grouped(self.packed_gu[e], self.meta_gu[e])
+        return self._gu[e]
+
+    def down(self, e: int) -> np.ndarray:
+        if e not in self._d:
+            self._d[e] = dequantize_int4_grouped(self.packed_d[e], self.meta_d[e])
+        return self._d[e]
+
+
 def _silu(g: np.ndarray) -> np.ndarray:
     return g / (1.0 + np.exp(-g))
 

@@ -119,3 +119,19 @@ def test_binding_fails_loudly_without_the_library(monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/libmoenf4.so")
     with pytest.raises(_lib.MoEError):
         _lib.load()
+
+
+def test_int4_calls_reject_bad_arguments(lib):
+    A, M = ALIGNED, MISALIGNED
+    # quantize: K % 128, null, misaligned
+    assert lib.moe_int4_quantize(A, 1, 8, 192, A, A, None, None) == 1
+    assert lib.moe_int4_quantize(None, 1, 8, 256, A, A, None, None) == 1
+    assert lib.moe_int4_quantize(A, 1, 8, 256, M, A, None, None) == 2
+    # grouped GEMM: N % 128 or K % 256 -> unsupported; bad epilogue / dtype;
+    # A_rows < M_total; misaligned output
+    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 64, 256, 8, 0, A, 0, None, None) == 3
+    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 384, 8, 0, A, 0, None, None) == 3
+    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 7, A, 0, None, None) == 1
+    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 9, None, None) == 1
+    assert lib.moe_int4_grouped_gemm(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, None, None) == 1
+    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 0, M, 0, None, None) == 2

@@ -140,3 +140,19 @@ def test_grouped_gemm_int4_matches_per_expert_matmul():
 def test_rejects_k_not_multiple_of_group():
     with pytest.raises(ValueError):
         oracle.quantize_int4_grouped(np.zeros((1, 64), np.float32))
+
+
+def test_int4_layer_equals_dense_brute_force():
+    # the routed layer on INT4 experts equals the all-experts-dense form
+    rng = np.random.default_rng(5)
+    E, k, H, I, T = 4, 2, 256, 128, 5
+    w_gu = (rng.standard_normal((E, 2 * I, H)) * 0.05).astype(np.float32)
+    w_d = (rng.standard_normal((E, H, I)) * 0.05).astype(np.float32)
+    p_gu, m_gu = oracle.quantize_int4_grouped(w_gu)
+    p_d, m_d = oracle.quantize_int4_grouped(w_d)
+    stack = oracle.Int4ExpertStack(p_gu, m_gu, p_d, m_d)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    y = oracle.moe_layer(x, lg, stack, k, True)
+    y_dense = oracle.moe_layer_dense(x, lg, stack, k, True)
+    np.testing.assert_allclose(y, y_dense, rtol=1e-9, atol=1e-12)
