@@ -23,6 +23,9 @@ Sources (web pages on the method, cited by page title and section):
   decode GEMV ("grouped-nf4-gemm & experts-4bit", third bullet; "MoE Training
   on Consumer GPUs", cerinamroth.com/ml, section "Task guides");
   ``oracle.int4`` states the format readings.
+* Per-expert LoRA adapters over the frozen 4-bit base ("4-bit
+  Mixture-of-Experts fine-tuning on small GPUs", jordananderson.work);
+  ``oracle.lora`` states the readings.
 
 Where the pages are silent the oracle takes one reading, documented at each
 function.  Every function is pinned by tests in ``tests/test_oracle_*.py``
@@ -48,6 +51,7 @@ from .int4 import (  # noqa: F401
     dequantize_int4_grouped,
     int4_scales_zeros,
 )
+from .lora import lora_delta  # noqa: F401
 from .routing import route_topk, permute_by_expert  # noqa: F401
 from .moe import (  # noqa: F401
     swiglu,
