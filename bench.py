@@ -56,6 +56,9 @@ def parse_args():
     p.add_argument("--algo", choices=["auto", "gemv", "tc"], default="auto")
     p.add_argument("--weights", choices=["nf4", "int4"], default="nf4",
                    help="expert weight format (int4: grouped GPTQ-style codes, decode GEMV)")
+    p.add_argument("--lora", type=int, default=0, metavar="RANK",
+                   help="per-expert LoRA adapters of this rank on both projections "
+                        "(0 = none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
@@ -214,11 +217,12 @@ def rank_seed(seed, rank):
 # ----------------------------------------------------------------- workload
 
 class Workload:
-    def __init__(self, shape, T, layers, seed, device="cuda", weights="nf4"):
+    def __init__(self, shape, T, layers, seed, device="cuda", weights="nf4", lora=0):
         import bit_mixture_experts_route_b200 as moe
         self.moe = moe
         self.shape, self.T, self.L = shape, T, layers
         self.int4 = weights == "int4"
+        self.lora = lora
         quantize = moe.int4_quantize if self.int4 else moe.nf4_quantize
         self.stacks = []
         for layer in range(layers):
@@ -252,6 +256,16 @@ class Workload:
         self.Y = torch.empty((T, H), dtype=torch.float32, device=dev)
         self.lws = torch.empty((max(moe.layer_workspace_size(T, E, k, H, I), 256),),
                                dtype=torch.uint8, device=dev)
+        if lora:
+            # adapted path: both GEMMs write fp32 pre-activations, the adapters
+            # add their term in place, SwiGLU runs standalone
+            self.adapters = [moe_synth.lora_adapters(shape, "gate_up", lora, seed * 1000 + layer,
+                                                     device=dev)
+                             + moe_synth.lora_adapters(shape, "down", lora, seed * 1000 + layer,
+                                                       device=dev)
+                             for layer in range(layers)]
+            self.GU = torch.empty((M, 2 * I), dtype=torch.float32, device=dev)
+            self.Yp32 = torch.empty((M, H), dtype=torch.float32, device=dev)
 
     def layer(self, layer, algo="auto", ev=None, X=None, logits=None):
         moe, sh, T = self.moe, self.shape, self.T
@@ -261,6 +275,9 @@ class Workload:
         r = moe.route_permute(logits, sh.k, sh.renormalize, workspace=self.rws, out=self.route)
         M = T * sh.k
         moe.permute_rows(X, r["sorted_rows"], sh.k, out=self.Xp)
+        if self.lora:
+            self._adapted_layer(layer, r, M, algo, ev)
+            return
         if ev is not None:
             ev[0].record()
         if self.int4:
@@ -278,6 +295,41 @@ class Workload:
             moe.nf4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
                                  out=self.Yp, algo=algo)
         moe.unpermute_combine(self.Yp, r["inv_perm"], r["topk_w"], out=self.Y)
+
+    def _gemm(self, A, packed, scales, offsets, M, out, algo):
+        if self.int4:
+            self.moe.int4_grouped_gemm(A, packed, scales, offsets, M, epilogue="none", out=out)
+        else:
+            self.moe.nf4_grouped_gemm(A, packed, scales, offsets, M, epilogue="none", out=out,
+                                      algo=algo)
+
+    def _adapted_layer(self, layer, r, M, algo, ev):
+        moe = self.moe
+        p_gu, a_gu, p_d, a_d = self.stacks[layer]
+        A_gu, B_gu, A_d, B_d = self.adapters[layer]
+        off = r["expert_offsets"]
+        scale = 32.0 / self.lora     # alpha = 32
+        if ev is not None:
+            ev[0].record()
+        self._gemm(self.Xp, p_gu, a_gu, off, M, self.GU, algo)
+        if ev is not None:
+            ev[1].record()
+            ev[2].record()
+        moe.lora_delta(self.Xp, off, A_gu, B_gu, scale, self.GU, M_total=M)
+        if ev is not None:
+            ev[3].record()
+        moe.swiglu(self.GU, out=self.Hbuf)
+        self._gemm(self.Hbuf, p_d, a_d, off, M, self.Yp32, algo)
+        moe.lora_delta(self.Hbuf, off, A_d, B_d, scale, self.Yp32, M_total=M)
+        moe.unpermute_combine(self.Yp32, r["inv_perm"], r["topk_w"], out=self.Y)
+
+    def lora_bytes(self, d):
+        """Algorithmic bytes of the gate_up adapter launch: the distinct
+        experts' A and B, the routed input rows, the fp32 pre-activation read
+        and written."""
+        sh, M = self.shape, self.T * self.shape.k
+        return (d * self.lora * (sh.H + 2 * sh.I) * 2 + M * sh.H * 2
+                + 2 * M * 2 * sh.I * 4)
 
     def step(self, algo="auto", evs=None):
         for layer in range(self.L):
@@ -298,11 +350,14 @@ class Workload:
         # per weight: 4-bit code + fp32 absmax per 64 (NF4) or fp16 scale and
         # zero in 4 bytes per 128 (INT4)
         w = d * (2 * sh.I * sh.H) * (0.53125 if self.int4 else 0.5625)
-        return w + T * sh.H * 2 + T * sh.k * sh.I * 2
+        # output: fp16 SwiGLU rows, or fp32 gate_up pre-activations when adapted
+        out = T * sh.k * 2 * sh.I * 4 if self.lora else T * sh.k * sh.I * 2
+        return w + T * sh.H * 2 + out
 
     def layer_bytes(self, d):
         sh, T = self.shape, self.T
-        return d * 3 * sh.H * sh.I * 0.5625 + T * sh.H * 2 + T * sh.E * 4 + T * sh.H * 4
+        per_w = 0.53125 if self.int4 else 0.5625
+        return d * 3 * sh.H * sh.I * per_w + T * sh.H * 2 + T * sh.E * 4 + T * sh.H * 4
 
     def gate_up_flops(self):
         sh = self.shape
@@ -442,7 +497,8 @@ def main():
     world, rank, local = dist_setup()
     import bit_mixture_experts_route_b200 as moe
     moe.load()
-    wl = Workload(shape, T, layers, rank_seed(args.seed, rank), weights=args.weights)
+    wl = Workload(shape, T, layers, rank_seed(args.seed, rank), weights=args.weights,
+                  lora=args.lora)
     if args.weights == "int4" and T * shape.k >= 36 * shape.E:
         raise SystemExit("int4 weights have the decode GEMV path only (fewer than 36 routed "
                          "rows per expert)")
@@ -454,8 +510,10 @@ def main():
         wl.step(args.algo)
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, events around every gate_up launch
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+    # ---- timed region: K steps, events around every gate_up launch (and the
+    # gate_up adapter launch when adapted)
+    n_ev = 4 if args.lora else 2
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
             for _ in range(layers)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
@@ -475,6 +533,7 @@ def main():
     value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
     gu_ms = [e[0].elapsed_time(e[1]) for st in evs for e in st]
     gu_avg_ms = sum(gu_ms) / len(gu_ms)
+    lora_ms = [e[2].elapsed_time(e[3]) for st in evs for e in st] if args.lora else []
 
     d = wl.distinct_experts()
     d_avg = sum(d) / len(d)
@@ -483,7 +542,9 @@ def main():
     # the tensor-core kernel serves the GEMMs from 36 routed rows per expert
     # on average (the AUTO dispatch rule); below that the decode GEMV does
     prefill = T * shape.k >= 36 * shape.E
-    workload_name = args.config + ("/int4" if args.weights == "int4" else "")
+    workload_name = (args.config + ("/int4" if args.weights == "int4" else "")
+                     + (f"/lora-r{args.lora}" if args.lora else ""))
+    epi_name = "(fp32 out, adapted)" if args.lora else "+ SwiGLU"
     workload_key = f"{workload_name}:T={T}"
     if prefill:
         achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
@@ -491,7 +552,7 @@ def main():
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
                 "traffic": recorded_traffic("grouped_gemm_tc.cu", workload_key),
-                "kernel": "grouped NF4 gate_up GEMM + SwiGLU",
+                "kernel": f"grouped NF4 gate_up GEMM {epi_name}",
                 "per_launch": f"{gu_flops:.4g} FLOP (2*T*k*H*2I)",
                 "peak_source": f"{peak_kind} bf16 dense"}
     else:
@@ -502,9 +563,9 @@ def main():
                 "traffic": recorded_traffic(
                     "grouped_gemm_int4.cu" if args.weights == "int4" else "grouped_gemm_decode.cu",
                     workload_key),
-                "kernel": f"grouped {args.weights.upper()} gate_up GEMV + SwiGLU",
+                "kernel": f"grouped {args.weights.upper()} gate_up GEMV {epi_name}",
                 "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*"
-                              f"{0.53125 if args.weights == 'int4' else 0.5625} + X + Hbuf)",
+                              f"{0.53125 if args.weights == 'int4' else 0.5625} + X + output)",
                 "peak_source": f"{peak_kind} HBM copy"}
 
     # ---- the same step as one CUDA graph (how a decode server replays it):
@@ -558,7 +619,7 @@ def main():
         X_d.copy_(X_h, non_blocking=True)
         L_d.copy_(L_h, non_blocking=True)
         for layer in range(layers):
-            if wl.int4:  # the five calls through the binding, on the copied inputs
+            if wl.int4 or wl.lora:  # the calls through the binding, on the copied inputs
                 wl.layer(layer, args.algo, X=X_d, logits=L_d[layer])
             else:
                 moe.layer_forward(X_d, L_d[layer], shape.k, shape.renormalize,
@@ -581,7 +642,10 @@ def main():
            "d2h_bytes_per_step": Y_h.numel() * 4}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.lora and not args.no_cpu_baseline:
+        cpu = {"skipped": "the oracle's layer has no adapters; the adapter delta's oracle "
+                          "is checked in the parity tests"}
+    elif rank == 0 and world == 1 and not args.no_cpu_baseline:
         ncpu, aff, threads = cpu_cores()
         n_tok = min(T, 64) if not prefill else 16
         n, dt = oracle_sample(shape, T, args.seed, n_tok, weights=args.weights)
@@ -600,7 +664,19 @@ def main():
         except ImportError:
             pass
 
-    launches_per_layer = 6  # route_tile, permute_scatter, permute_rows, gate_up, down, combine
+    # route_tile, permute_scatter, permute_rows, gate_up, down, combine; when
+    # adapted also two adapter launches and the standalone SwiGLU
+    launches_per_layer = 9 if args.lora else 6
+    lora = None
+    if args.lora:
+        lb = sum(wl.lora_bytes(x) for x in d) / len(d)
+        l_avg = sum(lora_ms) / len(lora_ms)
+        lach = lb / (l_avg / 1e3) / 1e9
+        lora = {"rank": args.lora, "kernel": "gate_up LoRA delta (in place on fp32)",
+                "us_per_launch": 1e3 * l_avg, "bytes_per_launch": lb,
+                "per_launch": f"distinct experts {d_avg:.1f} x r*(H+2I)*2 + X + 2 x fp32 out",
+                "achieved_GBs": lach, "frac_of_hbm": lach / hbm,
+                "flops_per_launch": 2.0 * T * shape.k * args.lora * (shape.H + 2 * shape.I)}
     eager = {"value": value, "ms_per_step": ms_per_step, "clocks": clk.summary(),
              "launch": "one host launch per kernel, CUDA events per gate_up launch"}
     clocks = clk.summary()
@@ -631,6 +707,8 @@ def main():
         "clocks": clocks,
         "gate_up_ms_avg": gu_avg_ms,
     }
+    if lora is not None:
+        line["lora"] = lora
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -20,6 +20,7 @@ from ._lib import (  # noqa: F401
     nf4_grouped_gemm,
     int4_quantize,
     int4_grouped_gemm,
+    lora_delta,
     permute_rows,
     swiglu,
     unpermute_combine,

@@ -42,6 +42,7 @@ SIGNATURES = {
                                   _I, _I, _P, _S]),
     "moe_int4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
     "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_lora_delta": (_I, [_P, _I, _P, _I, _I, _I, _I, _P, _P, ctypes.c_float, _I, _P, _P, _S]),
     "moe_permute_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _S]),
     "moe_swiglu": (_I, [_P, _I, _I, _I, _P, _I, _S]),
     "moe_unpermute_combine": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _S]),
@@ -220,6 +221,28 @@ def int4_grouped_gemm(A, packed, meta, expert_offsets, M_total, epilogue="none",
         _ptr(A), A.shape[0], _ptr(packed), _ptr(meta), _ptr(expert_offsets), E, N, K, M_total,
         EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
         "moe_int4_grouped_gemm")
+    return out
+
+
+def lora_delta(X, expert_offsets, lora_A, lora_B, scale, out, M_total=None, dev_err=None):
+    """In place: ``out[p] += scale * lora_B[e(p)] @ (lora_A[e(p)] @ X[p])`` for
+    the first ``M_total`` rows (default ``out``'s rows); ``X`` fp16 [>= M_total,
+    K], ``lora_A`` fp16 [E, r, K], ``lora_B`` fp16 [E, N, r], ``out`` fp32 [M_total, N]."""
+    _need(X, torch.float16, "X", 2)
+    _need(expert_offsets, torch.int32, "expert_offsets", 1)
+    _need(lora_A, torch.float16, "lora_A", 3)
+    _need(lora_B, torch.float16, "lora_B", 3)
+    _need(out, torch.float32, "out", 2)
+    E, r, K = lora_A.shape
+    N = lora_B.shape[1]
+    if lora_B.shape != (E, N, r) or X.shape[1] != K or out.shape[1] != N:
+        raise MoEError("lora_A [E, r, K], lora_B [E, N, r], X [*, K] and out [*, N] disagree")
+    M = out.shape[0] if M_total is None else M_total
+    if out.shape[0] < M:
+        raise MoEError("out has fewer than M_total rows")
+    _check(load().moe_lora_delta(_ptr(X), X.shape[0], _ptr(expert_offsets), E, N, K, r,
+                                 _ptr(lora_A), _ptr(lora_B), float(scale), M, _ptr(out),
+                                 _ptr(dev_err), _stream(X.device)), "moe_lora_delta")
     return out
 
 

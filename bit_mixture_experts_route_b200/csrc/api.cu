@@ -99,6 +99,24 @@ moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* pac
                                                  (cudaStream_t)stream));
 }
 
+moe_status_t moe_lora_delta(const void* X, int A_rows, const int32_t* expert_offsets, int E,
+                            int N, int K, int r, const void* lora_A, const void* lora_B,
+                            float scale, int M_total, float* out, int32_t* dev_err,
+                            void* stream) {
+  if (E < 1 || N < 1 || K < 1 || r < 1 || M_total < 0 || A_rows < M_total)
+    return MOE_ERR_INVALID_ARG;
+  if (!moe_launch::lora_delta_supported(E, K, r)) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offsets || !lora_A || !lora_B) return MOE_ERR_INVALID_ARG;
+  if (M_total > 0 && (!X || !out)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, expert_offsets, lora_A, lora_B, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  if (M_total == 0) return MOE_OK;
+  return from_cuda(moe_launch::lora_delta(X, expert_offsets, E, N, K, r, lora_A, lora_B, scale,
+                                          M_total, out, dev_err, (cudaStream_t)stream));
+}
+
 moe_status_t moe_nf4_dequantize(const uint8_t* packed, const float* absmax, int E, int N, int K,
                                 void* out, moe_dtype_t out_dtype, void* stream) {
   if (E < 1 || N < 1 || K < 1 || K % moe::kBlock || !valid_dtype(out_dtype))

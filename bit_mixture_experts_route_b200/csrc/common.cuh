@@ -257,6 +257,10 @@ cudaError_t grouped_gemm_int4(const void* A, int A_rows, const uint8_t* packed,
                               const uint32_t* meta, const int32_t* offsets, int E, int N, int K,
                               int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
                               int32_t* dev_err, cudaStream_t s);
+bool lora_delta_supported(int E, int K, int r);
+cudaError_t lora_delta(const void* X, const int32_t* offsets, int E, int N, int K, int r,
+                       const void* lora_A, const void* lora_B, float scale, int M_total,
+                       float* out, int32_t* dev_err, cudaStream_t s);
 cudaError_t permute_rows(const void* X, moe_dtype_t x_dt, int T, int K, const int32_t* rows,
                          int k, int M_total, void* Xp, int32_t* dev_err, cudaStream_t s);
 cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h,

@@ -1,0 +1,206 @@
+// Per-expert LoRA delta over the routed rows (fp16 adapters, fp32 sums).
+//
+// The pages fine-tune the 4-bit mixture with a LoRA adapter per expert over
+// the frozen base weights ("Jordan Anderson", jordananderson.work, section
+// "4-bit Mixture-of-Experts fine-tuning on small GPUs"; "MoE Training on
+// Consumer GPUs", cerinamroth.com/ml).  In LoRA's form the adapted projection
+// of routed row p of expert e is W_e x_p + scale * B_e (A_e x_p).  The grouped
+// GEMM writes the first term (fp32, no epilogue); this kernel adds the second
+// to it in place, before SiLU(gate) * up.
+//
+// One CTA per (tile of up to R rows of one expert's segment, column split).
+//   Phase 1: u[i][j] = A_e[j] . x_{p0+i} for the tile's rows, fp32.  Each warp
+//     takes a 4-row x 4-rank block at a time; lanes split K in 8-element
+//     (16-byte) vectors and a warp reduction writes the block to shared memory.
+//   Phase 2: each thread owns output columns n of the CTA's split and adds
+//     scale * sum_j B_e[n][j] u[i][j] to out[p0+i][n].
+// The adapters are tiny next to the 4-bit base (r (N + K) fp16 values per
+// expert against N K / 2 bytes); decode is bound by reading them and the fp32
+// pre-activation, prefill by the r (N + K) multiply-adds per row.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kLoraThreads = 256;
+constexpr int kLoraWarps = kLoraThreads / 32;
+constexpr int kLoraMaxRank = 64;
+constexpr int kLoraMaxE = 1024;
+
+__device__ __forceinline__ void h8_to_f32(const uint4& v, float (&f)[8]) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 t = __half22float2(h[q]);
+    f[2 * q] = t.x;
+    f[2 * q + 1] = t.y;
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(kLoraThreads) lora_delta_kernel(
+    const __half* __restrict__ X, const int32_t* __restrict__ offsets, int E, int N, int K, int r,
+    const __half* __restrict__ lA, const __half* __restrict__ lB, float scale, int M_total,
+    int nsplit, float* __restrict__ out, int32_t* dev_err) {
+  __shared__ int tile_prefix[kLoraMaxE + 1];
+  __shared__ int s_total;
+  __shared__ __align__(16) float u[R][kLoraMaxRank];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // tile_prefix[e] = sum over e' < e of ceil(count_e' / R); any offsets that
+  // are not monotone from 0 to M_total void the launch (no output written).
+  if (warp == 0) {
+    bool bad = offsets[0] != 0 || offsets[E] != M_total;
+    int run = 0;
+    for (int b0 = 0; b0 < E; b0 += 32) {
+      const int e = b0 + lane;
+      int c = 0;
+      if (e < E) {
+        c = offsets[e + 1] - offsets[e];
+        if (c < 0) { bad = true; c = 0; }
+      }
+      const int tiles = (c + R - 1) / R;
+      int incl = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (e < E) tile_prefix[e] = run + incl - tiles;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      tile_prefix[E] = run;
+      s_total = bad ? 0 : run;
+      if (bad && blockIdx.x == 0) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  const int tile = blockIdx.x / nsplit, split = blockIdx.x % nsplit;
+  if (tile >= s_total) return;
+
+  // the expert whose tiles hold `tile`: the last e with tile_prefix[e] <= tile
+  int lo = 0, hi = E;  // invariant: tile_prefix[lo] <= tile < tile_prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_prefix[mid] <= tile) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  const int row0 = offsets[e] + (tile - tile_prefix[e]) * R;
+  const int nrows = min(R, offsets[e + 1] - row0);
+
+  // ---- phase 1: u = A_e x for the tile's rows
+  const __half* Ae = lA + (int64_t)e * r * K;
+  const int pblocks = (nrows + 3) >> 2, jblocks = r >> 2;
+  for (int item = warp; item < pblocks * jblocks; item += kLoraWarps) {
+    const int pb = item / jblocks, jb = item - pb * jblocks;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][q] = 0.0f;
+    for (int k = lane * 8; k < K; k += 256) {
+      float xa[4][8], av[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ri = pb * 4 + i;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ri < nrows) v = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(row0 + ri) * K + k));
+        h8_to_f32(v, xa[i]);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(Ae + (int64_t)(jb * 4 + q) * K + k));
+        h8_to_f32(v, av[q]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) acc[i][q] = fmaf(xa[i][t], av[q][t], acc[i][q]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float s = warp_sum(acc[i][q]);
+        if (lane == 0 && pb * 4 + i < R) u[pb * 4 + i][jb * 4 + q] = s;
+      }
+  }
+  __syncthreads();
+
+  // ---- phase 2: out[p0 + i][n] += scale * B_e[n] . u[i] over this split's columns
+  const int cols = (N + nsplit - 1) / nsplit;
+  const int n_begin = split * cols, n_end = min(N, n_begin + cols);
+  const __half* Be = lB + (int64_t)e * N * r;
+  for (int n = n_begin + (int)threadIdx.x; n < n_end; n += kLoraThreads) {
+    float acc[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) acc[i] = 0.0f;
+    const __half* brow = Be + (int64_t)n * r;
+    for (int c = 0; c < r; c += 8) {
+      float b[8];
+      h8_to_f32(__ldg(reinterpret_cast<const uint4*>(brow + c)), b);
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const float4 u0 = *reinterpret_cast<const float4*>(&u[i][c]);
+        const float4 u1 = *reinterpret_cast<const float4*>(&u[i][c + 4]);
+        acc[i] = fmaf(b[0], u0.x, acc[i]);
+        acc[i] = fmaf(b[1], u0.y, acc[i]);
+        acc[i] = fmaf(b[2], u0.z, acc[i]);
+        acc[i] = fmaf(b[3], u0.w, acc[i]);
+        acc[i] = fmaf(b[4], u1.x, acc[i]);
+        acc[i] = fmaf(b[5], u1.y, acc[i]);
+        acc[i] = fmaf(b[6], u1.z, acc[i]);
+        acc[i] = fmaf(b[7], u1.w, acc[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      if (i < nrows) {
+        float* o = out + (int64_t)(row0 + i) * N + n;
+        *o = fmaf(scale, acc[i], *o);
+      }
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+namespace moe_launch {
+
+bool lora_delta_supported(int E, int K, int r) {
+  return E <= moe::kLoraMaxE && K % 8 == 0 && r >= 8 && r <= moe::kLoraMaxRank && r % 8 == 0;
+}
+
+cudaError_t lora_delta(const void* X, const int32_t* offsets, int E, int N, int K, int r,
+                       const void* lora_A, const void* lora_B, float scale, int M_total,
+                       float* out, int32_t* dev_err, cudaStream_t s) {
+  if (M_total == 0) return cudaSuccess;
+  // average rows per expert decides the tile height: 16 once the segments
+  // are long enough to fill it, else 8
+  const bool tall = (int64_t)M_total >= 16LL * E;
+  const int R = tall ? 16 : 8;
+  // every tile holds >= 1 row, and sum ceil(c / R) <= (M_total + E (R - 1)) / R
+  const int64_t tiles = std::min<int64_t>(M_total, ((int64_t)M_total + (int64_t)E * (R - 1)) / R);
+  // split the columns so that short launches still cover the SMs twice over,
+  // never below 256 columns a split
+  const int64_t want = (2LL * moe::device_sm_count() + tiles - 1) / tiles;
+  const int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, N / 256)));
+  const int64_t grid = tiles * nsplit;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const __half* Xh = reinterpret_cast<const __half*>(X);
+  const __half* Ah = reinterpret_cast<const __half*>(lora_A);
+  const __half* Bh = reinterpret_cast<const __half*>(lora_B);
+  if (tall)
+    moe::lora_delta_kernel<16><<<(unsigned)grid, moe::kLoraThreads, 0, s>>>(
+        Xh, offsets, E, N, K, r, Ah, Bh, scale, M_total, nsplit, out, dev_err);
+  else
+    moe::lora_delta_kernel<8><<<(unsigned)grid, moe::kLoraThreads, 0, s>>>(
+        Xh, offsets, E, N, K, r, Ah, Bh, scale, M_total, nsplit, out, dev_err);
+  return cudaGetLastError();
+}
+
+}  // namespace moe_launch

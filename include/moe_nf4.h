@@ -174,6 +174,34 @@ moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* pac
                                    moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
 
 /*
+ * moe_lora_delta -- adds each routed row's per-expert LoRA term to an fp32
+ * pre-activation in place: out[p] += scale * B[e(p)] @ (A[e(p)] @ X[p]) for
+ * every row p in expert e's segment [expert_offsets[e], expert_offsets[e+1]).
+ * ("Jordan Anderson", jordananderson.work, section "4-bit Mixture-of-Experts
+ * fine-tuning on small GPUs": LoRA adapters per expert over the frozen 4-bit
+ * base; the form W x + scale * B (A x), scale = alpha / r, is LoRA's.)  Run
+ * it after moe_nf4_grouped_gemm / moe_int4_grouped_gemm with MOE_EPI_NONE and
+ * F32 output, then moe_swiglu for gate_up.
+ *
+ *   X        fp16 [A_rows >= M_total, K]  the projection's input rows in
+ *            permuted order (the GEMM's A)
+ *   expert_offsets int32 [E+1] (device), monotone, offsets[0] == 0,
+ *            offsets[E] == M_total, else MOE_DEVERR_BAD_OFFSETS is set and
+ *            out is left unchanged
+ *   E <= 1024, N >= 1, K % 8 == 0, r % 8 == 0, 8 <= r <= 64
+ *   lora_A   fp16 [E, r, K]   (device, read only)
+ *   lora_B   fp16 [E, N, r]   (device, read only)
+ *   scale    the adapter's scale (alpha / r)
+ *   out      fp32 [M_total, N] (device), read and written
+ * Sums are fp32 (A X kept in fp32, not rounded to fp16).  All pointers
+ * 16-byte aligned.  Shapes outside the limits return MOE_ERR_UNSUPPORTED.
+ */
+moe_status_t moe_lora_delta(const void* X, int A_rows, const int32_t* expert_offsets, int E,
+                            int N, int K, int r, const void* lora_A, const void* lora_B,
+                            float scale, int M_total, float* out, int32_t* dev_err,
+                            void* stream);
+
+/*
  * Workspace bytes moe_route_permute needs for (T, E, k).  `bytes` is a HOST
  * pointer.  Host-only, no CUDA call.
  */

@@ -27,7 +27,7 @@ import math
 import torch
 
 # Seed offsets so every tensor of a layer has its own stream.
-_X, _LOGITS, _WGU, _WD, _OUTLIER = 1, 2, 3, 4, 5
+_X, _LOGITS, _WGU, _WD, _OUTLIER, _LORA = 1, 2, 3, 4, 5, 6
 
 
 @dataclasses.dataclass(frozen=True)
@@ -128,6 +128,19 @@ def logits(shape: MoEShape, T: int, seed: int, device="cpu") -> torch.Tensor:
     if shape.zipf_empty:
         out[:, ranks > E - shape.zipf_empty] = -1e4
     return out.to(device)
+
+
+def lora_adapters(shape: MoEShape, which: str, rank: int, seed: int,
+                  device="cpu"):
+    """fp16 per-expert LoRA adapters for ``which`` in {"gate_up", "down"}:
+    ``A [E, r, K] ~ N(0, 1/K)`` and ``B [E, N, r] ~ N(0, 0.02^2)`` (a trained
+    B is small; LoRA starts it at zero)."""
+    N, K = (2 * shape.I, shape.H) if which == "gate_up" else (shape.H, shape.I)
+    off = _WGU if which == "gate_up" else _WD
+    g = _gen(seed * 1_000_003 + _LORA * 10_007 + off, device)
+    A = torch.randn((shape.E, rank, K), generator=g, device=device) / math.sqrt(K)
+    B = torch.randn((shape.E, N, rank), generator=g, device=device) * 0.02
+    return A.to(torch.float16), B.to(torch.float16)
 
 
 def expected_distinct_experts(E: int, k: int, T: int) -> float:

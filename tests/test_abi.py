@@ -135,3 +135,18 @@ def test_int4_calls_reject_bad_arguments(lib):
     assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 9, None, None) == 1
     assert lib.moe_int4_grouped_gemm(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, None, None) == 1
     assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 0, M, 0, None, None) == 2
+
+
+def test_lora_delta_rejects_bad_arguments(lib):
+    A, M = ALIGNED, MISALIGNED
+    # (X, A_rows, offsets, E, N, K, r, lora_A, lora_B, scale, M_total, out, dev_err, stream)
+    # rank outside 8..64 or not a multiple of 8, K % 8, E > 1024 -> unsupported
+    assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 4, A, A, 1.0, 8, A, None, None) == 3
+    assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 12, A, A, 1.0, 8, A, None, None) == 3
+    assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 72, A, A, 1.0, 8, A, None, None) == 3
+    assert lib.moe_lora_delta(A, 8, A, 2, 64, 260, 16, A, A, 1.0, 8, A, None, None) == 3
+    assert lib.moe_lora_delta(A, 8, A, 1025, 64, 256, 16, A, A, 1.0, 8, A, None, None) == 3
+    # A_rows < M_total, null adapters, misaligned output
+    assert lib.moe_lora_delta(A, 4, A, 2, 64, 256, 16, A, A, 1.0, 8, A, None, None) == 1
+    assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 16, None, A, 1.0, 8, A, None, None) == 1
+    assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 16, A, A, 1.0, 8, M, None, None) == 2
