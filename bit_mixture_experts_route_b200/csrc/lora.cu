@@ -9,11 +9,11 @@
 // to it in place, before SiLU(gate) * up.
 //
 // One CTA per (tile of up to R rows of one expert's segment, column split).
-//   Phase 1: u[i][j] = A_e[j] . x_{p0+i} for the tile's rows, fp32.  Each warp
+//   Phase 1: u[i][j] = scale * (A_e[j] . x_{p0+i}) for the tile's rows, fp32.  Each warp
 //     takes a 4-row x 4-rank block at a time; lanes split K in 8-element
 //     (16-byte) vectors and a warp reduction writes the block to shared memory.
 //   Phase 2: each thread owns output columns n of the CTA's split and adds
-//     scale * sum_j B_e[n][j] u[i][j] to out[p0+i][n].
+//     sum_j B_e[n][j] u[i][j] to out[p0+i][n], accumulating onto the loaded value.
 // The adapters are tiny next to the 4-bit base (r (N + K) fp16 values per
 // expert against N K / 2 bytes); decode is bound by reading them and the fp32
 // pre-activation, prefill by the r (N + K) multiply-adds per row.
@@ -37,26 +37,47 @@ __device__ __forceinline__ void h8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
+// fp32 FMA of four 8-element x vectors against four 8-element a vectors
+__device__ __forceinline__ void dot4x4(const uint4 (&xr)[4], const uint4 (&ar)[4],
+                                       float (&acc)[4][4]) {
+  float a[4][8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) h8_to_f32(ar[q], a[q]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float x[8];
+    h8_to_f32(xr[i], x);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc[i][q] = fmaf(x[t], a[q][t], acc[i][q]);
+  }
+}
+
 template <int R>
-__global__ void __launch_bounds__(kLoraThreads) lora_delta_kernel(
+__global__ void __launch_bounds__(kLoraThreads, 2) lora_delta_kernel(
     const __half* __restrict__ X, const int32_t* __restrict__ offsets, int E, int N, int K, int r,
     const __half* __restrict__ lA, const __half* __restrict__ lB, float scale, int M_total,
     int nsplit, float* __restrict__ out, int32_t* dev_err) {
+  __shared__ int s_off[kLoraMaxE + 1];
   __shared__ int tile_prefix[kLoraMaxE + 1];
   __shared__ int s_total;
   __shared__ __align__(16) float u[R][kLoraMaxRank];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  // tile_prefix[e] = sum over e' < e of ceil(count_e' / R); any offsets that
-  // are not monotone from 0 to M_total void the launch (no output written).
+  // offsets into shared memory in one pass, then tile_prefix[e] = sum over
+  // e' < e of ceil(count_e' / R); offsets that are not monotone from 0 to
+  // M_total void the launch (no output written)
+  for (int i = threadIdx.x; i <= E; i += kLoraThreads) s_off[i] = offsets[i];
+  __syncthreads();
   if (warp == 0) {
-    bool bad = offsets[0] != 0 || offsets[E] != M_total;
+    bool bad = s_off[0] != 0 || s_off[E] != M_total;
     int run = 0;
     for (int b0 = 0; b0 < E; b0 += 32) {
       const int e = b0 + lane;
       int c = 0;
       if (e < E) {
-        c = offsets[e + 1] - offsets[e];
+        c = s_off[e + 1] - s_off[e];
         if (c < 0) { bad = true; c = 0; }
       }
       const int tiles = (c + R - 1) / R;
@@ -87,82 +108,102 @@ __global__ void __launch_bounds__(kLoraThreads) lora_delta_kernel(
     if (tile_prefix[mid] <= tile) lo = mid; else hi = mid;
   }
   const int e = lo;
-  const int row0 = offsets[e] + (tile - tile_prefix[e]) * R;
-  const int nrows = min(R, offsets[e + 1] - row0);
+  const int row0 = s_off[e] + (tile - tile_prefix[e]) * R;
+  const int nrows = min(R, s_off[e + 1] - row0);
 
-  // ---- phase 1: u = A_e x for the tile's rows
+  // ---- phase 1: u = A_e x for the tile's rows; the loads of the next
+  // 256-wide k step are in flight while the current one is multiplied
   const __half* Ae = lA + (int64_t)e * r * K;
   const int pblocks = (nrows + 3) >> 2, jblocks = r >> 2;
   for (int item = warp; item < pblocks * jblocks; item += kLoraWarps) {
     const int pb = item / jblocks, jb = item - pb * jblocks;
+    const __half* xrow[4];
+    const __half* arow[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // rows past the tile read row 0 of the tile (in range) and are dropped
+      const int ri = pb * 4 + i < nrows ? pb * 4 + i : 0;
+      xrow[i] = X + (int64_t)(row0 + ri) * K;
+      arow[i] = Ae + (int64_t)(jb * 4 + i) * K;
+    }
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[i][q] = 0.0f;
-    for (int k = lane * 8; k < K; k += 256) {
-      float xa[4][8], av[4][8];
+    int k = lane * 8;
+    uint4 xr[4], ar[4];
+    if (k < K) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int ri = pb * 4 + i;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (ri < nrows) v = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(row0 + ri) * K + k));
-        h8_to_f32(v, xa[i]);
+        xr[i] = __ldg(reinterpret_cast<const uint4*>(xrow[i] + k));
+        ar[i] = __ldg(reinterpret_cast<const uint4*>(arow[i] + k));
       }
+    }
+    for (; k < K; k += 256) {
+      uint4 xn[4], an[4];
+      const bool more = k + 256 < K;
+      if (more) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(Ae + (int64_t)(jb * 4 + q) * K + k));
-        h8_to_f32(v, av[q]);
+        for (int i = 0; i < 4; ++i) {
+          xn[i] = __ldg(reinterpret_cast<const uint4*>(xrow[i] + k + 256));
+          an[i] = __ldg(reinterpret_cast<const uint4*>(arow[i] + k + 256));
+        }
       }
+      dot4x4(xr, ar, acc);
+      if (more) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int t = 0; t < 8; ++t) acc[i][q] = fmaf(xa[i][t], av[q][t], acc[i][q]);
+        for (int i = 0; i < 4; ++i) {
+          xr[i] = xn[i];
+          ar[i] = an[i];
+        }
+      }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float s = warp_sum(acc[i][q]);
-        if (lane == 0 && pb * 4 + i < R) u[pb * 4 + i][jb * 4 + q] = s;
+        if (lane == 0) u[pb * 4 + i][jb * 4 + q] = scale * s;
       }
   }
   __syncthreads();
 
-  // ---- phase 2: out[p0 + i][n] += scale * B_e[n] . u[i] over this split's columns
+  // ---- phase 2: out[p0 + i][n] += B_e[n] . u[i] (u holds scale * A_e x) over this split's
+  // columns.  Every load of a column (its R outputs, its B_e row) comes
+  // before the first store, so the loads overlap in one round trip.
   const int cols = (N + nsplit - 1) / nsplit;
   const int n_begin = split * cols, n_end = min(N, n_begin + cols);
   const __half* Be = lB + (int64_t)e * N * r;
+  float* orow = out + (int64_t)row0 * N;
   for (int n = n_begin + (int)threadIdx.x; n < n_end; n += kLoraThreads) {
-    float acc[R];
-#pragma unroll
-    for (int i = 0; i < R; ++i) acc[i] = 0.0f;
     const __half* brow = Be + (int64_t)n * r;
-    for (int c = 0; c < r; c += 8) {
-      float b[8];
-      h8_to_f32(__ldg(reinterpret_cast<const uint4*>(brow + c)), b);
+    float o[R];
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const float4 u0 = *reinterpret_cast<const float4*>(&u[i][c]);
-        const float4 u1 = *reinterpret_cast<const float4*>(&u[i][c + 4]);
-        acc[i] = fmaf(b[0], u0.x, acc[i]);
-        acc[i] = fmaf(b[1], u0.y, acc[i]);
-        acc[i] = fmaf(b[2], u0.z, acc[i]);
-        acc[i] = fmaf(b[3], u0.w, acc[i]);
-        acc[i] = fmaf(b[4], u1.x, acc[i]);
-        acc[i] = fmaf(b[5], u1.y, acc[i]);
-        acc[i] = fmaf(b[6], u1.z, acc[i]);
-        acc[i] = fmaf(b[7], u1.w, acc[i]);
+    for (int i = 0; i < R; ++i) o[i] = i < nrows ? orow[(int64_t)i * N + n] : 0.0f;
+#pragma unroll
+    for (int c = 0; c < kLoraMaxRank / 8; ++c) {
+      if (c * 8 < r) {
+        float b[8];
+        h8_to_f32(__ldg(reinterpret_cast<const uint4*>(brow + c * 8)), b);
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+          const float4 u0 = *reinterpret_cast<const float4*>(&u[i][c * 8]);
+          const float4 u1 = *reinterpret_cast<const float4*>(&u[i][c * 8 + 4]);
+          o[i] = fmaf(b[0], u0.x, o[i]);
+          o[i] = fmaf(b[1], u0.y, o[i]);
+          o[i] = fmaf(b[2], u0.z, o[i]);
+          o[i] = fmaf(b[3], u0.w, o[i]);
+          o[i] = fmaf(b[4], u1.x, o[i]);
+          o[i] = fmaf(b[5], u1.y, o[i]);
+          o[i] = fmaf(b[6], u1.z, o[i]);
+          o[i] = fmaf(b[7], u1.w, o[i]);
+        }
       }
     }
 #pragma unroll
     for (int i = 0; i < R; ++i)
-      if (i < nrows) {
-        float* o = out + (int64_t)(row0 + i) * N + n;
-        *o = fmaf(scale, acc[i], *o);
-      }
+      if (i < nrows) orow[(int64_t)i * N + n] = o[i];
   }
 }
 
