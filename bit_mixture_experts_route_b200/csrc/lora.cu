@@ -54,6 +54,14 @@ __device__ __forceinline__ void dot4x4(const uint4 (&xr)[4], const uint4 (&ar)[4
   }
 }
 
+// L2 prefetch of [p, p + bytes), one request per 128-byte line, spread over
+// the CTA's threads; every address lies inside the range.
+__device__ __forceinline__ void prefetch_l2(const void* p, int64_t bytes) {
+  const char* c = static_cast<const char*>(p);
+  for (int64_t off = (int64_t)threadIdx.x * 128; off < bytes; off += (int64_t)kLoraThreads * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(c + off));
+}
+
 template <int R>
 __global__ void __launch_bounds__(kLoraThreads, 2) lora_delta_kernel(
     const __half* __restrict__ X, const int32_t* __restrict__ offsets, int E, int N, int K, int r,
@@ -111,9 +119,24 @@ __global__ void __launch_bounds__(kLoraThreads, 2) lora_delta_kernel(
   const int row0 = s_off[e] + (tile - tile_prefix[e]) * R;
   const int nrows = min(R, s_off[e + 1] - row0);
 
+  // Ask L2 for everything this CTA reads (the tile's input rows, A_e, its
+  // columns of B_e and of the output rows) before the first demand load, so
+  // that the dependent loads below meet L2 rather than HBM.
+  const int cols = (N + nsplit - 1) / nsplit;
+  const int n_begin = split * cols, n_end = min(N, n_begin + cols);
+  const __half* Ae = lA + (int64_t)e * r * K;
+  const __half* Be = lB + (int64_t)e * N * r;
+  float* orow = out + (int64_t)row0 * N;
+  prefetch_l2(X + (int64_t)row0 * K, (int64_t)nrows * K * 2);
+  prefetch_l2(Ae, (int64_t)r * K * 2);
+  if (n_begin < n_end) {
+    prefetch_l2(Be + (int64_t)n_begin * r, (int64_t)(n_end - n_begin) * r * 2);
+    for (int i = 0; i < nrows; ++i)
+      prefetch_l2(orow + (int64_t)i * N + n_begin, (int64_t)(n_end - n_begin) * 4);
+  }
+
   // ---- phase 1: u = A_e x for the tile's rows; the loads of the next
   // 256-wide k step are in flight while the current one is multiplied
-  const __half* Ae = lA + (int64_t)e * r * K;
   const int pblocks = (nrows + 3) >> 2, jblocks = r >> 2;
   for (int item = warp; item < pblocks * jblocks; item += kLoraWarps) {
     const int pb = item / jblocks, jb = item - pb * jblocks;
@@ -172,10 +195,6 @@ __global__ void __launch_bounds__(kLoraThreads, 2) lora_delta_kernel(
   // ---- phase 2: out[p0 + i][n] += B_e[n] . u[i] (u holds scale * A_e x) over this split's
   // columns.  Every load of a column (its R outputs, its B_e row) comes
   // before the first store, so the loads overlap in one round trip.
-  const int cols = (N + nsplit - 1) / nsplit;
-  const int n_begin = split * cols, n_end = min(N, n_begin + cols);
-  const __half* Be = lB + (int64_t)e * N * r;
-  float* orow = out + (int64_t)row0 * N;
   for (int n = n_begin + (int)threadIdx.x; n < n_end; n += kLoraThreads) {
     const __half* brow = Be + (int64_t)n * r;
     float o[R];
