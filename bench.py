@@ -673,6 +673,8 @@ def main():
         l_avg = sum(lora_ms) / len(lora_ms)
         lach = lb / (l_avg / 1e3) / 1e9
         lora = {"rank": args.lora, "kernel": "gate_up LoRA delta (in place on fp32)",
+                "timing": "CUDA events around each eager launch; at decode sizes the window "
+                          "can include the wait for the host to submit the launch",
                 "us_per_launch": 1e3 * l_avg, "bytes_per_launch": lb,
                 "per_launch": f"distinct experts {d_avg:.1f} x r*(H+2I)*2 + X + 2 x fp32 out",
                 "achieved_GBs": lach, "frac_of_hbm": lach / hbm,
