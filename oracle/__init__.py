@@ -26,6 +26,9 @@ Sources (web pages on the method, cited by page title and section):
 * Per-expert LoRA adapters over the frozen 4-bit base ("4-bit
   Mixture-of-Experts fine-tuning on small GPUs", jordananderson.work);
   ``oracle.lora`` states the readings.
+* The layer's backward with the 4-bit experts frozen ("grouped-nf4-gemm &
+  experts-4bit", jordananderson-pages.pages.dev, fourth bullet);
+  ``oracle.backward`` states the readings.
 
 Where the pages are silent the oracle takes one reading, documented at each
 function.  Every function is pinned by tests in ``tests/test_oracle_*.py``
@@ -52,6 +55,15 @@ from .int4 import (  # noqa: F401
     int4_scales_zeros,
 )
 from .lora import lora_delta  # noqa: F401
+from .backward import (  # noqa: F401
+    grouped_gemm_t,
+    swiglu_backward,
+    combine_backward,
+    route_backward,
+    moe_layer_backward,
+    moe_layer_backward_permuted,
+    lora_backward,
+)
 from .routing import route_topk, permute_by_expert  # noqa: F401
 from .moe import (  # noqa: F401
     swiglu,
