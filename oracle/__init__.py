@@ -26,6 +26,9 @@ Sources (web pages on the method, cited by page title and section):
 * Per-expert LoRA adapters over the frozen 4-bit base ("4-bit
   Mixture-of-Experts fine-tuning on small GPUs", jordananderson.work);
   ``oracle.lora`` states the readings.
+* MXFP4 experts, e2m1 codes with an e8m0 scale per 32 ("grouped-nf4-gemm &
+  experts-4bit", third bullet; "MoE Training on Consumer GPUs", "Task
+  guides"); ``oracle.mxfp4`` states the readings.
 * The layer's backward with the 4-bit experts frozen ("grouped-nf4-gemm &
   experts-4bit", jordananderson-pages.pages.dev, fourth bullet);
   ``oracle.backward`` states the readings.
@@ -54,6 +57,12 @@ from .int4 import (  # noqa: F401
     dequantize_int4_grouped,
     int4_scales_zeros,
 )
+from .mxfp4 import (  # noqa: F401
+    BLOCK as MXFP4_BLOCK,
+    e2m1_values,
+    quantize_mxfp4,
+    dequantize_mxfp4,
+)
 from .lora import lora_delta  # noqa: F401
 from .backward import (  # noqa: F401
     grouped_gemm_t,
@@ -69,10 +78,12 @@ from .moe import (  # noqa: F401
     swiglu,
     grouped_gemm,
     grouped_gemm_int4,
+    grouped_gemm_mxfp4,
     unpermute_combine,
     moe_layer,
     moe_layer_dense,
     moe_layer_permuted,
     ExpertStack,
     Int4ExpertStack,
+    Mxfp4ExpertStack,
 )

@@ -25,6 +25,7 @@ from __future__ import annotations
 import numpy as np
 
 from .int4 import dequantize_int4_grouped
+from .mxfp4 import dequantize_mxfp4
 from .nf4 import dequantize_blockwise
 from .routing import route_topk, permute_by_expert
 
@@ -91,6 +92,34 @@ class Int4ExpertStack:
         return self._d[e]
 
 
+class Mxfp4ExpertStack:
+    """MXFP4 gate_up and down stacks of one layer (``oracle.mxfp4``),
+    dequantized lazily per expert; same interface as ``ExpertStack``.
+
+    ``packed_gu uint8[E, 2I, H/2]``, ``scales_gu uint8[E, 2I, H/32]``,
+    ``packed_d uint8[E, H, I/2]``, ``scales_d uint8[E, H, I/32]``.
+    """
+
+    def __init__(self, packed_gu, scales_gu, packed_d, scales_d):
+        self.packed_gu, self.scales_gu = np.asarray(packed_gu, np.uint8), np.asarray(scales_gu)
+        self.packed_d, self.scales_d = np.asarray(packed_d, np.uint8), np.asarray(scales_d)
+        self.E, two_i, half_h = self.packed_gu.shape
+        self.I = two_i // 2
+        self.H = half_h * 2
+        assert self.packed_d.shape == (self.E, self.H, self.I // 2)
+        self._gu, self._d = {}, {}
+
+    def gate_up(self, e: int) -> np.ndarray:
+        if e not in self._gu:
+            self._gu[e] = dequantize_mxfp4(self.packed_gu[e], self.scales_gu[e])
+        return self._gu[e]
+
+    def down(self, e: int) -> np.ndarray:
+        if e not in self._d:
+            self._d[e] = dequantize_mxfp4(self.packed_d[e], self.scales_d[e])
+        return self._d[e]
+
+
 def _silu(g: np.ndarray) -> np.ndarray:
     return g / (1.0 + np.exp(-g))
 
@@ -144,6 +173,16 @@ def grouped_gemm_int4(A: np.ndarray, packed: np.ndarray, meta: np.ndarray,
     ``packed uint8[E, N, K/2]``, ``meta uint32[E, N, K/128]``."""
     E, N, half_k = packed.shape
     return _grouped(A, lambda e: dequantize_int4_grouped(packed[e], meta[e]), N, expert_offsets,
+                    gather, k, rows)
+
+
+def grouped_gemm_mxfp4(A: np.ndarray, packed: np.ndarray, scales: np.ndarray,
+                       expert_offsets: np.ndarray, gather=None, k: int = 1,
+                       rows=None) -> np.ndarray:
+    """The same grouped GEMM on MXFP4 weights (``oracle.mxfp4``):
+    ``packed uint8[E, N, K/2]``, ``scales uint8[E, N, K/32]``."""
+    E, N, half_k = packed.shape
+    return _grouped(A, lambda e: dequantize_mxfp4(packed[e], scales[e]), N, expert_offsets,
                     gather, k, rows)
 
 
