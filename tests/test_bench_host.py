@@ -1,0 +1,103 @@
+"""Host-side logic of bench.py, on CPU: the recorded-traffic lookup, the clock
+sampler's summary, and the reference arm (the oracle) on the tiny workload."""
+
+import json
+import os
+import shutil
+import types
+
+import pytest
+
+import bench
+
+
+def test_recorded_traffic_only_for_the_recorded_source(tmp_path, monkeypatch):
+    got = bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=64")
+    assert got is not None and got > 1e8
+    assert bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=7") is None
+    assert bench.recorded_traffic("no_such_kernel.cu", "olmoe-decode:T=64") is None
+    # a changed kernel source (different sha256) has no recorded traffic
+    root = tmp_path
+    (root / "profiles").mkdir()
+    (root / "bit_mixture_experts_route_b200" / "csrc").mkdir(parents=True)
+    shutil.copy(os.path.join(bench.ROOT, "profiles", "kernel_traffic.txt"), root / "profiles")
+    src = os.path.join(bench.ROOT, "bit_mixture_experts_route_b200", "csrc",
+                       "grouped_gemm_decode.cu")
+    dst = root / "bit_mixture_experts_route_b200" / "csrc" / "grouped_gemm_decode.cu"
+    dst.write_bytes(open(src, "rb").read() + b"\n// edited\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=64") is None
+
+
+def _line(ts, sm, reasons=("Not Active",) * 4):
+    return ", ".join([ts, "0", str(sm), "1965", "900.0", "0x0", *reasons])
+
+
+def test_clock_summary_keeps_the_timed_region_and_reports_reasons():
+    c = bench.ClockSampler(0)
+    t0 = c._stamp("2026/12/02 10:00:01.000")
+    c.t0, c.t1 = t0, t0 + 1.0
+    c.lines = [
+        _line("2026/12/02 10:00:00.500", 600),                        # before: dropped
+        _line("2026/12/02 10:00:01.100", 1965),
+        _line("2026/12/02 10:00:01.500", 1950,
+              ("Not Active", "Not Active", "Not Active", "Active")),  # power cap
+        _line("2026/12/02 10:00:01.900", 1965),
+        _line("2026/12/02 10:00:03.000", 300,
+              ("Active", "Not Active", "Not Active", "Not Active")),  # after: dropped
+        "garbage line",
+    ]
+    s = c.summary()
+    assert s["samples"] == 3 and s["samples_outside_timed_region"] == 2
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_summary_without_samples():
+    c = bench.ClockSampler(0)
+    c.lines = []
+    assert c.summary()["samples"] == 0
+
+
+def _args(**kw):
+    a = dict(gpus=1, steps=2, warmup=1, impl="reference", config="tiny", tokens=None,
+             layers=None, algo="auto", weights="nf4", lora=0, no_cpu_baseline=False, seed=0)
+    a.update(kw)
+    return types.SimpleNamespace(**a)
+
+
+def test_reference_arm_prints_one_line(capsys, monkeypatch):
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.delenv("RANK", raising=False)
+    shape, T, layers = bench.CONFIGS["tiny"]
+    bench.run_reference(_args(), shape, T, layers)
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "tiny"
+
+
+def test_reference_arm_is_silent_on_other_ranks(capsys, monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    shape, T, layers = bench.CONFIGS["tiny"]
+    bench.run_reference(_args(), shape, T, layers)
+    assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("weights,lora", [("nf4", 0), ("int4", 0), ("nf4", 16)])
+def test_gate_up_bytes_accounting(weights, lora):
+    # the per-launch algorithmic bytes, from the formats' per-weight sizes
+    sh, T = bench.moe_synth.OLMOE, 64
+    wl = object.__new__(bench.Workload)
+    wl.shape, wl.T, wl.int4, wl.lora = sh, T, weights == "int4", lora
+    per_w = 0.5 + (4 / 128 if weights == "int4" else 4 / 64)
+    out = T * sh.k * (2 * sh.I * 4 if lora else sh.I * 2)
+    assert wl.gate_up_bytes(64) == pytest.approx(64 * 2 * sh.I * sh.H * per_w + T * sh.H * 2 + out)
+    if lora:
+        M = T * sh.k
+        want = 64 * lora * (sh.H + 2 * sh.I) * 2 + M * sh.H * 2 + 2 * M * 2 * sh.I * 4
+        assert wl.lora_bytes(64) == want
