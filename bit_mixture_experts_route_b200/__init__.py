@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     DEVERR_BAD_OFFSETS,
     DEVERR_NONFINITE,
     DEVERR_TIMEOUT,
+    DEVERR_RANGE,
     load,
     nf4_levels,
     nf4_quantize,
@@ -21,6 +22,8 @@ from ._lib import (  # noqa: F401
     int4_quantize,
     int4_grouped_gemm,
     lora_delta,
+    mxfp4_quantize,
+    mxfp4_grouped_gemm,
     permute_rows,
     swiglu,
     unpermute_combine,

@@ -24,7 +24,7 @@ DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EPI = {"none": 0, "swiglu": 1}
 ALGO = {"auto": 0, "gemv": 1, "tc": 2}
 DEVERR_NONFINITE, DEVERR_BAD_OFFSETS, DEVERR_BAD_INDEX, DEVERR_TIMEOUT = 1, 2, 4, 8
-DEVERR_LAYOUT = 16
+DEVERR_LAYOUT, DEVERR_RANGE = 0x10, 0x20
 
 # Every exported symbol with (restype, argtypes); the header declares them.
 _P, _I, _Z, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
@@ -42,6 +42,8 @@ SIGNATURES = {
                                   _I, _I, _P, _S]),
     "moe_int4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
     "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_mxfp4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
+    "moe_mxfp4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
     "moe_lora_delta": (_I, [_P, _I, _P, _I, _I, _I, _I, _P, _P, ctypes.c_float, _I, _P, _P, _S]),
     "moe_permute_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _S]),
     "moe_swiglu": (_I, [_P, _I, _I, _I, _P, _I, _S]),
@@ -221,6 +223,42 @@ def int4_grouped_gemm(A, packed, meta, expert_offsets, M_total, epilogue="none",
         _ptr(A), A.shape[0], _ptr(packed), _ptr(meta), _ptr(expert_offsets), E, N, K, M_total,
         EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
         "moe_int4_grouped_gemm")
+    return out
+
+
+def mxfp4_quantize(W, packed=None, scales=None, dev_err=None):
+    """``W fp32 [E, N, K]`` -> ``(packed u8 [E, N, K/2], scales u8 [E, N, K/32])``:
+    E2M1 codes (element 2j in the low nibble) and E8M0 scale bytes."""
+    _need(W, torch.float32, "W", 3)
+    E, N, K = W.shape
+    if packed is None:
+        packed = torch.empty((E, N, K // 2), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=W.device)
+    _check(load().moe_mxfp4_quantize(_ptr(W), E, N, K, _ptr(packed), _ptr(scales), _ptr(dev_err),
+                                     _stream(W.device)), "moe_mxfp4_quantize")
+    return packed, scales
+
+
+def mxfp4_grouped_gemm(A, packed, scales, expert_offsets, M_total, epilogue="none",
+                       out_dtype=torch.float32, out=None, dev_err=None):
+    """Decode-shaped grouped GEMM on MXFP4 weights, all experts in one launch
+    (see the header); ``A`` fp16 rows in permuted order."""
+    _need(A, torch.float16, "A", 2)
+    _need(packed, torch.uint8, "packed", 3)
+    _need(scales, torch.uint8, "scales", 3)
+    _need(expert_offsets, torch.int32, "expert_offsets", 1)
+    E, N, half = packed.shape
+    K = 2 * half
+    if A.shape[1] != K or scales.shape != (E, N, K // 32):
+        raise MoEError("A's columns and the scales must match the weights' K")
+    n_out = N // 2 if epilogue == "swiglu" else N
+    if out is None:
+        out = torch.empty((M_total, n_out), dtype=out_dtype, device=A.device)
+    _check(load().moe_mxfp4_grouped_gemm(
+        _ptr(A), A.shape[0], _ptr(packed), _ptr(scales), _ptr(expert_offsets), E, N, K, M_total,
+        EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
+        "moe_mxfp4_grouped_gemm")
     return out
 
 

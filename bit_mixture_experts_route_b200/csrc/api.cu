@@ -99,6 +99,37 @@ moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* pac
                                                  (cudaStream_t)stream));
 }
 
+moe_status_t moe_mxfp4_quantize(const float* W, int E, int N, int K, uint8_t* packed,
+                                uint8_t* scales, int32_t* dev_err, void* stream) {
+  if (E < 1 || N < 1 || K < 1 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (!W || !packed || !scales) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scales)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(moe_launch::mxfp4_quantize(W, (int64_t)E * N, K, packed, scales, dev_err,
+                                              (cudaStream_t)stream));
+}
+
+moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
+                                    const uint8_t* scales, const int32_t* expert_offsets, int E,
+                                    int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
+                                    moe_dtype_t out_dtype, int32_t* dev_err, void* stream) {
+  if (E < 1 || E > 1024 || N < 1 || K < 1 || M_total < 0 || A_rows < M_total)
+    return MOE_ERR_INVALID_ARG;
+  if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (!valid_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
+  if (!moe_launch::grouped_gemm_mxfp4_supported(N, K)) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offsets || !packed || !scales) return MOE_ERR_INVALID_ARG;
+  if (M_total > 0 && (!A || !out)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {A, packed, scales, expert_offsets, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  if (M_total == 0) return MOE_OK;
+  return from_cuda(moe_launch::grouped_gemm_mxfp4(A, A_rows, packed, scales, expert_offsets, E, N,
+                                                  K, M_total, epilogue, out, out_dtype, dev_err,
+                                                  (cudaStream_t)stream));
+}
+
 moe_status_t moe_lora_delta(const void* X, int A_rows, const int32_t* expert_offsets, int E,
                             int N, int K, int r, const void* lora_A, const void* lora_B,
                             float scale, int M_total, float* out, int32_t* dev_err,

@@ -257,6 +257,13 @@ cudaError_t grouped_gemm_int4(const void* A, int A_rows, const uint8_t* packed,
                               const uint32_t* meta, const int32_t* offsets, int E, int N, int K,
                               int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
                               int32_t* dev_err, cudaStream_t s);
+cudaError_t mxfp4_quantize(const float* W, int64_t rows, int K, uint8_t* packed, uint8_t* scales,
+                           int32_t* dev_err, cudaStream_t s);
+bool grouped_gemm_mxfp4_supported(int N, int K);
+cudaError_t grouped_gemm_mxfp4(const void* A, int A_rows, const uint8_t* packed,
+                               const uint8_t* scales, const int32_t* offsets, int E, int N, int K,
+                               int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
+                               int32_t* dev_err, cudaStream_t s);
 bool lora_delta_supported(int E, int K, int r);
 cudaError_t lora_delta(const void* X, const int32_t* offsets, int E, int N, int K, int r,
                        const void* lora_A, const void* lora_B, float scale, int M_total,

@@ -80,6 +80,8 @@ typedef enum {
 #define MOE_DEVERR_TIMEOUT 0x8     /* a bounded wait inside a kernel expired */
 #define MOE_DEVERR_LAYOUT 0x10     /* a kernel's shared-memory layout did not
                                       fit this device; the call did no work */
+#define MOE_DEVERR_RANGE 0x20      /* an MXFP4 scale lies outside the range
+                                      the decode GEMV multiplies exactly */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_string(moe_status_t status);
@@ -172,6 +174,55 @@ moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* pac
                                    const uint32_t* meta, const int32_t* expert_offsets, int E,
                                    int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
                                    moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
+
+/*
+ * moe_mxfp4_quantize -- MXFP4 quantization of a fused expert stack, the format
+ * of moe_mxfp4_grouped_gemm.  ("grouped-nf4-gemm & experts-4bit",
+ * jordananderson-pages.pages.dev, third bullet: the kernel serves MXFP4 on a
+ * checkpoint's released bytes; e2m1 + e8m0 per "MoE Training on Consumer
+ * GPUs", cerinamroth.com/ml.  Format and conversion: OCP Microscaling v1.0.)
+ *
+ *   W       fp32   [E, N, K]      input weights (device, read only)
+ *   E, N, K >= 1, K % 32 == 0
+ *   packed  uint8  [E, N, K/2]    E2M1 codes, two per byte, element 2j of a
+ *                                 row in the LOW nibble of byte j (device)
+ *   scales  uint8  [E, N, K/32]   E8M0 byte b per 32 along K, 2^(b - 127)
+ *   dev_err int32 device word or NULL; MOE_DEVERR_NONFINITE if any weight is
+ *           NaN/Inf (its block's bytes are then unspecified).
+ * Per block: shared = clamp(floor(log2 max|x|) - 2, -127, 127), b = shared +
+ * 127; codes = nearest E2M1 value of x * 2^-shared (exact in fp32), ties to
+ * the even mantissa, saturating at +-6, a value rounding to zero -> code 0;
+ * an all-zero block -> b = 0, codes 0.  Deterministic, bit-exact.
+ * W, packed and scales must be 16-byte aligned.
+ */
+moe_status_t moe_mxfp4_quantize(const float* W, int E, int N, int K, uint8_t* packed,
+                                uint8_t* scales, int32_t* dev_err, void* stream);
+
+/*
+ * moe_mxfp4_grouped_gemm -- decode-shaped grouped GEMM on MXFP4 weights:
+ * out[p] = W[e(p)] @ A[p] for every row p in expert e's segment
+ * [expert_offsets[e], expert_offsets[e+1]), W[e] = 2^(b - 127) * e2m1(code)
+ * from (packed, scales) as written by moe_mxfp4_quantize or taken unchanged
+ * from a released MXFP4 checkpoint in this layout, all experts in one launch.
+ *
+ *   A        fp16 [A_rows >= M_total, K]  routed rows in permuted order
+ *   packed   uint8 [E, N, K/2], scales uint8 [E, N, K/32]
+ *   expert_offsets int32 [E+1] (device), monotone, offsets[E] == M_total
+ *   N % 128 == 0, K % 256 == 0, E <= 1024
+ *   epilogue MOE_EPI_NONE: out [M_total, N]; MOE_EPI_SWIGLU: rows [0, N/2)
+ *            are gate and [N/2, N) up, out [M_total, N/2] = silu(g) * u
+ *   out      F32 / F16 / BF16
+ *   dev_err  BAD_OFFSETS, TIMEOUT, LAYOUT as moe_nf4_grouped_gemm; RANGE when
+ *            a scale byte is neither 0 nor in [104, 140], where the weights
+ *            are not exact in fp16 (products then rounded or flushed)
+ * The weights enter the MMA as exact fp16 values (E2M1 times the scale's power
+ * of two); sums are fp32.  Streams every selected expert's bytes once.
+ * All pointers 16-byte aligned.
+ */
+moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
+                                    const uint8_t* scales, const int32_t* expert_offsets, int E,
+                                    int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
+                                    moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
 
 /*
  * moe_lora_delta -- adds each routed row's per-expert LoRA term to an fp32

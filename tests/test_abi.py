@@ -150,3 +150,20 @@ def test_lora_delta_rejects_bad_arguments(lib):
     assert lib.moe_lora_delta(A, 4, A, 2, 64, 256, 16, A, A, 1.0, 8, A, None, None) == 1
     assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 16, None, A, 1.0, 8, A, None, None) == 1
     assert lib.moe_lora_delta(A, 8, A, 2, 64, 256, 16, A, A, 1.0, 8, M, None, None) == 2
+
+
+def test_mxfp4_calls_reject_bad_arguments(lib):
+    A, M = ALIGNED, MISALIGNED
+    # quantize: K % 32, null, misaligned
+    assert lib.moe_mxfp4_quantize(A, 1, 8, 48, A, A, None, None) == 1
+    assert lib.moe_mxfp4_quantize(A, 1, 8, 64, A, None, None, None) == 1
+    assert lib.moe_mxfp4_quantize(A, 1, 8, 64, A, M, None, None) == 2
+    # grouped GEMM: N % 128 or K % 256 -> unsupported; bad epilogue / dtype;
+    # A_rows < M_total; misaligned scales
+    g = lib.moe_mxfp4_grouped_gemm
+    assert g(A, 8, A, A, A, 2, 64, 256, 8, 0, A, 0, None, None) == 3
+    assert g(A, 8, A, A, A, 2, 128, 288, 8, 0, A, 0, None, None) == 3
+    assert g(A, 8, A, A, A, 2, 128, 256, 8, 5, A, 0, None, None) == 1
+    assert g(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 4, None, None) == 1
+    assert g(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, None, None) == 1
+    assert g(A, 8, A, M, A, 2, 128, 256, 8, 0, A, 0, None, None) == 2
