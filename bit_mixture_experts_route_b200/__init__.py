@@ -22,6 +22,10 @@ from ._lib import (  # noqa: F401
     int4_quantize,
     int4_grouped_gemm,
     lora_delta,
+    nf4_grouped_gemm_t,
+    swiglu_backward,
+    combine_backward,
+    route_backward,
     mxfp4_quantize,
     mxfp4_grouped_gemm,
     permute_rows,

@@ -44,6 +44,10 @@ SIGNATURES = {
     "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
     "moe_mxfp4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
     "moe_mxfp4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_nf4_grouped_gemm_t": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_swiglu_backward": (_I, [_P, _P, _I, _I, _I, _P, _I, _S]),
+    "moe_combine_backward": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _P, _S]),
+    "moe_route_backward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _S]),
     "moe_lora_delta": (_I, [_P, _I, _P, _I, _I, _I, _I, _P, _P, ctypes.c_float, _I, _P, _P, _S]),
     "moe_permute_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _S]),
     "moe_swiglu": (_I, [_P, _I, _I, _I, _P, _I, _S]),
@@ -259,6 +263,74 @@ def mxfp4_grouped_gemm(A, packed, scales, expert_offsets, M_total, epilogue="non
         _ptr(A), A.shape[0], _ptr(packed), _ptr(scales), _ptr(expert_offsets), E, N, K, M_total,
         EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
         "moe_mxfp4_grouped_gemm")
+    return out
+
+
+def nf4_grouped_gemm_t(G, packed, absmax, expert_offsets, M_total, out_dtype=torch.float32,
+                       out=None, dev_err=None):
+    """Transposed grouped NF4 GEMM: ``out[p] = W[e(p)]^T @ G[p]`` -> ``[M_total, K]``;
+    ``G`` fp32 or fp16 ``[>= M_total, N]`` (the backward of ``nf4_grouped_gemm``)."""
+    if G.dtype not in (torch.float32, torch.float16):
+        raise MoEError("G must be fp32 or fp16")
+    _need(G, G.dtype, "G", 2)
+    _need(packed, torch.uint8, "packed", 3)
+    _need(absmax, torch.float32, "absmax")
+    _need(expert_offsets, torch.int32, "expert_offsets", 1)
+    E, N, half = packed.shape
+    K = 2 * half
+    if G.shape[1] != N:
+        raise MoEError("G's columns must equal the weights' N")
+    if out is None:
+        out = torch.empty((M_total, K), dtype=out_dtype, device=G.device)
+    _check(load().moe_nf4_grouped_gemm_t(_ptr(G), DT[G.dtype], G.shape[0], _ptr(packed),
+                                         _ptr(absmax), _ptr(expert_offsets), E, N, K, M_total,
+                                         _ptr(out), DT[out.dtype], _ptr(dev_err),
+                                         _stream(G.device)), "moe_nf4_grouped_gemm_t")
+    return out
+
+
+def swiglu_backward(gu, dh, out_dtype=torch.float32, out=None):
+    """``gu [M, 2I]``, ``dh [M, I]`` (same dtype, fp32 or fp16) -> ``dgu [M, 2I]``."""
+    _need(gu, gu.dtype, "gu", 2)
+    _need(dh, gu.dtype, "dh", 2)
+    M, two_i = gu.shape
+    if dh.shape != (M, two_i // 2):
+        raise MoEError("dh must be [M, I] for gu [M, 2I]")
+    if out is None:
+        out = torch.empty((M, two_i), dtype=out_dtype, device=gu.device)
+    _check(load().moe_swiglu_backward(_ptr(gu), _ptr(dh), DT[gu.dtype], M, two_i // 2, _ptr(out),
+                                      DT[out.dtype], _stream(gu.device)), "moe_swiglu_backward")
+    return out
+
+
+def combine_backward(dY, Yp, inv_perm, topk_w, dyp_dtype=torch.float32, dev_err=None):
+    """Adjoint of ``unpermute_combine``: ``(dYp [T*k, H], dw fp32 [T, k])``."""
+    _need(dY, torch.float32, "dY", 2)
+    _need(Yp, Yp.dtype, "Yp", 2)
+    _need(inv_perm, torch.int32, "inv_perm")
+    _need(topk_w, torch.float32, "topk_w", 2)
+    T, k = topk_w.shape
+    H = dY.shape[1]
+    dYp = torch.empty((T * k, H), dtype=dyp_dtype, device=dY.device)
+    dw = torch.empty((T, k), dtype=torch.float32, device=dY.device)
+    _check(load().moe_combine_backward(_ptr(dY), _ptr(Yp), DT[Yp.dtype], _ptr(inv_perm),
+                                       _ptr(topk_w), T, k, H, _ptr(dYp), DT[dYp.dtype], _ptr(dw),
+                                       _ptr(dev_err), _stream(dY.device)), "moe_combine_backward")
+    return dYp, dw
+
+
+def route_backward(logits, topk_idx, topk_w, dw, renormalize, dev_err=None):
+    """Gradient of the routing weights w.r.t. the logits -> ``fp32 [T, E]``."""
+    _need(logits, torch.float32, "logits", 2)
+    _need(topk_idx, torch.int32, "topk_idx", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(dw, torch.float32, "dw", 2)
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    out = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    _check(load().moe_route_backward(_ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(dw), T, E,
+                                     k, int(bool(renormalize)), _ptr(out), _ptr(dev_err),
+                                     _stream(logits.device)), "moe_route_backward")
     return out
 
 

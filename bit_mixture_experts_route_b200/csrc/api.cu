@@ -25,6 +25,7 @@ moe_status_t from_cuda(cudaError_t e) {
 }
 
 bool valid_dtype(moe_dtype_t d) { return d == MOE_DT_F32 || d == MOE_DT_BF16 || d == MOE_DT_F16; }
+bool f32_or_f16(moe_dtype_t d) { return d == MOE_DT_F32 || d == MOE_DT_F16; }
 
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -128,6 +129,66 @@ moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* pa
   return from_cuda(moe_launch::grouped_gemm_mxfp4(A, A_rows, packed, scales, expert_offsets, E, N,
                                                   K, M_total, epilogue, out, out_dtype, dev_err,
                                                   (cudaStream_t)stream));
+}
+
+moe_status_t moe_nf4_grouped_gemm_t(const void* G, moe_dtype_t g_dtype, int G_rows,
+                                    const uint8_t* packed, const float* absmax,
+                                    const int32_t* expert_offsets, int E, int N, int K,
+                                    int M_total, void* out, moe_dtype_t out_dtype,
+                                    int32_t* dev_err, void* stream) {
+  if (!f32_or_f16(g_dtype) || !f32_or_f16(out_dtype)) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 1024 || N < 1 || K < 1 || K % moe::kBlock || M_total < 0 || G_rows < M_total)
+    return MOE_ERR_INVALID_ARG;
+  if (!expert_offsets || !packed || !absmax) return MOE_ERR_INVALID_ARG;
+  if (M_total > 0 && (!G || !out)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {G, packed, absmax, expert_offsets, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(moe_launch::grouped_gemm_t(G, g_dtype, packed, absmax, expert_offsets, E, N, K,
+                                              M_total, out, out_dtype, dev_err,
+                                              (cudaStream_t)stream));
+}
+
+moe_status_t moe_swiglu_backward(const void* gu, const void* dh, moe_dtype_t in_dtype, int M,
+                                 int I, void* dgu, moe_dtype_t out_dtype, void* stream) {
+  if (!f32_or_f16(in_dtype) || !f32_or_f16(out_dtype) || M < 0 || I < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!gu || !dh || !dgu)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {gu, dh, dgu};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(
+      moe_launch::swiglu_backward(gu, dh, in_dtype, M, I, dgu, out_dtype, (cudaStream_t)stream));
+}
+
+moe_status_t moe_combine_backward(const float* dY, const void* Yp, moe_dtype_t yp_dtype,
+                                  const int32_t* inv_perm, const float* topk_w, int T, int k,
+                                  int H, void* dYp, moe_dtype_t dyp_dtype, float* dw,
+                                  int32_t* dev_err, void* stream) {
+  if (!f32_or_f16(yp_dtype) || !f32_or_f16(dyp_dtype) || T < 0 || k < 1 || k > 32 || H < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!dY || !Yp || !inv_perm || !topk_w || !dYp || !dw)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {dY, Yp, inv_perm, topk_w, dYp, dw};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(moe_launch::combine_backward(dY, Yp, yp_dtype, inv_perm, topk_w, T, k, H, dYp,
+                                                dyp_dtype, dw, dev_err, (cudaStream_t)stream));
+}
+
+moe_status_t moe_route_backward(const float* logits, const int32_t* topk_idx,
+                                const float* topk_w, const float* dw, int T, int E, int k,
+                                int renormalize, float* dlogits, int32_t* dev_err, void* stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_idx || !topk_w || !dw || !dlogits)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {logits, topk_idx, topk_w, dw, dlogits};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  return from_cuda(moe_launch::route_backward(logits, topk_idx, topk_w, dw, T, E, k, renormalize,
+                                              dlogits, dev_err, (cudaStream_t)stream));
 }
 
 moe_status_t moe_lora_delta(const void* X, int A_rows, const int32_t* expert_offsets, int E,

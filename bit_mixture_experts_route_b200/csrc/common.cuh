@@ -264,6 +264,19 @@ cudaError_t grouped_gemm_mxfp4(const void* A, int A_rows, const uint8_t* packed,
                                const uint8_t* scales, const int32_t* offsets, int E, int N, int K,
                                int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
                                int32_t* dev_err, cudaStream_t s);
+cudaError_t grouped_gemm_t(const void* G, moe_dtype_t g_dt, const uint8_t* packed,
+                           const float* absmax, const int32_t* offsets, int E, int N, int K,
+                           int M_total, void* out, moe_dtype_t out_dt, int32_t* dev_err,
+                           cudaStream_t s);
+cudaError_t swiglu_backward(const void* gu, const void* dh, moe_dtype_t in_dt, int M, int I,
+                            void* dgu, moe_dtype_t out_dt, cudaStream_t s);
+cudaError_t combine_backward(const float* dY, const void* Yp, moe_dtype_t yp_dt,
+                             const int32_t* inv_perm, const float* topk_w, int T, int k, int H,
+                             void* dYp, moe_dtype_t dyp_dt, float* dw, int32_t* dev_err,
+                             cudaStream_t s);
+cudaError_t route_backward(const float* logits, const int32_t* topk_idx, const float* topk_w,
+                           const float* dw, int T, int E, int k, int renormalize, float* dlogits,
+                           int32_t* dev_err, cudaStream_t s);
 bool lora_delta_supported(int E, int K, int r);
 cudaError_t lora_delta(const void* X, const int32_t* offsets, int E, int N, int K, int r,
                        const void* lora_A, const void* lora_B, float scale, int M_total,

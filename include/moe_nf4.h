@@ -225,6 +225,66 @@ moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* pa
                                     moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
 
 /*
+ * Backward of the layer with the 4-bit experts frozen ("grouped-nf4-gemm &
+ * experts-4bit", jordananderson-pages.pages.dev, fourth bullet: fine-tuning
+ * computes on the packed 4-bit weights, which stay byte-identical).  The
+ * gradients are the chain rule through the forward calls above; the
+ * scatter-add of routed-row gradients into tokens is moe_unpermute_combine
+ * with unit weights.  No weight gradient exists.
+ *
+ * moe_nf4_grouped_gemm_t -- out[p] = W[e(p)]^T @ G[p] for every row p in
+ * expert e's segment, W[e] the NF4 weights of moe_nf4_grouped_gemm.
+ *   G        F32 or F16 [G_rows >= M_total, N]   (device)
+ *   packed   uint8 [E, N, K/2], absmax fp32 [E, N*K/64]  (the forward's)
+ *   expert_offsets int32 [E+1] (device), monotone, offsets[E] == M_total,
+ *            else MOE_DEVERR_BAD_OFFSETS and no output
+ *   out      F32 or F16 [M_total, K]
+ *   E <= 1024, K % 64 == 0.  fp32 sums.  All pointers 16-byte aligned.
+ */
+moe_status_t moe_nf4_grouped_gemm_t(const void* G, moe_dtype_t g_dtype, int G_rows,
+                                    const uint8_t* packed, const float* absmax,
+                                    const int32_t* expert_offsets, int E, int N, int K,
+                                    int M_total, void* out, moe_dtype_t out_dtype,
+                                    int32_t* dev_err, void* stream);
+
+/*
+ * moe_swiglu_backward -- for gu [M, 2I] (gate | up pre-activations) and
+ * dh [M, I], both of in_dtype (F32 or F16): with s = sigmoid(g),
+ * dgu[m, i] = dh u s (1 + g (1 - s)) and dgu[m, I + i] = dh g s, into
+ * dgu [M, 2I] of out_dtype (F32 or F16).  Pointers 16-byte aligned.
+ */
+moe_status_t moe_swiglu_backward(const void* gu, const void* dh, moe_dtype_t in_dtype, int M,
+                                 int I, void* dgu, moe_dtype_t out_dtype, void* stream);
+
+/*
+ * moe_combine_backward -- adjoint of moe_unpermute_combine: for every routed
+ * row f = t*k + j at position pos = inv_perm[f],
+ *   dYp[pos, :] = topk_w[f] * dY[t, :]      (dYp [T*k, H] of dyp_dtype)
+ *   dw[f]       = <dY[t, :], Yp[pos, :]>   (fp32 [T, k], fp32 sums)
+ *   dY fp32 [T, H]; Yp [T*k, H] of yp_dtype (F32 or F16, the forward's);
+ *   1 <= k <= 32.  An inv_perm entry out of range sets MOE_DEVERR_BAD_INDEX
+ *   and that row's dw to 0.  Pointers 16-byte aligned.
+ */
+moe_status_t moe_combine_backward(const float* dY, const void* Yp, moe_dtype_t yp_dtype,
+                                  const int32_t* inv_perm, const float* topk_w, int T, int k,
+                                  int H, void* dYp, moe_dtype_t dyp_dtype, float* dw,
+                                  int32_t* dev_err, void* stream);
+
+/*
+ * moe_route_backward -- gradient of the routing weights w.r.t. the logits,
+ * the selection held fixed: renormalize != 0: dl[e_j] = w_j (dw_j - sum_j'
+ * dw_j' w_j') and 0 elsewhere; renormalize == 0 (w = softmax probabilities):
+ * dl_i = [i = e_j] dw_j w_j - p_i sum_j dw_j w_j with p = softmax(logits).
+ *   logits fp32 [T, E]; topk_idx int32 [T, k] and topk_w fp32 [T, k] (the
+ *   forward's outputs); dw fp32 [T, k]; dlogits fp32 [T, E].
+ *   1 <= k <= min(E, 32), E <= 1024.  An expert index out of range sets
+ *   MOE_DEVERR_BAD_INDEX and is skipped.  Pointers 16-byte aligned.
+ */
+moe_status_t moe_route_backward(const float* logits, const int32_t* topk_idx,
+                                const float* topk_w, const float* dw, int T, int E, int k,
+                                int renormalize, float* dlogits, int32_t* dev_err, void* stream);
+
+/*
  * moe_lora_delta -- adds each routed row's per-expert LoRA term to an fp32
  * pre-activation in place: out[p] += scale * B[e(p)] @ (A[e(p)] @ X[p]) for
  * every row p in expert e's segment [expert_offsets[e], expert_offsets[e+1]).

@@ -167,3 +167,23 @@ def test_mxfp4_calls_reject_bad_arguments(lib):
     assert g(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 4, None, None) == 1
     assert g(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, None, None) == 1
     assert g(A, 8, A, M, A, 2, 128, 256, 8, 0, A, 0, None, None) == 2
+
+
+def test_backward_calls_reject_bad_arguments(lib):
+    A, M = ALIGNED, MISALIGNED
+    # transposed GEMM: (G, g_dtype, G_rows, packed, absmax, offsets, E, N, K, M_total, out,
+    # out_dtype, dev_err, stream): bf16 G, K % 64, G_rows < M_total, misaligned out
+    t = lib.moe_nf4_grouped_gemm_t
+    assert t(A, 1, 8, A, A, A, 2, 128, 256, 8, A, 0, None, None) == 1
+    assert t(A, 0, 8, A, A, A, 2, 128, 96, 8, A, 0, None, None) == 1
+    assert t(A, 0, 4, A, A, A, 2, 128, 256, 8, A, 0, None, None) == 1
+    assert t(A, 0, 8, A, A, A, 2, 128, 256, 8, M, 0, None, None) == 2
+    # SwiGLU backward: bf16 inputs, null dh
+    assert lib.moe_swiglu_backward(A, A, 1, 4, 8, A, 0, None) == 1
+    assert lib.moe_swiglu_backward(A, None, 0, 4, 8, A, 0, None) == 1
+    # combine backward: k > 32, misaligned dw
+    assert lib.moe_combine_backward(A, A, 0, A, A, 2, 33, 8, A, 0, A, None, None) == 1
+    assert lib.moe_combine_backward(A, A, 0, A, A, 2, 2, 8, A, 0, M, None, None) == 2
+    # routing backward: k > E, E > 1024
+    assert lib.moe_route_backward(A, A, A, A, 2, 4, 5, 1, A, None, None) == 1
+    assert lib.moe_route_backward(A, A, A, A, 2, 2048, 8, 1, A, None, None) == 1
