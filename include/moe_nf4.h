@@ -12,6 +12,11 @@
  * .pages.dev), first bullet, and in the "grouped-nf4-gemm" bullet of the
  * pjordanandrsn GitHub profile page.
  *
+ * Beyond the NF4 forward: the same grouped GEMV on GPTQ-style INT4 and on
+ * MXFP4 weights, a per-expert LoRA delta, and the backward steps of the layer
+ * with the 4-bit experts frozen (transposed grouped GEMM, SwiGLU, combine and
+ * routing backward).
+ *
  * Conventions shared by every call
  * --------------------------------
  * - All pointers are DEVICE pointers unless a parameter says otherwise; the
