@@ -107,6 +107,25 @@ def _need(t, dtype, name, ndim=None):
         raise MoEError(f"{name} must have {ndim} dims")
 
 
+def _room(t, n, name, dtypes=None):
+    """``t`` is a contiguous CUDA tensor (of one of ``dtypes``) with at least
+    ``n`` elements: the kernels address that many, so a smaller buffer would
+    be read or written out of bounds on the device."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise MoEError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise MoEError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise MoEError(f"{name} must be one of {dtypes}, got {t.dtype}")
+    if t.numel() < n:
+        raise MoEError(f"{name} has {t.numel()} elements, the call needs {n}")
+
+
+_F = (torch.float32, torch.bfloat16, torch.float16)
+
+
 def nf4_levels():
     buf = (ctypes.c_float * 16)()
     _check(load().moe_nf4_levels(ctypes.cast(buf, ctypes.c_void_p)), "moe_nf4_levels")
@@ -121,6 +140,8 @@ def nf4_quantize(W, packed=None, absmax=None, dev_err=None):
         packed = torch.empty((E, N, K // 2), dtype=torch.uint8, device=W.device)
     if absmax is None:
         absmax = torch.empty((E, N * K // 64), dtype=torch.float32, device=W.device)
+    _room(packed, E * N * (K // 2), "packed", (torch.uint8,))
+    _room(absmax, E * N * (K // 64), "absmax", (torch.float32,))
     _check(load().moe_nf4_quantize(_ptr(W), E, N, K, 64, _ptr(packed), _ptr(absmax),
                                    _ptr(dev_err), _stream(W.device)), "moe_nf4_quantize")
     return packed, absmax
@@ -129,6 +150,7 @@ def nf4_quantize(W, packed=None, absmax=None, dev_err=None):
 def nf4_dequantize(packed, absmax, out_dtype=torch.float32):
     _need(packed, torch.uint8, "packed", 3)
     E, N, half = packed.shape
+    _room(absmax, E * N * (2 * half // 64), "absmax", (torch.float32,))
     out = torch.empty((E, N, 2 * half), dtype=out_dtype, device=packed.device)
     _check(load().moe_nf4_dequantize(_ptr(packed), _ptr(absmax), E, N, 2 * half, _ptr(out),
                                      DT[out_dtype], _stream(packed.device)),
@@ -157,9 +179,14 @@ def route_permute(logits, k, renormalize=True, workspace=None, out=None):
             "sorted_rows": torch.empty((T * k,), dtype=torch.int32, device=dev),
             "inv_perm": torch.empty((T * k,), dtype=torch.int32, device=dev),
         }
+    for key, n, dt in (("topk_idx", T * k, torch.int32), ("topk_w", T * k, torch.float32),
+                       ("expert_offsets", E + 1, torch.int32), ("sorted_rows", T * k, torch.int32),
+                       ("inv_perm", T * k, torch.int32)):
+        _room(out[key], n, key, (dt,))
     nbytes = route_permute_workspace_size(T, E, k)
     if workspace is None:
         workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=dev)
+    _room(workspace, 0, "workspace")
     _check(load().moe_route_permute(
         _ptr(logits), T, E, k, 1 if renormalize else 0, _ptr(out["topk_idx"]),
         _ptr(out["topk_w"]), _ptr(out["expert_offsets"]), _ptr(out["sorted_rows"]),
@@ -184,9 +211,13 @@ def nf4_grouped_gemm(A, packed, absmax, expert_offsets, M_total, gather=None, k=
         raise MoEError("A's columns must equal the weights' K")
     if gather is not None:
         _need(gather, torch.int32, "gather", 1)
+        _room(gather, M_total, "gather")
+    _room(absmax, E * N * (K // 64), "absmax")
+    _room(expert_offsets, E + 1, "expert_offsets")
     n_out = N // 2 if epilogue == "swiglu" else N
     if out is None:
         out = torch.empty((M_total, n_out), dtype=out_dtype, device=A.device)
+    _room(out, M_total * n_out, "out", _F)
     _check(load().moe_nf4_grouped_gemm(
         _ptr(A), DT[A.dtype], A.shape[0], _ptr(gather), k, _ptr(packed), _ptr(absmax),
         _ptr(expert_offsets), E, N, K, M_total, EPI[epilogue], _ptr(out), DT[out.dtype],
@@ -203,6 +234,8 @@ def int4_quantize(W, packed=None, meta=None, dev_err=None):
         packed = torch.empty((E, N, K // 2), dtype=torch.uint8, device=W.device)
     if meta is None:
         meta = torch.empty((E, N, K // 128), dtype=torch.int32, device=W.device)
+    _room(packed, E * N * (K // 2), "packed", (torch.uint8,))
+    _room(meta, E * N * (K // 128), "meta", (torch.int32,))
     _check(load().moe_int4_quantize(_ptr(W), E, N, K, _ptr(packed), _ptr(meta), _ptr(dev_err),
                                     _stream(W.device)), "moe_int4_quantize")
     return packed, meta
@@ -220,9 +253,12 @@ def int4_grouped_gemm(A, packed, meta, expert_offsets, M_total, epilogue="none",
     K = 2 * half
     if A.shape[1] != K:
         raise MoEError("A's columns must equal the weights' K")
+    _room(meta, E * N * (K // 128), "meta")
+    _room(expert_offsets, E + 1, "expert_offsets")
     n_out = N // 2 if epilogue == "swiglu" else N
     if out is None:
         out = torch.empty((M_total, n_out), dtype=out_dtype, device=A.device)
+    _room(out, M_total * n_out, "out", _F)
     _check(load().moe_int4_grouped_gemm(
         _ptr(A), A.shape[0], _ptr(packed), _ptr(meta), _ptr(expert_offsets), E, N, K, M_total,
         EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
@@ -239,6 +275,8 @@ def mxfp4_quantize(W, packed=None, scales=None, dev_err=None):
         packed = torch.empty((E, N, K // 2), dtype=torch.uint8, device=W.device)
     if scales is None:
         scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=W.device)
+    _room(packed, E * N * (K // 2), "packed", (torch.uint8,))
+    _room(scales, E * N * (K // 32), "scales", (torch.uint8,))
     _check(load().moe_mxfp4_quantize(_ptr(W), E, N, K, _ptr(packed), _ptr(scales), _ptr(dev_err),
                                      _stream(W.device)), "moe_mxfp4_quantize")
     return packed, scales
@@ -256,9 +294,11 @@ def mxfp4_grouped_gemm(A, packed, scales, expert_offsets, M_total, epilogue="non
     K = 2 * half
     if A.shape[1] != K or scales.shape != (E, N, K // 32):
         raise MoEError("A's columns and the scales must match the weights' K")
+    _room(expert_offsets, E + 1, "expert_offsets")
     n_out = N // 2 if epilogue == "swiglu" else N
     if out is None:
         out = torch.empty((M_total, n_out), dtype=out_dtype, device=A.device)
+    _room(out, M_total * n_out, "out", _F)
     _check(load().moe_mxfp4_grouped_gemm(
         _ptr(A), A.shape[0], _ptr(packed), _ptr(scales), _ptr(expert_offsets), E, N, K, M_total,
         EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
@@ -280,8 +320,11 @@ def nf4_grouped_gemm_t(G, packed, absmax, expert_offsets, M_total, out_dtype=tor
     K = 2 * half
     if G.shape[1] != N:
         raise MoEError("G's columns must equal the weights' N")
+    _room(absmax, E * N * (K // 64), "absmax")
+    _room(expert_offsets, E + 1, "expert_offsets")
     if out is None:
         out = torch.empty((M_total, K), dtype=out_dtype, device=G.device)
+    _room(out, M_total * K, "out", (torch.float32, torch.float16))
     _check(load().moe_nf4_grouped_gemm_t(_ptr(G), DT[G.dtype], G.shape[0], _ptr(packed),
                                          _ptr(absmax), _ptr(expert_offsets), E, N, K, M_total,
                                          _ptr(out), DT[out.dtype], _ptr(dev_err),
@@ -298,6 +341,7 @@ def swiglu_backward(gu, dh, out_dtype=torch.float32, out=None):
         raise MoEError("dh must be [M, I] for gu [M, 2I]")
     if out is None:
         out = torch.empty((M, two_i), dtype=out_dtype, device=gu.device)
+    _room(out, M * two_i, "out", (torch.float32, torch.float16))
     _check(load().moe_swiglu_backward(_ptr(gu), _ptr(dh), DT[gu.dtype], M, two_i // 2, _ptr(out),
                                       DT[out.dtype], _stream(gu.device)), "moe_swiglu_backward")
     return out
@@ -311,6 +355,10 @@ def combine_backward(dY, Yp, inv_perm, topk_w, dyp_dtype=torch.float32, dev_err=
     _need(topk_w, torch.float32, "topk_w", 2)
     T, k = topk_w.shape
     H = dY.shape[1]
+    if dY.shape[0] != T:
+        raise MoEError("dY must have one row per token of topk_w")
+    _room(Yp, T * k * H, "Yp", (torch.float32, torch.float16))
+    _room(inv_perm, T * k, "inv_perm")
     dYp = torch.empty((T * k, H), dtype=dyp_dtype, device=dY.device)
     dw = torch.empty((T, k), dtype=torch.float32, device=dY.device)
     _check(load().moe_combine_backward(_ptr(dY), _ptr(Yp), DT[Yp.dtype], _ptr(inv_perm),
@@ -327,6 +375,9 @@ def route_backward(logits, topk_idx, topk_w, dw, renormalize, dev_err=None):
     _need(dw, torch.float32, "dw", 2)
     T, E = logits.shape
     k = topk_idx.shape[1]
+    for t, name in ((topk_idx, "topk_idx"), (topk_w, "topk_w"), (dw, "dw")):
+        if tuple(t.shape) != (T, k):
+            raise MoEError(f"{name} must be [T, k] = [{T}, {k}]")
     out = torch.empty((T, E), dtype=torch.float32, device=logits.device)
     _check(load().moe_route_backward(_ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(dw), T, E,
                                      k, int(bool(renormalize)), _ptr(out), _ptr(dev_err),
@@ -350,6 +401,7 @@ def lora_delta(X, expert_offsets, lora_A, lora_B, scale, out, M_total=None, dev_
     M = out.shape[0] if M_total is None else M_total
     if out.shape[0] < M:
         raise MoEError("out has fewer than M_total rows")
+    _room(expert_offsets, E + 1, "expert_offsets")
     _check(load().moe_lora_delta(_ptr(X), X.shape[0], _ptr(expert_offsets), E, N, K, r,
                                  _ptr(lora_A), _ptr(lora_B), float(scale), M, _ptr(out),
                                  _ptr(dev_err), _stream(X.device)), "moe_lora_delta")
@@ -364,8 +416,10 @@ def permute_rows(X, sorted_rows, k, M_total=None, out=None, dev_err=None):
     _need(sorted_rows, torch.int32, "sorted_rows", 1)
     T, K = X.shape
     M = sorted_rows.numel() if M_total is None else M_total
+    _room(sorted_rows, M, "sorted_rows")
     if out is None:
         out = torch.empty((M, K), dtype=torch.float16, device=X.device)
+    _room(out, M * K, "out", (torch.float16,))
     _check(load().moe_permute_rows(_ptr(X), DT[X.dtype], T, K, _ptr(sorted_rows), k, M,
                                    _ptr(out), _ptr(dev_err), _stream(X.device)),
            "moe_permute_rows")
@@ -377,6 +431,7 @@ def swiglu(gu, h_dtype=torch.float32, out=None):
     M, two_i = gu.shape
     if out is None:
         out = torch.empty((M, two_i // 2), dtype=h_dtype, device=gu.device)
+    _room(out, M * (two_i // 2), "out", _F)
     _check(load().moe_swiglu(_ptr(gu), DT[gu.dtype], M, two_i // 2, _ptr(out), DT[out.dtype],
                              _stream(gu.device)), "moe_swiglu")
     return out
@@ -388,8 +443,11 @@ def unpermute_combine(Yp, inv_perm, topk_w, y_dtype=torch.float32, out=None):
     _need(topk_w, torch.float32, "topk_w", 2)
     T, k = topk_w.shape
     H = Yp.shape[1]
+    _room(Yp, T * k * H, "Yp", _F)
+    _room(inv_perm, T * k, "inv_perm")
     if out is None:
         out = torch.empty((T, H), dtype=y_dtype, device=Yp.device)
+    _room(out, T * H, "out", _F)
     _check(load().moe_unpermute_combine(_ptr(Yp), DT[Yp.dtype], _ptr(inv_perm), _ptr(topk_w),
                                         T, k, H, _ptr(out), DT[out.dtype], _stream(Yp.device)),
            "moe_unpermute_combine")
@@ -411,11 +469,19 @@ def layer_forward(X, logits, k, renormalize, packed_gu, absmax_gu, packed_d, abs
     T, H = X.shape
     E = logits.shape[1]
     I = packed_d.shape[2] * 2
+    if logits.shape[0] != T:
+        raise MoEError("logits must have one row per token of X")
+    _room(packed_gu, E * 2 * I * (H // 2), "packed_gu", (torch.uint8,))
+    _room(absmax_gu, E * 2 * I * (H // 64), "absmax_gu", (torch.float32,))
+    _room(packed_d, E * H * (I // 2), "packed_d", (torch.uint8,))
+    _room(absmax_d, E * H * (I // 64), "absmax_d", (torch.float32,))
     nbytes = layer_workspace_size(T, E, k, H, I)
     if workspace is None:
         workspace = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=X.device)
     if out is None:
         out = torch.empty((T, H), dtype=torch.float32, device=X.device)
+    _room(out, T * H, "out", (torch.float32,))
+    _room(workspace, 0, "workspace")
     _check(load().moe_layer_forward(
         _ptr(X), _ptr(logits), T, E, k, 1 if renormalize else 0, H, I, _ptr(packed_gu),
         _ptr(absmax_gu), _ptr(packed_d), _ptr(absmax_d), _ptr(out), _ptr(workspace),
