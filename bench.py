@@ -54,8 +54,11 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=None, help="token batch T")
     p.add_argument("--layers", type=int, default=None)
     p.add_argument("--algo", choices=["auto", "gemv", "tc"], default="auto")
-    p.add_argument("--weights", choices=["nf4", "int4"], default="nf4",
-                   help="expert weight format (int4: grouped GPTQ-style codes, decode GEMV)")
+    p.add_argument("--weights", choices=["nf4", "int4", "mxfp4"], default="nf4",
+                   help="expert weight format (int4: grouped GPTQ-style codes; mxfp4: e2m1 + "
+                        "e8m0 per 32; both run the decode GEMV only)")
+    p.add_argument("--backward", action="store_true",
+                   help="time forward + backward of each layer (4-bit experts frozen)")
     p.add_argument("--lora", type=int, default=0, metavar="RANK",
                    help="per-expert LoRA adapters of this rank on both projections "
                         "(0 = none)")
@@ -216,14 +219,23 @@ def rank_seed(seed, rank):
 
 # ----------------------------------------------------------------- workload
 
+# bytes per weight: the 4-bit code plus its share of the scales (NF4: fp32
+# absmax per 64; INT4: fp16 scale + zero in 4 B per 128; MXFP4: 1 B per 32)
+BYTES_PER_WEIGHT = {"nf4": 0.5625, "int4": 0.53125, "mxfp4": 0.53125}
+DECODE_KERNEL_SOURCE = {"nf4": "grouped_gemm_decode.cu", "int4": "grouped_gemm_int4.cu",
+                        "mxfp4": "grouped_gemm_mxfp4.cu"}
+
 class Workload:
-    def __init__(self, shape, T, layers, seed, device="cuda", weights="nf4", lora=0):
+    def __init__(self, shape, T, layers, seed, device="cuda", weights="nf4", lora=0,
+                 backward=False):
         import bit_mixture_experts_route_b200 as moe
         self.moe = moe
         self.shape, self.T, self.L = shape, T, layers
-        self.int4 = weights == "int4"
+        self.fmt = weights
         self.lora = lora
-        quantize = moe.int4_quantize if self.int4 else moe.nf4_quantize
+        self.backward = backward
+        quantize = {"nf4": moe.nf4_quantize, "int4": moe.int4_quantize,
+                    "mxfp4": moe.mxfp4_quantize}[weights]
         self.stacks = []
         for layer in range(layers):
             s = seed * 1000 + layer
@@ -256,16 +268,23 @@ class Workload:
         self.Y = torch.empty((T, H), dtype=torch.float32, device=dev)
         self.lws = torch.empty((max(moe.layer_workspace_size(T, E, k, H, I), 256),),
                                dtype=torch.uint8, device=dev)
+        if lora or backward:
+            # both GEMMs write fp32 pre-activations (the adapters add their
+            # term in place; the backward needs gate_up's), SwiGLU standalone
+            self.GU = torch.empty((M, 2 * I), dtype=torch.float32, device=dev)
+            self.Yp32 = torch.empty((M, H), dtype=torch.float32, device=dev)
+        if backward:
+            g = torch.Generator(device=dev)
+            g.manual_seed(seed * 1000 + 999)
+            self.dY = torch.randn((T, H), generator=g, device=dev, dtype=torch.float32)
+            self.ones = torch.ones((T, k), dtype=torch.float32, device=dev)
+            self.dX = torch.empty((T, H), dtype=torch.float32, device=dev)
         if lora:
-            # adapted path: both GEMMs write fp32 pre-activations, the adapters
-            # add their term in place, SwiGLU runs standalone
             self.adapters = [moe_synth.lora_adapters(shape, "gate_up", lora, seed * 1000 + layer,
                                                      device=dev)
                              + moe_synth.lora_adapters(shape, "down", lora, seed * 1000 + layer,
                                                        device=dev)
                              for layer in range(layers)]
-            self.GU = torch.empty((M, 2 * I), dtype=torch.float32, device=dev)
-            self.Yp32 = torch.empty((M, H), dtype=torch.float32, device=dev)
 
     def layer(self, layer, algo="auto", ev=None, X=None, logits=None):
         moe, sh, T = self.moe, self.shape, self.T
@@ -275,53 +294,59 @@ class Workload:
         r = moe.route_permute(logits, sh.k, sh.renormalize, workspace=self.rws, out=self.route)
         M = T * sh.k
         moe.permute_rows(X, r["sorted_rows"], sh.k, out=self.Xp)
-        if self.lora:
-            self._adapted_layer(layer, r, M, algo, ev)
+        if self.lora or self.backward:
+            self._adapted_layer(layer, r, M, algo, ev, logits)
             return
         if ev is not None:
             ev[0].record()
-        if self.int4:
-            moe.int4_grouped_gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, epilogue="swiglu",
-                                  out=self.Hbuf)
-        else:
-            moe.nf4_grouped_gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, epilogue="swiglu",
-                                 out=self.Hbuf, algo=algo)
+        self._gemm(self.Xp, p_gu, a_gu, r["expert_offsets"], M, self.Hbuf, algo, "swiglu")
         if ev is not None:
             ev[1].record()
-        if self.int4:
-            moe.int4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
-                                  out=self.Yp)
-        else:
-            moe.nf4_grouped_gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, epilogue="none",
-                                 out=self.Yp, algo=algo)
+        self._gemm(self.Hbuf, p_d, a_d, r["expert_offsets"], M, self.Yp, algo)
         moe.unpermute_combine(self.Yp, r["inv_perm"], r["topk_w"], out=self.Y)
 
-    def _gemm(self, A, packed, scales, offsets, M, out, algo):
-        if self.int4:
-            self.moe.int4_grouped_gemm(A, packed, scales, offsets, M, epilogue="none", out=out)
+    def _gemm(self, A, packed, scales, offsets, M, out, algo, epilogue="none"):
+        if self.fmt == "int4":
+            self.moe.int4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out)
+        elif self.fmt == "mxfp4":
+            self.moe.mxfp4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out)
         else:
-            self.moe.nf4_grouped_gemm(A, packed, scales, offsets, M, epilogue="none", out=out,
+            self.moe.nf4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out,
                                       algo=algo)
 
-    def _adapted_layer(self, layer, r, M, algo, ev):
+    def _adapted_layer(self, layer, r, M, algo, ev, logits):
+        """Forward with fp32 pre-activations (plus the adapters' deltas when
+        adapted), then, with --backward, the layer's backward for a fixed
+        output gradient: combine backward, transposed down, SwiGLU backward,
+        transposed gate_up, scatter-add into tokens, routing backward."""
         moe = self.moe
         p_gu, a_gu, p_d, a_d = self.stacks[layer]
-        A_gu, B_gu, A_d, B_d = self.adapters[layer]
         off = r["expert_offsets"]
-        scale = 32.0 / self.lora     # alpha = 32
+        if self.lora:
+            A_gu, B_gu, A_d, B_d = self.adapters[layer]
+            scale = 32.0 / self.lora     # alpha = 32
         if ev is not None:
             ev[0].record()
         self._gemm(self.Xp, p_gu, a_gu, off, M, self.GU, algo)
         if ev is not None:
             ev[1].record()
             ev[2].record()
-        moe.lora_delta(self.Xp, off, A_gu, B_gu, scale, self.GU, M_total=M)
+        if self.lora:
+            moe.lora_delta(self.Xp, off, A_gu, B_gu, scale, self.GU, M_total=M)
         if ev is not None:
             ev[3].record()
         moe.swiglu(self.GU, out=self.Hbuf)
         self._gemm(self.Hbuf, p_d, a_d, off, M, self.Yp32, algo)
-        moe.lora_delta(self.Hbuf, off, A_d, B_d, scale, self.Yp32, M_total=M)
+        if self.lora:
+            moe.lora_delta(self.Hbuf, off, A_d, B_d, scale, self.Yp32, M_total=M)
         moe.unpermute_combine(self.Yp32, r["inv_perm"], r["topk_w"], out=self.Y)
+        if self.backward:
+            dYp, dw = moe.combine_backward(self.dY, self.Yp32, r["inv_perm"], r["topk_w"])
+            dH = moe.nf4_grouped_gemm_t(dYp, p_d, a_d, off, M)
+            dGU = moe.swiglu_backward(self.GU, dH)
+            dXp = moe.nf4_grouped_gemm_t(dGU, p_gu, a_gu, off, M)
+            moe.unpermute_combine(dXp, r["inv_perm"], self.ones, out=self.dX)
+            moe.route_backward(logits, r["topk_idx"], r["topk_w"], dw, self.shape.renormalize)
 
     def lora_bytes(self, d):
         """Algorithmic bytes of the gate_up adapter launch: the distinct
@@ -347,16 +372,14 @@ class Workload:
 
     def gate_up_bytes(self, d):
         sh, T = self.shape, self.T
-        # per weight: 4-bit code + fp32 absmax per 64 (NF4) or fp16 scale and
-        # zero in 4 bytes per 128 (INT4)
-        w = d * (2 * sh.I * sh.H) * (0.53125 if self.int4 else 0.5625)
+        w = d * (2 * sh.I * sh.H) * BYTES_PER_WEIGHT[self.fmt]
         # output: fp16 SwiGLU rows, or fp32 gate_up pre-activations when adapted
-        out = T * sh.k * 2 * sh.I * 4 if self.lora else T * sh.k * sh.I * 2
+        out = T * sh.k * 2 * sh.I * 4 if (self.lora or self.backward) else T * sh.k * sh.I * 2
         return w + T * sh.H * 2 + out
 
     def layer_bytes(self, d):
         sh, T = self.shape, self.T
-        per_w = 0.53125 if self.int4 else 0.5625
+        per_w = BYTES_PER_WEIGHT[self.fmt]
         return d * 3 * sh.H * sh.I * per_w + T * sh.H * 2 + T * sh.E * 4 + T * sh.H * 4
 
     def gate_up_flops(self):
@@ -368,7 +391,7 @@ class Workload:
 
 def oracle_sample(shape, T, seed, n_tokens, start_token=0, threads=None, weights="nf4"):
     """Time the oracle on ``n_tokens`` tokens of layer 0: dequantize the NF4
-    (or INT4) experts they need and run the per-token expert MLPs.  Weights
+    (or INT4, MXFP4) experts they need and run the per-token expert MLPs.  Weights
     come from the same generator as the GPU run; quantization is untimed
     setup."""
     import oracle
@@ -382,6 +405,18 @@ def oracle_sample(shape, T, seed, n_tokens, start_token=0, threads=None, weights
     w_gu = moe_synth.weights(shape, "gate_up", s, experts=experts, device=dev).cpu().numpy()
     w_d = moe_synth.weights(shape, "down", s, experts=experts, device=dev).cpu().numpy()
     E, I, H = shape.E, shape.I, shape.H
+    if weights == "mxfp4":
+        p_gu = np.zeros((E, 2 * I, H // 2), np.uint8)
+        s_gu = np.zeros((E, 2 * I, H // 32), np.uint8)
+        p_d = np.zeros((E, H, I // 2), np.uint8)
+        s_d = np.zeros((E, H, I // 32), np.uint8)
+        for i, e in enumerate(experts):
+            p_gu[e], s_gu[e] = oracle.quantize_mxfp4(w_gu[i])
+            p_d[e], s_d[e] = oracle.quantize_mxfp4(w_d[i])
+        stack = oracle.Mxfp4ExpertStack(p_gu, s_gu, p_d, s_d)
+        t0 = time.perf_counter()
+        oracle.moe_layer(X, lg, stack, shape.k, shape.renormalize, tokens=toks)
+        return n_tokens, time.perf_counter() - t0
     if weights == "int4":
         p_gu = np.zeros((E, 2 * I, H // 2), np.uint8)
         m_gu = np.zeros((E, 2 * I, H // 128), np.uint32)
@@ -497,11 +532,13 @@ def main():
     world, rank, local = dist_setup()
     import bit_mixture_experts_route_b200 as moe
     moe.load()
+    if args.weights != "nf4" and T * shape.k >= 36 * shape.E:
+        raise SystemExit(f"{args.weights} weights have the decode GEMV path only (fewer than 36 "
+                         "routed rows per expert)")
+    if args.backward and args.weights != "nf4":
+        raise SystemExit("--backward runs on NF4 weights (the transposed GEMM is NF4)")
     wl = Workload(shape, T, layers, rank_seed(args.seed, rank), weights=args.weights,
-                  lora=args.lora)
-    if args.weights == "int4" and T * shape.k >= 36 * shape.E:
-        raise SystemExit("int4 weights have the decode GEMV path only (fewer than 36 routed "
-                         "rows per expert)")
+                  lora=args.lora, backward=args.backward)
     hbm, tf_burst, tf_sust, peak_kind = load_peaks()
     stream = torch.cuda.current_stream()
 
@@ -512,7 +549,7 @@ def main():
 
     # ---- timed region: K steps, events around every gate_up launch (and the
     # gate_up adapter launch when adapted)
-    n_ev = 4 if args.lora else 2
+    n_ev = 4 if (args.lora or args.backward) else 2
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
             for _ in range(layers)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -542,9 +579,10 @@ def main():
     # the tensor-core kernel serves the GEMMs from 36 routed rows per expert
     # on average (the AUTO dispatch rule); below that the decode GEMV does
     prefill = T * shape.k >= 36 * shape.E
-    workload_name = (args.config + ("/int4" if args.weights == "int4" else "")
-                     + (f"/lora-r{args.lora}" if args.lora else ""))
-    epi_name = "(fp32 out, adapted)" if args.lora else "+ SwiGLU"
+    workload_name = (args.config + (f"/{args.weights}" if args.weights != "nf4" else "")
+                     + (f"/lora-r{args.lora}" if args.lora else "")
+                     + ("/fwd+bwd" if args.backward else ""))
+    epi_name = "(fp32 out)" if (args.lora or args.backward) else "+ SwiGLU"
     workload_key = f"{workload_name}:T={T}"
     if prefill:
         achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
@@ -560,12 +598,10 @@ def main():
         peak = hbm
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak,
-                "traffic": recorded_traffic(
-                    "grouped_gemm_int4.cu" if args.weights == "int4" else "grouped_gemm_decode.cu",
-                    workload_key),
+                "traffic": recorded_traffic(DECODE_KERNEL_SOURCE[args.weights], workload_key),
                 "kernel": f"grouped {args.weights.upper()} gate_up GEMV {epi_name}",
                 "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*"
-                              f"{0.53125 if args.weights == 'int4' else 0.5625} + X + output)",
+                              f"{BYTES_PER_WEIGHT[args.weights]} + X + output)",
                 "peak_source": f"{peak_kind} HBM copy"}
 
     # ---- the same step as one CUDA graph (how a decode server replays it):
@@ -619,7 +655,7 @@ def main():
         X_d.copy_(X_h, non_blocking=True)
         L_d.copy_(L_h, non_blocking=True)
         for layer in range(layers):
-            if wl.int4 or wl.lora:  # the calls through the binding, on the copied inputs
+            if wl.fmt != "nf4" or wl.lora or wl.backward:  # the calls one by one
                 wl.layer(layer, args.algo, X=X_d, logits=L_d[layer])
             else:
                 moe.layer_forward(X_d, L_d[layer], shape.k, shape.renormalize,
@@ -642,9 +678,9 @@ def main():
            "d2h_bytes_per_step": Y_h.numel() * 4}
 
     cpu = None
-    if args.lora and not args.no_cpu_baseline:
-        cpu = {"skipped": "the oracle's layer has no adapters; the adapter delta's oracle "
-                          "is checked in the parity tests"}
+    if (args.lora or args.backward) and not args.no_cpu_baseline:
+        cpu = {"skipped": "the oracle's timed layer is the plain forward; the adapter and "
+                          "backward oracles are checked in the tests"}
     elif rank == 0 and world == 1 and not args.no_cpu_baseline:
         ncpu, aff, threads = cpu_cores()
         n_tok = min(T, 64) if not prefill else 16
@@ -664,9 +700,12 @@ def main():
         except ImportError:
             pass
 
-    # route_tile, permute_scatter, permute_rows, gate_up, down, combine; when
-    # adapted also two adapter launches and the standalone SwiGLU
-    launches_per_layer = 9 if args.lora else 6
+    # route_tile, permute_scatter, permute_rows, gate_up, down, combine; the
+    # standalone SwiGLU when adapted or with the backward; two adapter
+    # launches; the backward's combine backward, two transposed GEMMs, SwiGLU
+    # backward, scatter-add and routing backward
+    launches_per_layer = (6 + (1 if (args.lora or args.backward) else 0) + (2 if args.lora else 0)
+                          + (6 if args.backward else 0))
     lora = None
     if args.lora:
         lb = sum(wl.lora_bytes(x) for x in d) / len(d)

@@ -61,7 +61,8 @@ def test_clock_summary_without_samples():
 
 def _args(**kw):
     a = dict(gpus=1, steps=2, warmup=1, impl="reference", config="tiny", tokens=None,
-             layers=None, algo="auto", weights="nf4", lora=0, no_cpu_baseline=False, seed=0)
+             layers=None, algo="auto", weights="nf4", lora=0, backward=False,
+             no_cpu_baseline=False, seed=0)
     a.update(kw)
     return types.SimpleNamespace(**a)
 
@@ -88,14 +89,16 @@ def test_reference_arm_is_silent_on_other_ranks(capsys, monkeypatch):
     assert capsys.readouterr().out == ""
 
 
-@pytest.mark.parametrize("weights,lora", [("nf4", 0), ("int4", 0), ("nf4", 16)])
-def test_gate_up_bytes_accounting(weights, lora):
+@pytest.mark.parametrize("weights,lora,backward", [("nf4", 0, False), ("int4", 0, False),
+                                                   ("mxfp4", 0, False), ("nf4", 16, False),
+                                                   ("nf4", 0, True)])
+def test_gate_up_bytes_accounting(weights, lora, backward):
     # the per-launch algorithmic bytes, from the formats' per-weight sizes
     sh, T = bench.moe_synth.OLMOE, 64
     wl = object.__new__(bench.Workload)
-    wl.shape, wl.T, wl.int4, wl.lora = sh, T, weights == "int4", lora
-    per_w = 0.5 + (4 / 128 if weights == "int4" else 4 / 64)
-    out = T * sh.k * (2 * sh.I * 4 if lora else sh.I * 2)
+    wl.shape, wl.T, wl.fmt, wl.lora, wl.backward = sh, T, weights, lora, backward
+    per_w = 0.5 + {"nf4": 4 / 64, "int4": 4 / 128, "mxfp4": 1 / 32}[weights]
+    out = T * sh.k * (2 * sh.I * 4 if (lora or backward) else sh.I * 2)
     assert wl.gate_up_bytes(64) == pytest.approx(64 * 2 * sh.I * sh.H * per_w + T * sh.H * 2 + out)
     if lora:
         M = T * sh.k
