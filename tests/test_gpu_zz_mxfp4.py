@@ -1,9 +1,9 @@
 """GPU parity of the MXFP4 path (quantize bit-exact, decode GEMV within
 tolerance) against the CPU oracle (``oracle.mxfp4``).
 
-PENDING: the MXFP4 quantize and decode GEMV have been compiled but never run on a GPU, so this file
-is not collected (its name does not start with ``test_``).  After its first
-green run on a B200 it is renamed to ``test_gpu_*.py`` and joins the suite.
+The MXFP4 quantize and decode GEMV were first checked on a B200 through the C ABI alone
+(``tests/c_abi``); this file checks them through the Python binding.  The
+file name sorts after the forward-path GPU tests.
 """
 
 import numpy as np
