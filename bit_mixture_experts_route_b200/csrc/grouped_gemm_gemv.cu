@@ -7,7 +7,7 @@
 // bullet: one launch for all active experts, the 16-entry codebook decoded in
 // registers, no dequantized weight copy in memory.  At decode sizes the work
 // is streaming the NF4 bytes of every expert that received a token, so this
-// kernel is judged against HBM bandwidth.
+// kernel is measured against HBM bandwidth.
 //
 // Design (swap-AB): the weights are the M side of mma.sync.m16n8k16 (16
 // weight rows per warp), the routed tokens the N side (8 per MMA).  Per
