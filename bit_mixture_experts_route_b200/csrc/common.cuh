@@ -100,6 +100,32 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
 
+// True when storing v as OutT loses it: an fp16 store of a magnitude that
+// rounds past 65504 (>= 65520) or of a NaN.  fp32 and bf16 stores hold every
+// finite fp32 product of this library, so they never report.
+template <typename OutT>
+__device__ __forceinline__ bool overflows_out(float v) {
+  if constexpr (std::is_same<OutT, __half>::value) return !(fabsf(v) < 65520.0f);
+  else return false;
+}
+
+// out[i] = v rounded once to OutT; an fp16 overflow sets MOE_DEVERR_RANGE.
+template <typename OutT>
+__device__ __forceinline__ void store_checked(OutT* out, size_t i, float v, int32_t* dev_err) {
+  if (overflows_out<OutT>(v)) set_dev_err(dev_err, MOE_DEVERR_RANGE);
+  out[i] = from_f32<OutT>(v);
+}
+
+// Any of the eight fp16 values packed in a uint4 infinite or NaN.
+__device__ __forceinline__ bool any_f16x8_nonfinite(uint4 o) {
+  const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    bad |= ((w[i] & 0x7C00u) == 0x7C00u) || ((w[i] & 0x7C000000u) == 0x7C000000u);
+  return bad;
+}
+
 // silu(g) * u with silu(g) = g / (1 + exp(-g)), IEEE division.
 __device__ __forceinline__ float swiglu_f32(float g, float u) {
   return __fdiv_rn(g, 1.0f + expf(-g)) * u;

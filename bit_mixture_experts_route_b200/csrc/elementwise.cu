@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const InT* __restrict__ Yp
 
 // Xp[p, :] = X[sorted_rows[p] / k, :] converted to fp16, one warp per row,
 // 16-byte accesses.  Rows whose id is out of range are zero-filled and flagged.
+// A bf16 value beyond fp16's range becomes inf in Xp and sets
+// MOE_DEVERR_RANGE.
 template <typename InT>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict__ X, int T, int K,
                                                            const int32_t* __restrict__ rows, int k,
@@ -101,6 +103,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict
                                                            int32_t* dev_err) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  bool ovf = false;
   for (int p = warp; p < M_total; p += nwarps) {
     const int f = rows[p];
     const bool ok = f >= 0 && f < M_total && f / k < T;
@@ -115,12 +118,15 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict
         const uint4 u = *reinterpret_cast<const uint4*>(src + c);
         o = make_uint4(bf16x2_to_f16x2(u.x), bf16x2_to_f16x2(u.y), bf16x2_to_f16x2(u.z),
                        bf16x2_to_f16x2(u.w));
+        ovf |= any_f16x8_nonfinite(o);
       } else {
         o = *reinterpret_cast<const uint4*>(src + c);
       }
       *reinterpret_cast<uint4*>(dst + c) = o;
     }
   }
+  // every lane of the warp leaves the row loop together (warp-uniform p)
+  if (__any_sync(0xffffffffu, ovf) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
 }
 
 int sm_count() { return device_sm_count(); }

@@ -272,11 +272,11 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
       if (EPI == MOE_EPI_SWIGLU) {
         const int I = N / 2;
         const int col = it.rtile * (ROWS / 2) + 8 * warp + sg;
-        out[p * I + col] = from_f32<OutT>(swiglu_f32(acc[j][q], acc[j][q + 2]));
+        store_checked(out, p * I + col, swiglu_f32(acc[j][q], acc[j][q + 2]), dev_err);
       } else {
         const int col = it.rtile * ROWS + 16 * warp + sg;
-        out[p * N + col] = from_f32<OutT>(acc[j][q]);
-        out[p * N + col + 8] = from_f32<OutT>(acc[j][q + 2]);
+        store_checked(out, p * N + col, acc[j][q], dev_err);
+        store_checked(out, p * N + col + 8, acc[j][q + 2], dev_err);
       }
     }
   }

@@ -66,10 +66,7 @@ __device__ __forceinline__ void load_x16<__nv_bfloat16>(const __nv_bfloat16* __r
   xf[6] = bf16x2_to_f16x2(v.z); xf[7] = bf16x2_to_f16x2(v.w);
 }
 
-template <typename OutT>
-__device__ __forceinline__ void store_out(OutT* out, size_t idx, float v) {
-  out[idx] = from_f32<OutT>(v);
-}
+
 
 // Process one chunk of up to 8*NT8 tokens of expert e for this warp's rows.
 template <typename AT, int EPI, typename OutT, int NT8>
@@ -180,10 +177,11 @@ __device__ __forceinline__ void gemv_chunk(
       if (tok >= cnt) continue;
       const size_t p = (size_t)(p0 + tok);
       if (EPI == MOE_EPI_SWIGLU) {
-        store_out(out, p * (size_t)(N / 2) + outColA, swiglu_f32(acc[j][q], acc[j][q + 2]));
+        store_checked(out, p * (size_t)(N / 2) + outColA, swiglu_f32(acc[j][q], acc[j][q + 2]),
+                  dev_err);
       } else {
-        store_out(out, p * (size_t)N + outColA, acc[j][q]);
-        store_out(out, p * (size_t)N + outColB, acc[j][q + 2]);
+        store_checked(out, p * (size_t)N + outColA, acc[j][q], dev_err);
+        store_checked(out, p * (size_t)N + outColB, acc[j][q + 2], dev_err);
       }
     }
   }

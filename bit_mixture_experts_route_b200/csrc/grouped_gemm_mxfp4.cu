@@ -271,10 +271,10 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
       if (tok >= it.cnt) continue;
       const size_t p = (size_t)(it.start + tok);
       if (EPI == MOE_EPI_SWIGLU) {
-        out[p * (N / 2) + gA] = from_f32<OutT>(swiglu_f32(acc[j][q], acc[j][q + 2]));
+        store_checked(out, p * (N / 2) + gA, swiglu_f32(acc[j][q], acc[j][q + 2]), dev_err);
       } else {
-        out[p * N + gA] = from_f32<OutT>(acc[j][q]);
-        out[p * N + gB] = from_f32<OutT>(acc[j][q + 2]);
+        store_checked(out, p * N + gA, acc[j][q], dev_err);
+        store_checked(out, p * N + gB, acc[j][q + 2], dev_err);
       }
     }
   }

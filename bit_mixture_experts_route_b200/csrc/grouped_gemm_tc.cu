@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     const float* n_row = row_absmax(n_t);
     float a_cur = n_row ? __ldg(n_row + n_ks) : 0.0f;
     bool have = n_row != nullptr;
+    bool bad_scale = false;  // an absmax whose fp16 is subnormal or not finite
     for (int S = g; have; S += GROUPS) {
       const int slot = S % RING, rslot = S % RAW_RING;
       const uint32_t ph = (uint32_t)(S / RING) & 1u, rph = (uint32_t)(S / RAW_RING) & 1u;
@@ -484,6 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[rslot], rph, sm, dev_err))) break;
       const uint8_t* rp = sm.raw[rslot] + rrow * (BK / 2);
       const uint4 w0 = lds128(rp), w1 = lds128(rp + 16);
+      bad_scale |= a_cur != 0.0f && !(a_cur >= 6.103515625e-05f && a_cur <= 65504.0f);
       const __half2 ah = __float2half2_rn(a_cur);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.a_empty[slot], ph ^ 1, sm, dev_err))) break;
       tc_fence_after();
@@ -513,6 +515,8 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       a_cur = a_next;
       have = have_next;
     }
+    // the loop exits are warp-uniform, so every lane takes part
+    if (__any_sync(0xffffffffu, bad_scale) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
   } else {
     // ---------------- epilogue: warp (q, hc) reads TMEM lanes 32q .. 32q+31,
     // columns of half hc of each 64-column block (two warps per lane quarter)
@@ -526,6 +530,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     constexpr int ROWB = OUT_COLS * (int)sizeof(OutT);
     constexpr int V = ROWB / 16;  // 16-byte pieces per staged row
     bool ok = true;
+    bool ovf = false;  // an fp16 output that overflowed
     int lt = 0;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
       const TileInfo ti = tile_info(sm, E, n_tiles, t);
@@ -559,13 +564,18 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
             const float gt = up ? recv : lo, u = up ? hi : recv;
             // silu(g) * u with the fast exp and division intrinsics: their
             // relative error (~1e-6) is far below the fp16/bf16 output rounding
-            reinterpret_cast<OutT*>(stg + ((up ? 16 : 0) + i) * ROWB)[p] =
-                from_f32<OutT>(__fdividef(gt, 1.0f + __expf(-gt)) * u);
+            const float h = __fdividef(gt, 1.0f + __expf(-gt)) * u;
+            const int tok = (up ? 16 : 0) + i;
+            ovf |= c0 + tok < ti.nrows && overflows_out<OutT>(h);
+            reinterpret_cast<OutT*>(stg + tok * ROWB)[p] = from_f32<OutT>(h);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            reinterpret_cast<OutT*>(stg + i * ROWB)[lane] = from_f32<OutT>(__uint_as_float(v[i]));
+          for (int i = 0; i < 32; ++i) {
+            const float y = __uint_as_float(v[i]);
+            ovf |= c0 + i < ti.nrows && overflows_out<OutT>(y);
+            reinterpret_cast<OutT*>(stg + i * ROWB)[lane] = from_f32<OutT>(y);
+          }
         }
         __syncwarp();
         // staged rows -> global, 16 bytes per lane
@@ -585,6 +595,8 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         mbar_arrive(&sm.acc_empty);
       }
     }
+    // the loop exits are warp-uniform, so every lane takes part
+    if (__any_sync(0xffffffffu, ovf) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
   }
 
   // single-lane roles (producers, MMA issuer) rejoin their warp before the

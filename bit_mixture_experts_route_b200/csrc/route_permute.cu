@@ -410,25 +410,59 @@ namespace {
 
 __device__ __align__(256) unsigned char g_route_scratch[MOE_ROUTE_NOALLOC_SCRATCH_BYTES];
 
-// The array's device address on each device, looked up once per device.  In
-// host code `g_route_scratch` only names a host-side stand-in, so the kernel
-// must be given the address that cudaGetSymbolAddress reports.
+// The array's device address in each CUDA context, looked up once per
+// context.  A __device__ variable has one address per context (normally a
+// device's primary context, but a caller may make another context current),
+// so the cache is keyed by the context that is current when the call runs.
+// In host code `g_route_scratch` only names a host-side stand-in, so the
+// kernel must be given the address that cudaGetSymbolAddress reports.
 std::mutex g_scratch_mu;
-void* g_scratch_addr[64] = {};
+constexpr int kMaxContexts = 64;
+CUcontext g_scratch_ctx[kMaxContexts] = {};
+void* g_scratch_addr[kMaxContexts] = {};
+int g_scratch_n = 0;
 
-cudaError_t scratch_for_current_device(void** out) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+// cuCtxGetCurrent from the driver, looked up once through the runtime (the
+// library has no link-time dependency on libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
     void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_route_scratch);  // current device = dev
-    if (err != cudaSuccess) return err;
-    g_scratch_addr[dev] = p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+cudaError_t scratch_for_current_context(void** out) {
+  const CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (!get_ctx) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (ctx) {
+    for (int i = 0; i < g_scratch_n; ++i)
+      if (g_scratch_ctx[i] == ctx) {
+        *out = g_scratch_addr[i];
+        return cudaSuccess;
+      }
   }
-  *out = g_scratch_addr[dev];
+  // First call in this context (or no context yet: the runtime then makes
+  // the current device's primary context current while it looks the symbol
+  // up).
+  void* p = nullptr;
+  cudaError_t err = cudaGetSymbolAddress(&p, g_route_scratch);
+  if (err != cudaSuccess) return err;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorInitializationError;
+  if (g_scratch_n < kMaxContexts) {
+    g_scratch_ctx[g_scratch_n] = ctx;
+    g_scratch_addr[g_scratch_n] = p;
+    ++g_scratch_n;
+  }
+  *out = p;
   return cudaSuccess;
 }
 
@@ -442,7 +476,7 @@ cudaError_t route_permute_noalloc(const float* logits, int T, int E, int k, int 
                                   int32_t* topk_idx, float* topk_w, int32_t* offsets,
                                   int32_t* sorted_rows, int32_t* inv_perm, cudaStream_t s) {
   void* ws = nullptr;
-  cudaError_t err = scratch_for_current_device(&ws);
+  cudaError_t err = scratch_for_current_context(&ws);
   if (err != cudaSuccess) return err;
   // Nothing in the scratch has to start at zero: the routing kernel writes
   // every rank and every tile count before the scatter kernel reads them, so

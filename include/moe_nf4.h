@@ -20,8 +20,12 @@
  * Conventions shared by every call
  * --------------------------------
  * - All pointers are DEVICE pointers unless a parameter says otherwise; the
- *   caller allocates and owns every buffer (inputs, outputs, workspace).  The
- *   library keeps no mutable global state between calls.
+ *   caller allocates and owns every buffer (inputs, outputs, workspace); the
+ *   library allocates no device memory.  It does keep process-wide state of
+ *   two kinds: (1) host-side caches -- encoded TMA tensor maps, keyed by
+ *   every argument that determines them, and per-device attributes -- which
+ *   never change a result; (2) the fixed scratch array of
+ *   moe_route_permute_noalloc (see there).
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream).  Every call only enqueues work: it is asynchronous and
  *   stream-ordered, and never synchronizes the device.
@@ -85,8 +89,15 @@ typedef enum {
 #define MOE_DEVERR_TIMEOUT 0x8     /* a bounded wait inside a kernel expired */
 #define MOE_DEVERR_LAYOUT 0x10     /* a kernel's shared-memory layout did not
                                       fit this device; the call did no work */
-#define MOE_DEVERR_RANGE 0x20      /* an MXFP4 scale lies outside the range
-                                      the decode GEMV multiplies exactly */
+#define MOE_DEVERR_RANGE 0x20      /* a value outside the range of the 16-bit
+                                      type it passes through: an fp16
+                                      activation, intermediate or output
+                                      that overflowed; an NF4 absmax that is
+                                      subnormal or too large in fp16 (tensor-
+                                      core GEMM); an MXFP4 scale outside the
+                                      range the decode GEMV multiplies
+                                      exactly.  The work is done; the
+                                      affected values carry the error */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_string(moe_status_t status);
@@ -368,8 +379,9 @@ moe_status_t moe_route_permute(const float* logits, int T, int E, int k,
  * - Size limit: moe_route_permute_workspace_size(T, E, k) must not exceed
  *   MOE_ROUTE_NOALLOC_SCRATCH_BYTES (T*k up to about 200,000 routed rows at
  *   E = 128); larger problems return MOE_ERR_WORKSPACE and enqueue nothing.
- * - Set-up: the first call on each device looks up the array's device
- *   address (cudaGetSymbolAddress) with that device current; make that first
+ * - Set-up: the first call in each CUDA context (normally a device's
+ *   primary context) looks up the array's device address there
+ *   (cudaGetSymbolAddress) and caches it for that context; make that first
  *   call before any stream capture on the device.
  * - Sharing: all calls on a device use the same array, which keeps the last
  *   call's contents (nothing in it needs to start at zero).  Calls whose
@@ -415,7 +427,12 @@ moe_status_t moe_route_permute_noalloc(const float* logits, int T, int E, int k,
  * TC kernel (tcgen05): weights enter as fp16(fp16(level) * fp16(absmax));
  * it needs gather == NULL and F16 A (rows already permuted, e.g. by
  * moe_permute_rows), N % 128 == 0, absmax < 65504.  AUTO uses it when those
- * hold and M_total >= 36 * E.
+ * hold and M_total >= 36 * E.  A call WITH `gather` therefore never reaches
+ * the tensor cores: it always runs the general GEMV kernel (MOE_ALGO_TC then
+ * returns MOE_ERR_UNSUPPORTED); prefill-sized callers permute first.
+ * An absmax that is not 0 and lies outside [2^-14, 65504) -- where
+ * fp16(absmax) is subnormal or not finite -- sets MOE_DEVERR_RANGE in the
+ * TC kernel (the result then carries fp16 underflow error).
  * All pointers 16-byte aligned.
  */
 moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype,
@@ -445,15 +462,22 @@ moe_status_t moe_permute_rows(const void* X, moe_dtype_t x_dtype, int T, int K,
 /*
  * moe_swiglu -- standalone h[m, i] = silu(gu[m, i]) * gu[m, I + i],
  * silu(g) = g / (1 + exp(-g)), for gu [M, 2I] (F32, BF16 or F16) into
- * h [M, I] of h_dtype.  The fused path never calls this; it exists for
- * callers that keep gate_up outputs.  I % 4 == 0, pointers 16-byte aligned.
+ * h [M, I] of h_dtype.  (The pages name the experts' matmuls but not their
+ * activation; the SiLU(gate) * up step between the two grouped projections
+ * is fixed by the problem statement this library implements.)  The fused
+ * path never calls this -- the gate_up GEMM applies it in its epilogue; it
+ * exists for callers that keep gate_up outputs (e.g. to add a LoRA term
+ * first).  I % 4 == 0, pointers 16-byte aligned.
  */
 moe_status_t moe_swiglu(const void* gu, moe_dtype_t gu_dtype, int M, int I,
                         void* h, moe_dtype_t h_dtype, void* stream);
 
 /*
  * moe_unpermute_combine -- Y[t, :] = sum_{j<k} topk_w[t, j] *
- * Yp[inv_perm[t*k + j], :], summed in j order in fp32.
+ * Yp[inv_perm[t*k + j], :], summed in j order in fp32.  (The pages print no
+ * formula for it; the routing-weighted scatter-combine that closes the layer
+ * is fixed by the problem statement this library implements, and it is the
+ * inverse of the permutation of moe_route_permute.)
  *   Yp [T*k, H] of yp_dtype (F32, BF16, F16), Y [T, H] of y_dtype.
  *   1 <= k <= 32, H % 4 == 0, pointers 16-byte aligned.
  */

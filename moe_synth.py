@@ -14,7 +14,8 @@ Workload shapes (the mixture-of-experts models the pages discuss):
   intermediate 768; decode batches 1..64 and a 4096-token prefill, with
   Zipf-skewed routing (s = 1.1).
 * Qwen3-235B-A22B-shaped: E=128, top-8 renormalised, hidden 4096,
-  intermediate 1536, weights N(0, 0.015) with 0.1 % outliers at 8 sigma.
+  intermediate 1536, weights N(0, 0.015) with 0.1 % outliers at 8 sigma;
+  uniform (N(0,1) logits) and Zipf-skewed routing.
 
 Weights are fp32 N(0, sigma); activations bf16 N(0, 1); logits fp32.
 """
@@ -58,8 +59,11 @@ QWEN3_30B = MoEShape("qwen3-30b-a3b", E=128, k=8, H=2048, I=768,
                      renormalize=True, routing="zipf")
 QWEN3_235B = MoEShape("qwen3-235b-a22b", E=128, k=8, H=4096, I=1536,
                       renormalize=True, sigma=0.015, outlier_frac=1e-3)
+# The same layer with Zipf-skewed routing (same weights for the same seed:
+# the weights depend only on E, H, I, sigma and the outliers).
+QWEN3_235B_ZIPF = dataclasses.replace(QWEN3_235B, name="qwen3-235b-a22b-zipf", routing="zipf")
 
-SHAPES = {s.name: s for s in (TINY, OLMOE, QWEN3_30B, QWEN3_235B)}
+SHAPES = {s.name: s for s in (TINY, OLMOE, QWEN3_30B, QWEN3_235B, QWEN3_235B_ZIPF)}
 
 
 def _gen(seed: int, device) -> torch.Generator:

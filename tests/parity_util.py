@@ -26,6 +26,18 @@ def errors(y, ref):
     return rel, mae / rms
 
 
+def assert_close_16bit(y, ref, dtype, what=""):
+    """A 16-bit output against the oracle, both ways.  The survey's reading
+    counts the output's own rounding as error, so ``y`` must meet the bar
+    against the unrounded oracle value; it must also meet it against that
+    value rounded once to ``dtype``, which isolates the kernel's arithmetic
+    from the final rounding."""
+    r1 = assert_close(y, ref, f"{what} (unrounded oracle)")
+    ref_rounded = torch.from_numpy(np.asarray(ref, dtype=np.float64)).to(dtype).double().numpy()
+    r2 = assert_close(y, ref_rounded, f"{what} (oracle rounded to {dtype})")
+    return r1, r2
+
+
 def assert_close(y, ref, what=""):
     y = np.asarray(y, dtype=np.float64)
     assert np.all(np.isfinite(y)), f"{what}: non-finite GPU output"
@@ -44,7 +56,9 @@ def gpu_stack(shape, seed, device="cuda"):
     Returns ``((packed_gu, absmax_gu, packed_d, absmax_d), (w_gu, w_d))`` with
     the fp32 weights kept on the device for the oracle to copy per expert."""
     import bit_mixture_experts_route_b200 as moe
-    key = (shape, seed)
+    # the weights depend on these fields only, so shapes that differ in their
+    # routing alone (uniform / Zipf) share one stack and its oracle experts
+    key = (shape.E, shape.H, shape.I, shape.sigma, shape.outlier_frac, seed)
     if key not in _STACKS:
         _STACKS.clear()
         w_gu = moe_synth.weights(shape, "gate_up", seed, device=device)

@@ -12,20 +12,24 @@ import bench
 
 
 def test_recorded_traffic_only_for_the_recorded_source(tmp_path, monkeypatch):
-    got = bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=64")
-    assert got is not None and got > 1e8
-    assert bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=7") is None
-    assert bench.recorded_traffic("no_such_kernel.cu", "olmoe-decode:T=64") is None
-    # a changed kernel source (different sha256) has no recorded traffic
+    # a table written for one kernel source: its value is used only while the
+    # source keeps the recorded sha256, and only for the recorded workload
+    import hashlib
     root = tmp_path
     (root / "profiles").mkdir()
-    (root / "bit_mixture_experts_route_b200" / "csrc").mkdir(parents=True)
-    shutil.copy(os.path.join(bench.ROOT, "profiles", "kernel_traffic.txt"), root / "profiles")
-    src = os.path.join(bench.ROOT, "bit_mixture_experts_route_b200", "csrc",
-                       "grouped_gemm_decode.cu")
-    dst = root / "bit_mixture_experts_route_b200" / "csrc" / "grouped_gemm_decode.cu"
-    dst.write_bytes(open(src, "rb").read() + b"\n// edited\n")
+    csrc = root / "bit_mixture_experts_route_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    src = csrc / "grouped_gemm_decode.cu"
+    src.write_bytes(b"// kernel source\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    (root / "profiles" / "kernel_traffic.txt").write_text(
+        "# kernel_source  sha256  workload  bytes_per_launch\n"
+        f"grouped_gemm_decode.cu {sha} olmoe-decode:T=64 157830656\n")
     monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=64") == 157830656
+    assert bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=7") is None
+    assert bench.recorded_traffic("no_such_kernel.cu", "olmoe-decode:T=64") is None
+    src.write_bytes(b"// kernel source\n// edited\n")
     assert bench.recorded_traffic("grouped_gemm_decode.cu", "olmoe-decode:T=64") is None
 
 

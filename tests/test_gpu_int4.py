@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import assert_close
+from parity_util import assert_close, assert_close_16bit
 
 pytestmark = pytest.mark.gpu
 
@@ -86,9 +86,7 @@ def test_int4_grouped_gemm_output_dtypes(out_dtype):
     torch.cuda.synchronize()
     p_ref, m_ref = oracle.quantize_int4_grouped(W.numpy())
     ref = oracle.grouped_gemm_int4(X.float().numpy(), p_ref, m_ref, off)
-    # the output's own rounding is part of the reference
-    ref_r = torch.from_numpy(ref).to(out_dtype).float().numpy()
-    assert_close(out.float().cpu().numpy(), ref_r, f"int4 out {out_dtype}")
+    assert_close_16bit(out.double().cpu().numpy(), ref, out_dtype, f"int4 out {out_dtype}")
 
 
 def test_int4_grouped_gemm_flags_bad_offsets():

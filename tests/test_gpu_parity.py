@@ -12,7 +12,8 @@ import torch
 
 import moe_synth
 import oracle
-from parity_util import LazyOracleStack, assert_close, gpu_stack, run_layer_steps
+from parity_util import (LazyOracleStack, assert_close, assert_close_16bit, gpu_stack,
+                         run_layer_steps)
 
 pytestmark = pytest.mark.gpu
 
@@ -196,10 +197,10 @@ def test_grouped_gemm_output_dtypes(out_dtype):
                                out_dtype=out_dtype)
     pr, ar = oracle.quantize_blockwise(W.numpy())
     ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
-    # A 16-bit output carries its own rounding (bf16: up to 2^-9 relative),
-    # so it is compared with the oracle's value rounded once to that type.
-    ref_rounded = torch.from_numpy(ref).to(out_dtype).double().numpy()
-    assert_close(_np(out.float()), ref_rounded, str(out_dtype))
+    # A 16-bit output carries its own rounding (bf16: up to 2^-9 relative).
+    # It must meet the bar against the unrounded oracle (that rounding counted
+    # as error) and against the oracle rounded once to the output type.
+    assert_close_16bit(_np(out.double()), ref, out_dtype, str(out_dtype))
     assert out.dtype == out_dtype
 
 
@@ -255,20 +256,35 @@ def test_combine():
 # ----------------------------------------------------------------- whole layer
 
 def _layer_parity(shape, T, seed, tokens=None, algo="auto", via_layer_call=False):
+    """The layer on seeded inputs against the oracle on ``tokens`` (all by
+    default).  ``via_layer_call=False`` runs the exported calls one by one with
+    the gate_up GEMM gathering its rows (``sorted_rows``): that always takes the
+    general GEMV kernel.  ``via_layer_call=True`` runs ``moe_layer_forward``,
+    which permutes the rows first and lets the AUTO rule pick the decode GEMV
+    or, from 36 routed rows per expert on average, the tensor-core kernel."""
     stack_gpu, weights = gpu_stack(shape, seed)
     stack = LazyOracleStack.shared(stack_gpu, weights)
     X = moe_synth.activations(T, shape.H, seed)
     lg = moe_synth.logits(shape, T, seed)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
     if via_layer_call:
-        Y = moe.layer_forward(X.cuda(), lg.cuda(), shape.k, shape.renormalize, *stack_gpu)
+        Y = moe.layer_forward(X.cuda(), lg.cuda(), shape.k, shape.renormalize, *stack_gpu,
+                              dev_err=err)
     else:
         Y, *_ = run_layer_steps(X.cuda(), lg.cuda(), shape.k, shape.renormalize, stack_gpu,
                                 algo=algo)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
     toks = list(range(T)) if tokens is None else tokens
     ref = oracle.moe_layer(X.float().numpy(), lg.numpy(), stack, shape.k, shape.renormalize,
                            tokens=toks)
     assert stack.checked > 0
     return assert_close(_np(Y)[toks], ref, f"{shape.name} T={T}")
+
+
+def _sample(T, n, seed):
+    rng = np.random.default_rng(seed)
+    return sorted(rng.choice(T, size=min(n, T), replace=False).tolist())
 
 
 def test_layer_tiny_all_tokens():
@@ -284,37 +300,67 @@ def test_layer_olmoe_decode(T):
     _layer_parity(moe_synth.OLMOE, T, 0)
 
 
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
+def test_layer_olmoe_decode_single_call(T):
+    # the bench's layer: permuted rows, decode GEMV (TMA + warp MMA)
+    _layer_parity(moe_synth.OLMOE, T, 0, via_layer_call=True)
+
+
 def test_layer_olmoe_decode_last_layer():
     # layer 15 of the 16-layer decode stack (its own weights and logits)
     _layer_parity(moe_synth.OLMOE, 16, 15)
 
 
-def test_layer_qwen3_30b_decode():
+# Qwen3-30B-A3B-shaped decode, Zipf routing: the token sweep 1..64, all tokens
+@pytest.mark.parametrize("T", [1, 2, 4, 8, 16, 32, 64])
+def test_layer_qwen3_30b_decode_sweep(T):
+    _layer_parity(moe_synth.QWEN3_30B, T, 1, via_layer_call=True)
+
+
+def test_layer_qwen3_30b_decode_gather_path():
     _layer_parity(moe_synth.QWEN3_30B, 64, 1)
 
 
 def test_layer_qwen3_30b_decode_last_layer():
     # layer 47 of the 48-layer decode stack
-    _layer_parity(moe_synth.QWEN3_30B, 8, 47)
+    _layer_parity(moe_synth.QWEN3_30B, 8, 47, via_layer_call=True)
 
 
-def test_layer_qwen3_30b_prefill_sampled():
-    # 256 seeded tokens of 4096 (Zipf routing: 0 to ~1500 rows per expert,
-    # empty experts included; the grouped GEMMs run on the tensor cores)
-    rng = np.random.default_rng(0)
-    toks = sorted(rng.choice(4096, size=256, replace=False).tolist())
-    _layer_parity(moe_synth.QWEN3_30B, 4096, 2, tokens=toks)
+def test_layer_qwen3_30b_prefill_gather_path_sampled():
+    # 4096 tokens, Zipf routing (0 to ~1500 rows per expert, empty experts
+    # included), through the gathering calls: both grouped GEMMs run on the
+    # general GEMV kernel.  The tensor-core form of this layer is checked in
+    # test_gpu_tc.py.
+    _layer_parity(moe_synth.QWEN3_30B, 4096, 2, tokens=_sample(4096, 128, 0))
 
 
-def test_layer_qwen3_235b_decode():
-    # hidden 4096, moe_intermediate 1536, 0.1 % of the weights at 8 sigma
-    _layer_parity(moe_synth.QWEN3_235B, 1, 3)
+# Qwen3-235B-A22B-shaped layer: hidden 4096, moe_intermediate 1536, weights
+# N(0, 0.015) with 0.1 % at 8 sigma.  Every case uses the weights of seed 3,
+# so the oracle quantizes and checks each expert once for all of them.
+_S235 = 3
 
 
-def test_layer_qwen3_235b_prefill_sampled():
-    rng = np.random.default_rng(1)
-    toks = sorted(rng.choice(2048, size=4, replace=False).tolist())
-    _layer_parity(moe_synth.QWEN3_235B, 2048, 5, tokens=toks)
+@pytest.mark.parametrize("T", [1, 8, 32])
+def test_layer_qwen3_235b_decode(T):
+    _layer_parity(moe_synth.QWEN3_235B, T, _S235, via_layer_call=True)
+
+
+@pytest.mark.parametrize("T", [8, 32])
+def test_layer_qwen3_235b_decode_zipf(T):
+    _layer_parity(moe_synth.QWEN3_235B_ZIPF, T, _S235, via_layer_call=True)
+
+
+def test_layer_qwen3_235b_decode_gather_path():
+    _layer_parity(moe_synth.QWEN3_235B, 8, _S235)
+
+
+@pytest.mark.parametrize("shape", [moe_synth.QWEN3_235B, moe_synth.QWEN3_235B_ZIPF],
+                         ids=["uniform", "zipf"])
+def test_layer_qwen3_235b_prefill_tc_sampled(shape):
+    # 2048 tokens (16384 routed rows, 128 per expert on average): the one-call
+    # layer runs both grouped GEMMs on the tensor-core kernel; 128 seeded
+    # tokens are checked against the oracle
+    _layer_parity(shape, 2048, _S235, tokens=_sample(2048, 128, 1), via_layer_call=True)
 
 
 def test_layer_single_expert_dense():
@@ -330,3 +376,94 @@ def test_layer_deterministic():
     y1 = moe.layer_forward(X, lg, shape.k, shape.renormalize, *stack_gpu)
     y2 = moe.layer_forward(X, lg, shape.k, shape.renormalize, *stack_gpu)
     assert torch.equal(y1, y2)
+
+
+# ----------------------------------------------------------------- range guards
+
+def _range_case(sigma_w, x_scale, epi, seed):
+    E, K = 3, 256
+    N = 512 if epi == "swiglu" else 256
+    counts = np.array([5, 0, 40])
+    off = _ragged_offsets(E, counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(seed)
+    W = torch.randn((E, N, K), generator=g) * sigma_w
+    X = (torch.randn((M, K), generator=g) * x_scale).to(torch.float16)
+    p, a = moe.nf4_quantize(W.cuda())
+    pr, ar = oracle.quantize_blockwise(W.numpy())
+    ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
+    if epi == "swiglu":
+        ref = oracle.swiglu(ref)
+    return X.cuda(), p, a, torch.from_numpy(off).cuda(), M, ref
+
+
+@pytest.mark.parametrize("algo", ["gemv", "tc"])
+def test_range_tiny_weights(algo):
+    # Weights ~N(0, 1e-5): every absmax lies below fp16's smallest normal
+    # (2^-14).  The GEMV kernels apply the fp32 absmax to fp32 partial sums and
+    # stay exact; the tensor-core kernel feeds fp16(level * absmax) and must
+    # say so with MOE_DEVERR_RANGE.
+    X, p, a, off, M, ref = _range_case(1e-5, 1.0, "none", 21)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.nf4_grouped_gemm(X, p, a, off, M, out_dtype=torch.float32, algo=algo, dev_err=err)
+    torch.cuda.synchronize()
+    if algo == "gemv":
+        assert int(err.item()) == 0
+        assert_close(_np(out), ref, "gemv, weights 1e-5")
+    else:
+        assert int(err.item()) == moe.DEVERR_RANGE
+
+
+@pytest.mark.parametrize("algo", ["gemv", "tc"])
+def test_range_large_activations(algo):
+    # Activations x 1e3 (fp16 holds them): fp32 and fp16 outputs in range meet
+    # the bar with no flag on both kernels.
+    X, p, a, off, M, ref = _range_case(0.02, 1e3, "none", 22)
+    assert float(np.max(np.abs(ref))) < 6e4
+    for dt in (torch.float32, torch.float16):
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = moe.nf4_grouped_gemm(X, p, a, off, M, out_dtype=dt, algo=algo, dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        if dt == torch.float32:
+            assert_close(_np(out), ref, f"{algo}, x 1e3")
+        else:
+            assert_close_16bit(_np(out.double()), ref, dt, f"{algo}, x 1e3")
+
+
+@pytest.mark.parametrize("algo", ["gemv", "tc"])
+def test_range_fp16_output_overflow_flagged(algo):
+    # x 1e3 activations through gate_up + SwiGLU: h = silu(g) * u reaches
+    # ~1e5, beyond fp16.  An fp32 output is exact and unflagged; an fp16
+    # output overflows and sets MOE_DEVERR_RANGE.
+    X, p, a, off, M, ref = _range_case(0.05, 1e3, "swiglu", 23)
+    assert float(np.max(np.abs(ref))) > 7e4
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.nf4_grouped_gemm(X, p, a, off, M, epilogue="swiglu", out_dtype=torch.float32,
+                               algo=algo, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert_close(_np(out), ref, f"{algo} swiglu fp32, x 1e3")
+    out16 = moe.nf4_grouped_gemm(X, p, a, off, M, epilogue="swiglu", out_dtype=torch.float16,
+                                 algo=algo, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == moe.DEVERR_RANGE
+    assert torch.isinf(out16).any()
+
+
+def test_range_permute_rows_overflow_flagged():
+    # bf16 activations beyond fp16's range become inf in the fp16 rows the
+    # grouped GEMMs read, and the call says so.
+    T, K, k = 9, 256, 2
+    X = torch.randn((T, K)).to(torch.bfloat16)
+    X[4, 17] = 1e5
+    rows = torch.arange(T * k, dtype=torch.int32)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Xp = moe.permute_rows(X.cuda(), rows.cuda(), k, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == moe.DEVERR_RANGE
+    assert torch.isinf(Xp[8, 17]) and torch.isinf(Xp[9, 17])
+    err.zero_()
+    moe.permute_rows((X * 0.5).clamp(-100, 100).cuda(), rows.cuda(), k, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0

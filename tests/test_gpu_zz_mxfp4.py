@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import assert_close
+from parity_util import assert_close, assert_close_16bit
 
 pytestmark = pytest.mark.gpu
 
@@ -90,8 +90,7 @@ def test_mxfp4_grouped_gemm_output_dtypes(out_dtype):
     torch.cuda.synchronize()
     p_ref, s_ref = oracle.quantize_mxfp4(W.numpy())
     ref = oracle.grouped_gemm_mxfp4(X.float().numpy(), p_ref, s_ref, off)
-    ref = torch.from_numpy(ref).to(out_dtype).double().numpy()
-    assert_close(out.double().cpu().numpy(), ref, f"mxfp4 out {out_dtype}")
+    assert_close_16bit(out.double().cpu().numpy(), ref, out_dtype, f"mxfp4 out {out_dtype}")
 
 
 def test_mxfp4_scale_out_of_exact_range_is_flagged():

@@ -44,9 +44,12 @@ def _noalloc(logits, k, renorm):
 def test_noalloc_routing_matches_workspace_routing_twice():
     import bit_mixture_experts_route_b200 as moe
     g = torch.Generator().manual_seed(123)
-    # A large call first, then a small one that runs on the scratch contents
-    # the large call left behind.
-    cases = [(4096, 128, 8, True), (37, 64, 6, False)]
+    # A large call first (32768 routed rows), then a smaller one (4800 rows)
+    # that also takes the two-launch path through the scratch, so it runs on
+    # the ranks and tile counts the large call left behind.  Both sizes lie
+    # above the 4096 routed rows that the one-launch path (which needs no
+    # scratch) handles.
+    cases = [(4096, 128, 8, True), (600, 64, 8, False)]
     for T, E, k, renorm in cases:
         logits = torch.randn((T, E), generator=g).cuda()
         ref = moe.route_permute(logits, k, renorm)
