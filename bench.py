@@ -6,9 +6,14 @@ GEMM with fused SwiGLU, grouped down GEMM, combine -- over one token batch,
 through a stack of independent MoE layers whose NF4 weights together exceed
 the 126 MB L2 (every layer's weights stream from HBM once per step).
 
-Default workload: OLMoE-shaped decode (E=64, top-8, hidden 2048, expert
-intermediate 1024, plain softmax weights), T=64 tokens, 16 layers
-(3.6 GB of NF4 weights).  ``--config`` selects the other shapes.
+Headline workload (the N = 1 line's ``value``): the largest single-GPU shape,
+a Qwen3-235B-A22B-shaped layer (E=128, top-8, hidden 4096, expert
+intermediate 1536, 1.36 GB of NF4) at a 2048-token prefill, where both grouped
+GEMMs run on the tensor cores.  Every other configuration of the workload list
+-- Tiny, OLMoE decode T = 1/4/16/64, Qwen3-30B-A3B decode (48 layers) and
+prefill, Qwen3-235B decode T = 1/8/32 and the Zipf-routed prefill -- is timed
+in the same run and reported under ``workloads``, each with its own roofline
+and CPU-oracle baseline.  ``--config`` / ``--tokens`` time one workload alone.
 
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 instead (bounded samples of the same workload).
@@ -40,8 +45,20 @@ CONFIGS = {
     "qwen3-30b-prefill": (moe_synth.QWEN3_30B, 4096, 2),
     "qwen3-235b-decode": (moe_synth.QWEN3_235B, 32, 8),
     "qwen3-235b-prefill": (moe_synth.QWEN3_235B, 2048, 1),
-    "tiny": (moe_synth.TINY, 16, 1),
+    "qwen3-235b-prefill-zipf": (moe_synth.QWEN3_235B_ZIPF, 2048, 1),
+    "tiny": (moe_synth.TINY, 16, 128),
 }
+HEADLINE = "qwen3-235b-prefill"
+# The rest of the workload list, timed after the headline: (config, T).
+SWEEP = [("tiny", 16),
+         ("olmoe-decode", 1), ("olmoe-decode", 4), ("olmoe-decode", 16), ("olmoe-decode", 64),
+         ("qwen3-30b-decode", 1), ("qwen3-30b-decode", 8), ("qwen3-30b-decode", 64),
+         ("qwen3-30b-prefill", 4096),
+         ("qwen3-235b-decode", 1), ("qwen3-235b-decode", 8), ("qwen3-235b-decode", 32),
+         ("qwen3-235b-prefill-zipf", 2048)]
+SWEEP_STEPS = 20          # timed steps per sweep workload (at most --steps)
+# Nominal B200 figures, for the second fraction each roofline carries.
+NOMINAL_HBM_GBS, NOMINAL_BF16_TFLOPS = 8000.0, 2250.0
 
 
 def parse_args():
@@ -50,7 +67,9 @@ def parse_args():
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--config", choices=sorted(CONFIGS), default="olmoe-decode")
+    p.add_argument("--config", choices=sorted(CONFIGS), default=HEADLINE)
+    p.add_argument("--no-sweep", action="store_true",
+                   help="time the headline (or --config) workload only")
     p.add_argument("--tokens", type=int, default=None, help="token batch T")
     p.add_argument("--layers", type=int, default=None)
     p.add_argument("--algo", choices=["auto", "gemv", "tc"], default="auto")
@@ -226,11 +245,14 @@ DECODE_KERNEL_SOURCE = {"nf4": "grouped_gemm_decode.cu", "int4": "grouped_gemm_i
                         "mxfp4": "grouped_gemm_mxfp4.cu"}
 
 class Workload:
+    """One configuration's NF4 (or INT4, MXFP4) layer stacks on the device,
+    and the token-batch buffers of the current ``T`` (``set_tokens``)."""
+
     def __init__(self, shape, T, layers, seed, device="cuda", weights="nf4", lora=0,
                  backward=False):
         import bit_mixture_experts_route_b200 as moe
         self.moe = moe
-        self.shape, self.T, self.L = shape, T, layers
+        self.shape, self.L, self.seed, self.dev = shape, layers, seed, device
         self.fmt = weights
         self.lora = lora
         self.backward = backward
@@ -247,12 +269,24 @@ class Workload:
             del w
             self.stacks.append((p_gu, a_gu, p_d, a_d))
         torch.cuda.empty_cache()
-        self.X = moe_synth.activations(T, shape.H, seed, device=device)
-        self.logits = torch.stack([moe_synth.logits(shape, T, seed * 1000 + layer, device=device)
-                                   for layer in range(layers)])
+        if lora:
+            self.adapters = [moe_synth.lora_adapters(shape, "gate_up", lora, seed * 1000 + layer,
+                                                     device=device)
+                             + moe_synth.lora_adapters(shape, "down", lora, seed * 1000 + layer,
+                                                       device=device)
+                             for layer in range(layers)]
+        self.set_tokens(T)
+
+    def set_tokens(self, T):
+        """Inputs and intermediates of a T-token batch (``shape`` may differ
+        from the weights' in its routing only)."""
+        moe, shape, seed, dev = self.moe, self.shape, self.seed, self.dev
+        self.T = T
+        self.X = moe_synth.activations(T, shape.H, seed, device=dev)
+        self.logits = torch.stack([moe_synth.logits(shape, T, seed * 1000 + layer, device=dev)
+                                   for layer in range(self.L)])
         k, E, H, I = shape.k, shape.E, shape.H, shape.I
         M = T * k
-        dev = device
         self.route = {
             "topk_idx": torch.empty((T, k), dtype=torch.int32, device=dev),
             "topk_w": torch.empty((T, k), dtype=torch.float32, device=dev),
@@ -268,23 +302,17 @@ class Workload:
         self.Y = torch.empty((T, H), dtype=torch.float32, device=dev)
         self.lws = torch.empty((max(moe.layer_workspace_size(T, E, k, H, I), 256),),
                                dtype=torch.uint8, device=dev)
-        if lora or backward:
+        if self.lora or self.backward:
             # both GEMMs write fp32 pre-activations (the adapters add their
             # term in place; the backward needs gate_up's), SwiGLU standalone
             self.GU = torch.empty((M, 2 * I), dtype=torch.float32, device=dev)
             self.Yp32 = torch.empty((M, H), dtype=torch.float32, device=dev)
-        if backward:
+        if self.backward:
             g = torch.Generator(device=dev)
             g.manual_seed(seed * 1000 + 999)
             self.dY = torch.randn((T, H), generator=g, device=dev, dtype=torch.float32)
             self.ones = torch.ones((T, k), dtype=torch.float32, device=dev)
             self.dX = torch.empty((T, H), dtype=torch.float32, device=dev)
-        if lora:
-            self.adapters = [moe_synth.lora_adapters(shape, "gate_up", lora, seed * 1000 + layer,
-                                                     device=dev)
-                             + moe_synth.lora_adapters(shape, "down", lora, seed * 1000 + layer,
-                                                       device=dev)
-                             for layer in range(layers)]
 
     def layer(self, layer, algo="auto", ev=None, X=None, logits=None):
         moe, sh, T = self.moe, self.shape, self.T
@@ -309,7 +337,8 @@ class Workload:
         if self.fmt == "int4":
             self.moe.int4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out)
         elif self.fmt == "mxfp4":
-            self.moe.mxfp4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out)
+            self.moe.mxfp4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out,
+                                        algo=algo)
         else:
             self.moe.nf4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out,
                                       algo=algo)
@@ -356,7 +385,17 @@ class Workload:
         return (d * self.lora * (sh.H + 2 * sh.I) * 2 + M * sh.H * 2
                 + 2 * M * 2 * sh.I * 4)
 
-    def step(self, algo="auto", evs=None):
+    def step(self, algo="auto", evs=None, fused=False):
+        """One pass through every layer.  ``fused``: each layer is the one C
+        call ``moe_layer_forward`` (its GEMMs in chain mode: each starts
+        streaming its weights while the kernel before it finishes); else the
+        exported calls one by one, with CUDA events around gate_up."""
+        if fused and self.fmt == "nf4" and not (self.lora or self.backward) and algo == "auto":
+            sh = self.shape
+            for layer in range(self.L):
+                self.moe.layer_forward(self.X, self.logits[layer], sh.k, sh.renormalize,
+                                       *self.stacks[layer], workspace=self.lws, out=self.Y)
+            return
         for layer in range(self.L):
             self.layer(layer, algo, None if evs is None else evs[layer])
 
@@ -517,6 +556,193 @@ def run_reference(args, shape, T, layers):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- one workload
+
+def graphed_replay(wl, algo, steps, warmup, world, local):
+    """The layer steps captured as one CUDA graph and replayed ``steps``
+    times (how a decode server issues a step): same kernels and work as the
+    eager launches, no per-launch host cost.  Returns (timing dict or error,
+    clock summary)."""
+    stream = torch.cuda.current_stream()
+    g = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            wl.step(algo, fused=True)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            wl.step(algo, fused=True)
+        for _ in range(max(3, warmup)):
+            g.replay()
+        torch.cuda.synchronize()
+        captured = 1.0
+    except Exception as exc:  # noqa: BLE001
+        err = {"error": str(exc)[:200]}
+        captured = 0.0
+    # every rank takes the same collective steps: time only if all captured
+    if -max_over_ranks(-captured, world) <= 0:
+        del g
+        return (err if captured == 0.0 else {"error": "another rank failed to capture"}), None
+    gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.mark_start()
+        gs.record()
+        for _ in range(steps):
+            g.replay()
+        ge.record()
+        torch.cuda.synchronize()
+        clk.mark_end()
+        barrier(world)
+    gms = max_over_ranks(gs.elapsed_time(ge), world)
+    del g
+    return {"ms_per_step": gms / steps, "elapsed_ms": gms}, clk.summary()
+
+
+def run_workload(wl, name, args, steps, world, local, hbm, tf_burst, tf_sust, peak_kind):
+    """Time one workload: K eager steps with CUDA events around every gate_up
+    launch (the dominant kernel), then the same steps as one CUDA graph.
+    Returns the workload's entry (value = graphed layer-tokens/s)."""
+    shape, T, layers = wl.shape, wl.T, wl.L
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        wl.step(args.algo)
+    torch.cuda.synchronize()
+
+    n_ev = 4 if (args.lora or args.backward) else 2
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+            for _ in range(layers)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.mark_start()
+        start.record(stream)
+        for s in range(steps):
+            wl.step(args.algo, evs[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+        clk.mark_end()
+        barrier(world)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
+    tokens_per_step = T * layers          # layer-tokens: T tokens through each layer
+    eager_value = world * tokens_per_step * steps / (elapsed_ms / 1e3)
+    gu_ms = [e[0].elapsed_time(e[1]) for st in evs for e in st]
+    gu_avg_ms = sum(gu_ms) / len(gu_ms)
+    lora_ms = [e[2].elapsed_time(e[3]) for st in evs for e in st] if args.lora else []
+
+    d = wl.distinct_experts()
+    d_avg = sum(d) / len(d)
+    gu_bytes = sum(wl.gate_up_bytes(x) for x in d) / len(d)
+    gu_flops = wl.gate_up_flops()
+    # the tensor-core kernel serves the GEMMs from 36 routed rows per expert
+    # on average (the AUTO dispatch rule); below that the decode GEMV does
+    prefill = T * shape.k >= 36 * shape.E and args.algo != "gemv"
+    epi_name = "(fp32 out)" if (args.lora or args.backward) else "+ SwiGLU"
+    workload_key = f"{name}:T={T}"
+    if prefill:
+        achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
+                "frac": achieved / tf_burst,
+                "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
+                "traffic": recorded_traffic("grouped_gemm_tc.cu", workload_key),
+                "kernel": f"grouped {args.weights.upper()} gate_up GEMM {epi_name} (tcgen05)",
+                "per_launch": f"{gu_flops:.4g} FLOP (2*T*k*H*2I, real routed rows)",
+                "us_per_launch": 1e3 * gu_avg_ms,
+                "peak_source": f"{peak_kind} bf16 dense (burst); nominal "
+                               f"{NOMINAL_BF16_TFLOPS:.0f} for frac_of_nominal"}
+    else:
+        achieved = gu_bytes / (gu_avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                "traffic": recorded_traffic(DECODE_KERNEL_SOURCE[args.weights], workload_key),
+                "kernel": f"grouped {args.weights.upper()} gate_up GEMV {epi_name}",
+                "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*"
+                              f"{BYTES_PER_WEIGHT[args.weights]} + X + output)",
+                "us_per_launch": 1e3 * gu_avg_ms,
+                "peak_source": f"{peak_kind} HBM copy; nominal {NOMINAL_HBM_GBS:.0f} for "
+                               "frac_of_nominal"}
+
+    graphed, gclk = graphed_replay(wl, args.algo, steps, args.warmup, world, local)
+    entry = {"workload": name, "T": T, "layers": layers}
+    if "ms_per_step" in graphed:
+        entry["value"] = world * tokens_per_step * steps / (graphed["elapsed_ms"] / 1e3)
+        entry["ms_per_step"] = graphed["ms_per_step"]
+        entry["clocks"] = gclk
+        entry["timing"] = "graphed"
+    else:
+        entry["value"] = eager_value
+        entry["ms_per_step"] = elapsed_ms / steps
+        entry["clocks"] = clk.summary()
+        entry["timing"] = f"eager (graph capture failed: {graphed.get('error')})"
+    entry["unit"] = "layer-tokens/s"
+    entry["eager"] = {"value": eager_value, "ms_per_step": elapsed_ms / steps,
+                      "clocks": clk.summary()}
+    entry["roofline"] = roof
+    entry["distinct_experts_per_layer"] = d_avg
+    layer_ms = entry["ms_per_step"] / layers
+    if not prefill:
+        # the whole layer against the decode bytes it must move
+        lb = sum(wl.layer_bytes(x) for x in d) / len(d)
+        entry["layer_hbm"] = {"bytes_per_layer": lb, "us_per_layer": 1e3 * layer_ms,
+                              "achieved_GBs": lb / (layer_ms / 1e3) / 1e9,
+                              "frac": lb / (layer_ms / 1e3) / 1e9 / hbm}
+    else:
+        lf = 3 * gu_flops / 2
+        entry["layer_tensor"] = {"flops_per_layer": lf, "us_per_layer": 1e3 * layer_ms,
+                                 "achieved_TFLOPs": lf / (layer_ms / 1e3) / 1e12,
+                                 "frac": lf / (layer_ms / 1e3) / 1e12 / tf_burst}
+    entry["tokens_per_s_through_all_layers"] = world * T / (layer_ms * layers / 1e3)
+    entry["gate_up_ms_avg"] = gu_avg_ms
+    if args.lora:
+        lb = sum(wl.lora_bytes(x) for x in d) / len(d)
+        l_avg = sum(lora_ms) / len(lora_ms)
+        lach = lb / (l_avg / 1e3) / 1e9
+        entry["lora"] = {"rank": args.lora, "kernel": "gate_up LoRA delta (in place on fp32)",
+                         "timing": "CUDA events around each eager launch; at decode sizes the "
+                                   "window can include the wait for the host to submit it",
+                         "us_per_launch": 1e3 * l_avg, "bytes_per_launch": lb,
+                         "per_launch": f"distinct experts {d_avg:.1f} x r*(H+2I)*2 + X + 2 x "
+                                       "fp32 out",
+                         "achieved_GBs": lach, "frac_of_hbm": lach / hbm,
+                         "flops_per_launch": 2.0 * T * shape.k * args.lora
+                                             * (shape.H + 2 * shape.I)}
+    return entry
+
+
+def cpu_baseline_for(shape, T, name, args, cache):
+    """The oracle on the host cores on a bounded sample of this workload's
+    tokens (rank 0 at N = 1 only); one sample per shape serves every batch
+    size of that shape, since the oracle's cost per token does not depend on
+    the batch."""
+    key = (shape.name, args.weights)
+    if key in cache:
+        out = dict(cache[key])
+        out["sample"] = out["sample"] + f" (measured on {out['measured_on']}, reused)"
+        return out
+    ncpu, aff, threads = cpu_cores()
+    n_tok = min(T, 16 if shape.H <= 256 else 4 if shape.H <= 2048 else 2)
+    n, dt = oracle_sample(shape, T, args.seed, n_tok, weights=args.weights)
+    cpu = {"value": n / dt, "unit": "layer-tokens/s", "cores": threads, "kind": "oracle",
+           "blas_threads": threads, "measured_on": f"{name}:T={T}",
+           "sample": f"{n} tokens of layer 0 (their experts dequantized, per-token fp64 "
+                     f"expert MLPs); host cpu_count={ncpu}, affinity={aff}; {dt:.2f} s"}
+    try:  # the same oracle on one thread
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            n1, dt1 = oracle_sample(shape, T, args.seed, max(1, n_tok // 2), weights=args.weights)
+        cpu["value_1thread"] = n1 / dt1
+        cpu["sample"] += f"; 1-thread run: {n1} tokens in {dt1:.2f} s"
+    except ImportError:
+        pass
+    cache[key] = cpu
+    return dict(cpu)
+
+
 # ----------------------------------------------------------------- main
 
 def main():
@@ -532,118 +758,20 @@ def main():
     world, rank, local = dist_setup()
     import bit_mixture_experts_route_b200 as moe
     moe.load()
-    if args.weights != "nf4" and T * shape.k >= 36 * shape.E:
-        raise SystemExit(f"{args.weights} weights have the decode GEMV path only (fewer than 36 "
-                         "routed rows per expert)")
+    if args.weights == "int4" and T * shape.k >= 36 * shape.E:
+        raise SystemExit("int4 weights have the decode GEMV path only (fewer than 36 routed rows "
+                         "per expert)")
     if args.backward and args.weights != "nf4":
         raise SystemExit("--backward runs on NF4 weights (the transposed GEMM is NF4)")
-    wl = Workload(shape, T, layers, rank_seed(args.seed, rank), weights=args.weights,
-                  lora=args.lora, backward=args.backward)
     hbm, tf_burst, tf_sust, peak_kind = load_peaks()
-    stream = torch.cuda.current_stream()
-
-    # ---- warm-up
-    for _ in range(max(args.warmup, 3)):
-        wl.step(args.algo)
-    torch.cuda.synchronize()
-
-    # ---- timed region: K steps, events around every gate_up launch (and the
-    # gate_up adapter launch when adapted)
-    n_ev = 4 if (args.lora or args.backward) else 2
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-            for _ in range(layers)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        clk.mark_start()
-        start.record(stream)
-        for s in range(args.steps):
-            wl.step(args.algo, evs[s])
-        end.record(stream)
-        torch.cuda.synchronize()
-        clk.mark_end()
-        barrier(world)
-    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
-    ms_per_step = elapsed_ms / args.steps
-    tokens_per_step = T * layers          # layer-tokens: T tokens through each layer
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
-    gu_ms = [e[0].elapsed_time(e[1]) for st in evs for e in st]
-    gu_avg_ms = sum(gu_ms) / len(gu_ms)
-    lora_ms = [e[2].elapsed_time(e[3]) for st in evs for e in st] if args.lora else []
-
-    d = wl.distinct_experts()
-    d_avg = sum(d) / len(d)
-    gu_bytes = sum(wl.gate_up_bytes(x) for x in d) / len(d)
-    gu_flops = wl.gate_up_flops()
-    # the tensor-core kernel serves the GEMMs from 36 routed rows per expert
-    # on average (the AUTO dispatch rule); below that the decode GEMV does
-    prefill = T * shape.k >= 36 * shape.E
+    seed = rank_seed(args.seed, rank)
+    wl = Workload(shape, T, layers, seed, weights=args.weights, lora=args.lora,
+                  backward=args.backward)
     workload_name = (args.config + (f"/{args.weights}" if args.weights != "nf4" else "")
                      + (f"/lora-r{args.lora}" if args.lora else "")
                      + ("/fwd+bwd" if args.backward else ""))
-    epi_name = "(fp32 out)" if (args.lora or args.backward) else "+ SwiGLU"
-    workload_key = f"{workload_name}:T={T}"
-    if prefill:
-        achieved = gu_flops / (gu_avg_ms / 1e3) / 1e12
-        peak = tf_burst
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                "traffic": recorded_traffic("grouped_gemm_tc.cu", workload_key),
-                "kernel": f"grouped NF4 gate_up GEMM {epi_name}",
-                "per_launch": f"{gu_flops:.4g} FLOP (2*T*k*H*2I)",
-                "peak_source": f"{peak_kind} bf16 dense"}
-    else:
-        achieved = gu_bytes / (gu_avg_ms / 1e3) / 1e9
-        peak = hbm
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak,
-                "traffic": recorded_traffic(DECODE_KERNEL_SOURCE[args.weights], workload_key),
-                "kernel": f"grouped {args.weights.upper()} gate_up GEMV {epi_name}",
-                "per_launch": f"{gu_bytes:.4g} B (distinct experts {d_avg:.1f} x 2I*H*"
-                              f"{BYTES_PER_WEIGHT[args.weights]} + X + output)",
-                "peak_source": f"{peak_kind} HBM copy"}
-
-    # ---- the same step as one CUDA graph (how a decode server replays it):
-    # same kernels, same work, no per-launch host cost
-    graphed = None
-    gclk = None
-    g = None
-    try:
-        g = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            wl.step(args.algo)
-        stream.wait_stream(side)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g):
-            wl.step(args.algo)
-        for _ in range(max(3, args.warmup)):
-            g.replay()
-        torch.cuda.synchronize()
-        captured = 1.0
-    except Exception as exc:  # noqa: BLE001
-        graphed = {"error": str(exc)[:200]}
-        captured = 0.0
-    # every rank takes the same collective steps: time only if all captured
-    if -max_over_ranks(-captured, world) > 0:
-        gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(local) as gclk:
-            barrier(world)
-            torch.cuda.synchronize()
-            gclk.mark_start()
-            gs.record()
-            for _ in range(args.steps):
-                g.replay()
-            ge.record()
-            torch.cuda.synchronize()
-            gclk.mark_end()
-            barrier(world)
-        gms = max_over_ranks(gs.elapsed_time(ge), world)
-        graphed = {"value": world * tokens_per_step * args.steps / (gms / 1e3),
-                   "ms_per_step": gms / args.steps}
-    del g
+    head = run_workload(wl, workload_name, args, args.steps, world, local, hbm, tf_burst,
+                        tf_sust, peak_kind)
 
     # ---- end to end through the one-call C API with host buffers
     X_h = wl.X.cpu().pin_memory()
@@ -673,32 +801,48 @@ def main():
     ee.record()
     torch.cuda.synchronize()
     ems = max_over_ranks(es.elapsed_time(ee), world)
-    e2e = {"value": world * tokens_per_step * args.steps / (ems / 1e3), "unit": "tokens/s",
+    e2e = {"value": world * T * layers * args.steps / (ems / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": X_h.numel() * 2 + L_h.numel() * 4,
-           "d2h_bytes_per_step": Y_h.numel() * 4}
+           "d2h_bytes_per_step": Y_h.numel() * 4,
+           "path": "moe_layer_forward per layer (C ABI), pinned host X and logits in, Y out"}
+    del wl
+    torch.cuda.empty_cache()
 
+    baselines = {}
     cpu = None
+    do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
     if (args.lora or args.backward) and not args.no_cpu_baseline:
         cpu = {"skipped": "the oracle's timed layer is the plain forward; the adapter and "
                           "backward oracles are checked in the tests"}
-    elif rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ncpu, aff, threads = cpu_cores()
-        n_tok = min(T, 64) if not prefill else 16
-        n, dt = oracle_sample(shape, T, args.seed, n_tok, weights=args.weights)
-        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "blas_threads": threads,
-               "sample": f"{n} tokens of layer 0 of this workload (NF4 experts dequantized, "
-                         f"per-token fp64 expert MLPs); host cpu_count={ncpu}, "
-                         f"affinity={aff}; {dt:.1f} s"}
-        try:  # the same oracle on one thread, on a quarter of the tokens
-            from threadpoolctl import threadpool_limits
-            with threadpool_limits(limits=1):
-                n1, dt1 = oracle_sample(shape, T, args.seed, max(2, n_tok // 4),
-                                        weights=args.weights)
-            cpu["value_1thread"] = n1 / dt1
-            cpu["sample"] += f"; 1-thread run: {n1} tokens in {dt1:.1f} s"
-        except ImportError:
-            pass
+    elif do_cpu:
+        cpu = cpu_baseline_for(shape, T, workload_name, args, baselines)
+
+    # ---- the rest of the workload list (same collective steps on every rank)
+    workloads = []
+    plain = args.weights == "nf4" and not args.lora and not args.backward
+    if plain and not args.no_sweep and args.config == HEADLINE and args.tokens is None \
+            and args.layers is None:
+        sweep_steps = min(args.steps, SWEEP_STEPS)
+        current = None
+        for cfg, t in SWEEP:
+            sh, _, nl = CONFIGS[cfg]
+            if current is None or current[0] != cfg:
+                current = None
+                torch.cuda.empty_cache()
+                current = (cfg, Workload(sh, t, nl, seed))
+            w = current[1]
+            w.set_tokens(t)
+            entry = run_workload(w, cfg, args, sweep_steps, world, local, hbm, tf_burst,
+                                 tf_sust, peak_kind)
+            if do_cpu:
+                entry["cpu_baseline"] = cpu_baseline_for(sh, t, cfg, args, baselines)
+            entry["config"] = {"E": sh.E, "k": sh.k, "hidden": sh.H, "intermediate": sh.I,
+                               "renormalize": sh.renormalize, "routing": sh.routing,
+                               "l2": f"{nl} layers x {sh.E * sh.nf4_bytes_per_expert / 1e6:.1f}"
+                                     " MB NF4 weights"}
+            workloads.append(entry)
+        current = None
+        torch.cuda.empty_cache()
 
     # route_tile, permute_scatter, permute_rows, gate_up, down, combine; the
     # standalone SwiGLU when adapted or with the backward; two adapter
@@ -706,50 +850,39 @@ def main():
     # backward, scatter-add and routing backward
     launches_per_layer = (6 + (1 if (args.lora or args.backward) else 0) + (2 if args.lora else 0)
                           + (6 if args.backward else 0))
-    lora = None
-    if args.lora:
-        lb = sum(wl.lora_bytes(x) for x in d) / len(d)
-        l_avg = sum(lora_ms) / len(lora_ms)
-        lach = lb / (l_avg / 1e3) / 1e9
-        lora = {"rank": args.lora, "kernel": "gate_up LoRA delta (in place on fp32)",
-                "timing": "CUDA events around each eager launch; at decode sizes the window "
-                          "can include the wait for the host to submit the launch",
-                "us_per_launch": 1e3 * l_avg, "bytes_per_launch": lb,
-                "per_launch": f"distinct experts {d_avg:.1f} x r*(H+2I)*2 + X + 2 x fp32 out",
-                "achieved_GBs": lach, "frac_of_hbm": lach / hbm,
-                "flops_per_launch": 2.0 * T * shape.k * args.lora * (shape.H + 2 * shape.I)}
-    eager = {"value": value, "ms_per_step": ms_per_step, "clocks": clk.summary(),
-             "launch": "one host launch per kernel, CUDA events per gate_up launch"}
-    clocks = clk.summary()
-    if graphed is not None and "value" in graphed:
-        value, ms_per_step = graphed["value"], graphed["ms_per_step"]
-        clocks = gclk.summary()
     line = {
-        "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic",
+        "metric": "MoE layer tokens/s", "value": head["value"], "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": workload_name, "T": T, "layers": layers, "E": shape.E,
                    "k": shape.k, "hidden": shape.H, "intermediate": shape.I,
-                   "weights": args.weights, "renormalize": shape.renormalize, "routing": shape.routing,
+                   "weights": args.weights, "renormalize": shape.renormalize,
+                   "routing": shape.routing,
                    "value_counts": "layer-tokens: T tokens through each of the layers",
                    "l2": f"inputs larger than L2: {layers} layers x "
                          f"{shape.E * shape.nf4_bytes_per_expert / 1e6:.0f} MB NF4 weights",
-                   "distinct_experts_per_layer": d_avg, "algo": args.algo,
+                   "distinct_experts_per_layer": head["distinct_experts_per_layer"],
+                   "algo": args.algo,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": roof,
-        "timing": "value = the layer steps replayed as one CUDA graph; eager = the same "
-                  "launches one by one from the host",
-        "graphed": graphed,
-        "eager": eager,
+        "roofline": head["roofline"],
+        "timing": "value = the layer steps replayed as one CUDA graph of moe_layer_forward "
+                  "calls (the library's chained launches); eager = the exported calls one by "
+                  "one from the host, CUDA events around each gate_up launch",
+        "graphed": {"value": head["value"], "ms_per_step": head["ms_per_step"]}
+        if head["timing"] == "graphed" else {"error": head["timing"]},
+        "eager": head["eager"],
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": launches_per_layer * layers * args.steps,
-        "clocks": clocks,
-        "gate_up_ms_avg": gu_avg_ms,
+        "clocks": head["clocks"],
+        "gate_up_ms_avg": head["gate_up_ms_avg"],
     }
-    if lora is not None:
-        line["lora"] = lora
+    for key in ("layer_hbm", "layer_tensor", "lora"):
+        if key in head:
+            line[key] = head[key]
+    if workloads:
+        line["workloads"] = workloads
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

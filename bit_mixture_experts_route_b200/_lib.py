@@ -43,7 +43,8 @@ SIGNATURES = {
     "moe_int4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
     "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
     "moe_mxfp4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
-    "moe_mxfp4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_mxfp4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P,
+                                    _S]),
     "moe_nf4_grouped_gemm_t": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _S]),
     "moe_swiglu_backward": (_I, [_P, _P, _I, _I, _I, _P, _I, _S]),
     "moe_combine_backward": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _P, _S]),
@@ -283,9 +284,10 @@ def mxfp4_quantize(W, packed=None, scales=None, dev_err=None):
 
 
 def mxfp4_grouped_gemm(A, packed, scales, expert_offsets, M_total, epilogue="none",
-                       out_dtype=torch.float32, out=None, dev_err=None):
-    """Decode-shaped grouped GEMM on MXFP4 weights, all experts in one launch
-    (see the header); ``A`` fp16 rows in permuted order."""
+                       out_dtype=torch.float32, algo="auto", out=None, dev_err=None):
+    """Grouped GEMM on MXFP4 weights, all experts in one launch (decode GEMV
+    or tensor-core kernel, see the header); ``A`` fp16 rows in permuted
+    order."""
     _need(A, torch.float16, "A", 2)
     _need(packed, torch.uint8, "packed", 3)
     _need(scales, torch.uint8, "scales", 3)
@@ -301,7 +303,7 @@ def mxfp4_grouped_gemm(A, packed, scales, expert_offsets, M_total, epilogue="non
     _room(out, M_total * n_out, "out", _F)
     _check(load().moe_mxfp4_grouped_gemm(
         _ptr(A), A.shape[0], _ptr(packed), _ptr(scales), _ptr(expert_offsets), E, N, K, M_total,
-        EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
+        EPI[epilogue], _ptr(out), DT[out.dtype], ALGO[algo], _ptr(dev_err), _stream(A.device)),
         "moe_mxfp4_grouped_gemm")
     return out
 

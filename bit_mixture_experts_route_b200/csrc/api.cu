@@ -113,12 +113,21 @@ moe_status_t moe_mxfp4_quantize(const float* W, int E, int N, int K, uint8_t* pa
 moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
                                     const uint8_t* scales, const int32_t* expert_offsets, int E,
                                     int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
-                                    moe_dtype_t out_dtype, int32_t* dev_err, void* stream) {
+                                    moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
+                                    void* stream) {
   if (E < 1 || E > 1024 || N < 1 || K < 1 || M_total < 0 || A_rows < M_total)
     return MOE_ERR_INVALID_ARG;
   if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (!valid_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
-  if (!moe_launch::grouped_gemm_mxfp4_supported(N, K)) return MOE_ERR_UNSUPPORTED;
+  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC)
+    return MOE_ERR_INVALID_ARG;
+  const bool gemv_ok = moe_launch::grouped_gemm_mxfp4_supported(N, K);
+  const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue);
+  bool use_tc;
+  if (algo == MOE_ALGO_TC) use_tc = true;
+  else if (algo == MOE_ALGO_GEMV) use_tc = false;
+  else use_tc = tc_ok && ((int64_t)M_total >= 36LL * E || !gemv_ok);  // the NF4 rule
+  if (use_tc ? !tc_ok : !gemv_ok) return MOE_ERR_UNSUPPORTED;
   if (!expert_offsets || !packed || !scales) return MOE_ERR_INVALID_ARG;
   if (M_total > 0 && (!A || !out)) return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {A, packed, scales, expert_offsets, out};
@@ -126,6 +135,10 @@ moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* pa
     if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
   if (moe_status_t st = check_device()) return st;
   if (M_total == 0) return MOE_OK;
+  if (use_tc)
+    return from_cuda(moe_launch::grouped_gemm_tc_mxfp4(A, A_rows, packed, scales, expert_offsets,
+                                                       E, N, K, M_total, epilogue, out,
+                                                       out_dtype, dev_err, (cudaStream_t)stream));
   return from_cuda(moe_launch::grouped_gemm_mxfp4(A, A_rows, packed, scales, expert_offsets, E, N,
                                                   K, M_total, epilogue, out, out_dtype, dev_err,
                                                   (cudaStream_t)stream));
@@ -267,12 +280,19 @@ moe_status_t moe_route_permute_noalloc(const float* logits, int T, int E, int k,
                                                      (cudaStream_t)stream));
 }
 
-moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows,
-                                  const int32_t* gather, int k, const uint8_t* packed, const float* absmax,
-                                  const int32_t* expert_offsets, int E, int N, int K,
-                                  int M_total, moe_epilogue_t epilogue, void* out,
-                                  moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
-                                  void* stream) {
+}  // extern "C"
+
+namespace {
+
+// moe_nf4_grouped_gemm; chain = true only from moe_layer_forward, where the
+// expert offsets were written two or more kernels before this one (see
+// moe_launch::grouped_gemm_gemv).
+moe_status_t nf4_grouped_gemm_impl(const void* A, moe_dtype_t a_dtype, int A_rows,
+                                   const int32_t* gather, int k, const uint8_t* packed,
+                                   const float* absmax, const int32_t* expert_offsets, int E,
+                                   int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
+                                   moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
+                                   void* stream, bool chain) {
   if (a_dtype != MOE_DT_BF16 && a_dtype != MOE_DT_F16) return MOE_ERR_INVALID_ARG;
   if (!valid_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
   if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
@@ -308,10 +328,25 @@ moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows
   if (use_tc)
     return from_cuda(moe_launch::grouped_gemm_tc(A, a_dtype, A_rows, gather, k, packed, absmax,
                                                  expert_offsets, E, N, K, M_total, epilogue,
-                                                 out, out_dtype, dev_err, s));
+                                                 out, out_dtype, dev_err, s, chain));
   return from_cuda(moe_launch::grouped_gemm_gemv(A, a_dtype, A_rows, gather, k, packed, absmax,
                                                  expert_offsets, E, N, K, M_total, epilogue,
-                                                 out, out_dtype, dev_err, s));
+                                                 out, out_dtype, dev_err, s, chain));
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype, int A_rows,
+                                  const int32_t* gather, int k, const uint8_t* packed,
+                                  const float* absmax, const int32_t* expert_offsets, int E,
+                                  int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
+                                  moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
+                                  void* stream) {
+  return nf4_grouped_gemm_impl(A, a_dtype, A_rows, gather, k, packed, absmax, expert_offsets, E,
+                               N, K, M_total, epilogue, out, out_dtype, algo, dev_err, stream,
+                               false);
 }
 
 moe_status_t moe_permute_rows(const void* X, moe_dtype_t x_dtype, int T, int K,
@@ -409,12 +444,16 @@ moe_status_t moe_layer_forward(const void* X, const float* logits, int T, int E,
   void* xp = ws + off[8];
   st = moe_permute_rows(X, MOE_DT_BF16, T, H, sorted_rows, k, M, xp, dev_err, stream);
   if (st) return st;
-  st = moe_nf4_grouped_gemm(xp, MOE_DT_F16, M, nullptr, 1, packed_gu, absmax_gu, offsets, E,
-                            2 * I, H, M, MOE_EPI_SWIGLU, hbuf, MOE_DT_F16, MOE_ALGO_AUTO,
-                            dev_err, stream);
+  // The GEMMs run in chain mode: the offsets come from the routing two and
+  // three kernels back, so each GEMM starts streaming its weights while the
+  // kernel before it finishes.
+  st = nf4_grouped_gemm_impl(xp, MOE_DT_F16, M, nullptr, 1, packed_gu, absmax_gu, offsets, E,
+                             2 * I, H, M, MOE_EPI_SWIGLU, hbuf, MOE_DT_F16, MOE_ALGO_AUTO,
+                             dev_err, stream, true);
   if (st) return st;
-  st = moe_nf4_grouped_gemm(hbuf, MOE_DT_F16, M, nullptr, 1, packed_d, absmax_d, offsets, E, H, I,
-                            M, MOE_EPI_NONE, yp, MOE_DT_F16, MOE_ALGO_AUTO, dev_err, stream);
+  st = nf4_grouped_gemm_impl(hbuf, MOE_DT_F16, M, nullptr, 1, packed_d, absmax_d, offsets, E, H,
+                             I, M, MOE_EPI_NONE, yp, MOE_DT_F16, MOE_ALGO_AUTO, dev_err, stream,
+                             true);
   if (st) return st;
   return moe_unpermute_combine(yp, MOE_DT_F16, inv_perm, topk_w, T, k, H, Y, MOE_DT_F32, stream);
 }

@@ -14,6 +14,7 @@
 #include <string>
 #include <type_traits>
 #include <unordered_map>
+#include <utility>
 
 #include "../../include/moe_nf4.h"
 
@@ -126,9 +127,64 @@ __device__ __forceinline__ bool any_f16x8_nonfinite(uint4 o) {
   return bad;
 }
 
+// MXFP4 (OCP Microscaling v1.0) decoding shared by the MXFP4 GEMV and the
+// tensor-core GEMM.
+// fp16 bits of an E2M1 code's value: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6,
+// bit 3 the sign.
+__device__ __forceinline__ uint32_t e2m1_h(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const uint32_t mag = m == 0 ? 0u : m == 1 ? 0x3800u : m == 2 ? 0x3C00u : m == 3 ? 0x3E00u
+                     : m == 4 ? 0x4000u : m == 5 ? 0x4200u : m == 6 ? 0x4400u : 0x4600u;
+  return mag | ((c & 8u) << 12);
+}
+
+// E8M0 byte -> {2^(b-127), 2^(b-127)} as fp16 bits, exact for b in [103, 142]
+// (fp16 subnormals from 2^-24); 0 below.  `bad` is set when b is not 0 and
+// the scaled E2M1 values would not all be exact in fp16 (b outside
+// [104, 140]).
+__device__ __forceinline__ uint32_t mx_scale_h2(uint32_t b, bool& bad) {
+  bad |= (b != 0u) && (b < 104u || b > 140u);
+  uint32_t h = 0;
+  if (b >= 113u && b <= 142u) h = (b - 112u) << 10;   // normal: exponent field b - 127 + 15
+  else if (b >= 103u && b < 113u) h = 1u << (b - 103u);  // subnormal: 2^-24 * 2^(b - 103)
+  return h * 0x00010001u;
+}
+
+// Weight formats of the tensor-core GEMM.
+enum WeightFormat { kFmtNF4 = 0, kFmtMXFP4 = 1 };
+
 // silu(g) * u with silu(g) = g / (1 + exp(-g)), IEEE division.
 __device__ __forceinline__ float swiglu_f32(float g, float u) {
   return __fdiv_rn(g, 1.0f + expf(-g)) * u;
+}
+
+// Programmatic dependent launch.  Every kernel of the layer is launched with
+// programmatic stream serialization (launch_pdl below), so it may start
+// while the kernel before it on the stream is still running.  Such a kernel
+// calls pdl_wait() before it touches any memory the earlier kernel may read
+// or write (pdl_wait returns once that kernel has completed and its writes
+// are visible), and pdl_trigger() only after its own pdl_wait(), so at most
+// two kernels of a stream ever overlap.  Launched without the attribute,
+// pdl_wait() returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
@@ -256,26 +312,38 @@ cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
                           int32_t* topk_idx, float* topk_w, int32_t* offsets,
                           int32_t* sorted_rows, int32_t* inv_perm, void* ws,
                           cudaStream_t s);
+// The grouped NF4 GEMMs.  chain = true only inside the library's own layer
+// sequence (route -> permute_rows -> gate_up -> down), where expert_offsets
+// were written at least two kernels earlier: the GEMM then reads them, and
+// starts streaming weights, before the kernel right before it (which writes
+// A) has finished.  chain = false waits for that kernel before any access.
 cudaError_t grouped_gemm_gemv(const void* A, moe_dtype_t a_dt, int A_rows,
                               const int32_t* gather, int k,
                               const uint8_t* packed, const float* absmax,
                               const int32_t* offsets, int E, int N, int K,
                               int M_total, moe_epilogue_t epi, void* out,
                               moe_dtype_t out_dt, int32_t* dev_err,
-                              cudaStream_t s);
+                              cudaStream_t s, bool chain = false);
 bool grouped_gemm_decode_supported(int N, int K);
 cudaError_t grouped_gemm_decode(const void* A, int A_rows, const uint8_t* packed,
                                 const float* absmax, const int32_t* offsets, int E, int N,
                                 int K, int M_total, moe_epilogue_t epi, void* out,
-                                moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);
+                                moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s,
+                                bool chain = false);
 cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows,
                             const int32_t* gather, int k,
                             const uint8_t* packed, const float* absmax,
                             const int32_t* offsets, int E, int N, int K,
                             int M_total, moe_epilogue_t epi, void* out,
                             moe_dtype_t out_dt, int32_t* dev_err,
-                            cudaStream_t s);
+                            cudaStream_t s, bool chain = false);
 bool grouped_gemm_tc_supported(int N, int K, moe_epilogue_t epi);
+// The same tensor-core kernel on MXFP4 weights (scales uint8 [E, N, K/32]);
+// A fp16 rows in permuted order.
+cudaError_t grouped_gemm_tc_mxfp4(const void* A, int A_rows, const uint8_t* packed,
+                                  const uint8_t* scales, const int32_t* offsets, int E, int N,
+                                  int K, int M_total, moe_epilogue_t epi, void* out,
+                                  moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);
 cudaError_t int4_quantize(const float* W, int64_t rows, int K, uint8_t* packed, uint32_t* meta,
                           int32_t* dev_err, cudaStream_t s);
 bool grouped_gemm_int4_supported(int N, int K);

@@ -44,6 +44,8 @@ __device__ __forceinline__ void store4(T* p, const float (&f)[4]) {
 template <typename InT, typename OutT>
 __global__ void __launch_bounds__(256) swiglu_kernel(const InT* __restrict__ gu, int M, int I,
                                                      OutT* __restrict__ h) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t per_row = I / 4;
   const int64_t total = (int64_t)M * per_row;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -68,6 +70,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const InT* __restrict__ Yp
   // row loads of a thread are independent and issue back to back.
   __shared__ int s_p[32];
   __shared__ float s_w[32];
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   if (t >= T) return;
   const int total = T * k;
@@ -101,6 +105,8 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict
                                                            const int32_t* __restrict__ rows, int k,
                                                            int M_total, __half* __restrict__ Xp,
                                                            int32_t* dev_err) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   bool ovf = false;
@@ -136,10 +142,13 @@ cudaError_t swiglu_out(const InT* gu, int M, int I, void* h, moe_dtype_t h_dt, c
   const int64_t total = (int64_t)M * (I / 4);
   int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
   if (grid < 1) grid = 1;
-  if (h_dt == MOE_DT_F32) swiglu_kernel<<<grid, 256, 0, s>>>(gu, M, I, (float*)h);
-  else if (h_dt == MOE_DT_F16) swiglu_kernel<<<grid, 256, 0, s>>>(gu, M, I, (__half*)h);
-  else swiglu_kernel<<<grid, 256, 0, s>>>(gu, M, I, (__nv_bfloat16*)h);
-  return cudaGetLastError();
+  if (h_dt == MOE_DT_F32)
+    return launch_pdl(swiglu_kernel<InT, float>, dim3(grid), dim3(256), 0, s, gu, M, I, (float*)h);
+  if (h_dt == MOE_DT_F16)
+    return launch_pdl(swiglu_kernel<InT, __half>, dim3(grid), dim3(256), 0, s, gu, M, I,
+                      (__half*)h);
+  return launch_pdl(swiglu_kernel<InT, __nv_bfloat16>, dim3(grid), dim3(256), 0, s, gu, M, I,
+                    (__nv_bfloat16*)h);
 }
 
 template <typename InT>
@@ -148,10 +157,14 @@ cudaError_t combine_out(const InT* Yp, const int32_t* inv_perm, const float* w, 
   const int threads = 256;
   const int ychunks = std::max(1, std::min((H / 4 + threads - 1) / threads, 8));
   const dim3 grid(T, ychunks);
-  if (y_dt == MOE_DT_F32) combine_kernel<<<grid, threads, 0, s>>>(Yp, inv_perm, w, T, k, H, (float*)Y);
-  else if (y_dt == MOE_DT_F16) combine_kernel<<<grid, threads, 0, s>>>(Yp, inv_perm, w, T, k, H, (__half*)Y);
-  else combine_kernel<<<grid, threads, 0, s>>>(Yp, inv_perm, w, T, k, H, (__nv_bfloat16*)Y);
-  return cudaGetLastError();
+  if (y_dt == MOE_DT_F32)
+    return launch_pdl(combine_kernel<InT, float>, grid, dim3(threads), 0, s, Yp, inv_perm, w, T,
+                      k, H, (float*)Y);
+  if (y_dt == MOE_DT_F16)
+    return launch_pdl(combine_kernel<InT, __half>, grid, dim3(threads), 0, s, Yp, inv_perm, w, T,
+                      k, H, (__half*)Y);
+  return launch_pdl(combine_kernel<InT, __nv_bfloat16>, grid, dim3(threads), 0, s, Yp, inv_perm,
+                    w, T, k, H, (__nv_bfloat16*)Y);
 }
 
 }  // namespace
@@ -165,12 +178,11 @@ cudaError_t permute_rows(const void* X, moe_dtype_t x_dt, int T, int K, const in
   const int grid = (int)std::min<int64_t>(((int64_t)M_total + 7) / 8,
                                           (int64_t)moe::sm_count() * 16);
   if (x_dt == MOE_DT_BF16)
-    moe::permute_rows_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, T, K, rows, k, M_total,
-                                                  (__half*)Xp, dev_err);
-  else
-    moe::permute_rows_kernel<<<grid, 256, 0, s>>>((const __half*)X, T, K, rows, k, M_total,
-                                                  (__half*)Xp, dev_err);
-  return cudaGetLastError();
+    return moe::launch_pdl(moe::permute_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
+                           (const __nv_bfloat16*)X, T, K, rows, k, M_total, (__half*)Xp,
+                           dev_err);
+  return moe::launch_pdl(moe::permute_rows_kernel<__half>, dim3(grid), dim3(256), 0, s,
+                         (const __half*)X, T, K, rows, k, M_total, (__half*)Xp, dev_err);
 }
 
 cudaError_t swiglu(const void* gu, moe_dtype_t gu_dt, int M, int I, void* h, moe_dtype_t h_dt,

@@ -12,9 +12,10 @@
 //   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
 //   rows; an expert with more routed rows yields one item per 16).
 // * One producer thread streams each item through a 5-stage ring with TMA
-//   tile loads, 256 k per stage: the packed rows (128 x 128 bytes), their
-//   absmax (128 x 4 fp32) and the routed activation rows (fp16, 8-row boxes
-//   of 64 k), with 128-byte swizzle.
+//   tile loads, 256 k per stage and six copies per stage: the packed rows
+//   (one 3-D box of 2 x 64 rows x 128 bytes), their absmax (one 3-D box of
+//   2 x 64 rows x 4 fp32) and the routed activation rows (one box of 8 or 16
+//   rows per 64-k block), with 128-byte swizzle.
 // * Eight consumer warps each own 16 weight rows and run mma.sync.m16n8k16
 //   with the weights as the M side and the routed rows as N (swap-AB).  A
 //   lane turns each packed byte into an fp16 pair {L[hi], L[lo]} with ONE
@@ -111,6 +112,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
@@ -286,9 +295,14 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
 template <int EPI, typename OutT>
 __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
-    const __grid_constant__ CUtensorMap xmap, const int32_t* __restrict__ offsets, int E, int N,
-    int K, int M_total, OutT* __restrict__ out, int32_t* dev_err) {
+    const __grid_constant__ CUtensorMap xmap8, const __grid_constant__ CUtensorMap xmap16,
+    const int32_t* __restrict__ offsets, int E, int N, int K, int M_total,
+    OutT* __restrict__ out, int32_t* dev_err, int chain) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (!chain) {  // nothing is read or written before the previous kernel is done
+    pdl_wait();
+    pdl_trigger();
+  }
   const uint32_t base = smem_u32(smem_raw);
   if (base > kStage0) {  // layout assumption broken: do nothing, say so
     if (threadIdx.x == 0) set_dev_err(dev_err, MOE_DEVERR_LAYOUT);
@@ -351,33 +365,59 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
   if (warp == CWARPS) {
     // ---------------- producer
     if (lane == 0) {
-      int stage = 0;
+      // the item's 128 weight rows as two 64-row halves (y, z .. z+1) of the
+      // 3-D weight and absmax maps: SwiGLU items take the gate rows and the
+      // matching up rows (z = 2e + half), plain items 128 consecutive rows
+      auto rows_of = [&](const Item& it, int& wy, int& wz) {
+        if (EPI == MOE_EPI_SWIGLU) {
+          wy = it.rtile * (ROWS / 2);
+          wz = 2 * it.expert;
+        } else {
+          wy = 0;
+          wz = it.expert * (N / (ROWS / 2)) + 2 * it.rtile;
+        }
+      };
+      // Chain mode: the weights and absmax of the first ring's worth of
+      // stages are requested before the previous kernel (which writes A) has
+      // finished; their barriers already expect the activation bytes too.
+      int pre = 0;
+      if (chain) {
+        for (int i = blockIdx.x; i < total && pre < STAGES; i += gridDim.x) {
+          const Item it = item_info(ms, offsets, E, rtiles, i);
+          int wy, wz;
+          rows_of(it, wy, wz);
+          const int nr8 = (it.cnt + 7) / 8;
+          for (int s = 0; s < KS && pre < STAGES; ++s, ++pre) {
+            const uint32_t full = smem_u32(&ms.full[pre]);
+            const uint32_t sb = stage_addr(pre);
+            mbar_arrive_expect_tx(full, kWBytes + kABytes + nr8 * 4 * XBOX);
+            tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
+            tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
+          }
+        }
+        pdl_wait();
+        pdl_trigger();
+      }
+      int stage = 0, g = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         const Item it = item_info(ms, offsets, E, rtiles, i);
-        int y0, y1;
-        if (EPI == MOE_EPI_SWIGLU) {
-          y0 = it.expert * N + it.rtile * (ROWS / 2);
-          y1 = y0 + N / 2;
-        } else {
-          y0 = it.expert * N + it.rtile * ROWS;
-          y1 = y0 + ROWS / 2;
-        }
+        int wy, wz;
+        rows_of(it, wy, wz);
         const int nr8 = (it.cnt + 7) / 8;
-        for (int s = 0; s < KS; ++s) {
+        const CUtensorMap* xmap = nr8 > 1 ? &xmap16 : &xmap8;
+        for (int s = 0; s < KS; ++s, ++g) {
           const uint32_t full = smem_u32(&ms.full[stage]);
-          if (!(ok = mbar_wait(smem_u32(&ms.empty[stage]), phase ^ 1, ms, dev_err))) break;
           const uint32_t sb = stage_addr(stage);
-          mbar_arrive_expect_tx(full, kWBytes + kABytes + nr8 * 4 * XBOX);
-          tma_load_2d(sb, &wmap, full, s * SB, y0);
-          tma_load_2d(sb + (ROWS / 2) * SB, &wmap, full, s * SB, y1);
-          tma_load_2d(sb + kWBytes + kXBytes, &amap, full, s * 4, y0);
-          tma_load_2d(sb + kWBytes + kXBytes + (ROWS / 2) * 16, &amap, full, s * 4, y1);
+          if (g >= pre) {  // stages g < pre are slot g, phase 0, weights already requested
+            if (!(ok = mbar_wait(smem_u32(&ms.empty[stage]), phase ^ 1, ms, dev_err))) break;
+            mbar_arrive_expect_tx(full, kWBytes + kABytes + nr8 * 4 * XBOX);
+            tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
+            tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
+          }
           for (int b = 0; b < 4; ++b)
-            for (int r = 0; r < nr8; ++r)
-              tma_load_2d(sb + kWBytes + b * XKBOX + r * XBOX, &xmap, full, s * SK + b * kBlock,
-                          it.start + 8 * r);
+            tma_load_2d(sb + kWBytes + b * XKBOX, xmap, full, s * SK + b * kBlock, it.start);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -405,38 +445,47 @@ int sm_count() { return device_sm_count(); }
 template <int EPI, typename OutT>
 cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
                    const int32_t* offsets, int E, int N, int K, int M_total, void* out,
-                   int32_t* dev_err, cudaStream_t s) {
+                   int32_t* dev_err, cudaStream_t s, bool chain) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
-  CUtensorMap wmap, amap, xmap;
-  const cuuint32_t estr[2] = {1, 1};
+  CUtensorMap wmap, amap, xmap8, xmap16;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  // Weight rows as [z][y][k]: SwiGLU z = 2e + half (gate / up), y = row in
+  // the half; plain z = 64-row group, y = row in the group.  One box of
+  // 2 x 64 rows is an item's 128 rows for one stage.
+  const cuuint64_t ry = (EPI == MOE_EPI_SWIGLU) ? (cuuint64_t)N / 2 : (cuuint64_t)ROWS / 2;
+  const cuuint64_t rz = (cuuint64_t)E * N / ry;
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)E * N};
-    const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
-    const cuuint32_t box[2] = {SB, ROWS / 2};
-    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
+    const cuuint64_t dims[3] = {(cuuint64_t)K / 2, ry, rz};
+    const cuuint64_t strides[2] = {(cuuint64_t)K / 2, ry * (K / 2)};
+    const cuuint32_t box[3] = {SB, ROWS / 2, 2};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)K / kBlock, (cuuint64_t)E * N};
-    const cuuint64_t strides[1] = {(cuuint64_t)K / kBlock * 4};
-    const cuuint32_t box[2] = {SK / kBlock, ROWS / 2};
-    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(absmax), dims, strides,
+    // the absmax of the same rows, 4 blocks (one stage) per row; the L2
+    // fetches whole 128-byte lines, so later stages of a row hit in L2
+    const cuuint64_t dims[3] = {(cuuint64_t)K / kBlock, ry, rz};
+    const cuuint64_t strides[2] = {(cuuint64_t)K / kBlock * 4, ry * (K / kBlock) * 4};
+    const cuuint32_t box[3] = {SK / kBlock, ROWS / 2, 2};
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(absmax), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)A_rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {kBlock, 8};
-    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  for (int rows : {8, 16}) {
+    // routed activation rows: one 64-k block of 8 or 16 rows per box
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)A_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {kBlock, (cuuint32_t)rows};
+    if (enc(rows == 8 ? &xmap8 : &xmap16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   const size_t smem = kEnd;  // absolute layout; the window starts at or below 1 KB
@@ -445,23 +494,22 @@ cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float
   if (err != cudaSuccess) return err;
   const int64_t max_items = ((int64_t)M_total / TOK + E) * (N / ROWS);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_items));
-  kern<<<grid, THREADS, smem, s>>>(wmap, amap, xmap, offsets, E, N, K, M_total,
-                                   reinterpret_cast<OutT*>(out), dev_err);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, wmap, amap, xmap8, xmap16, offsets,
+                    E, N, K, M_total, reinterpret_cast<OutT*>(out), dev_err, chain ? 1 : 0);
 }
 
 template <int EPI>
 cudaError_t launch_out(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
                        const int32_t* offsets, int E, int N, int K, int M_total, void* out,
-                       moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s) {
+                       moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s, bool chain) {
   if (out_dt == MOE_DT_F32)
     return launch<EPI, float>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                              dev_err, s);
+                              dev_err, s, chain);
   if (out_dt == MOE_DT_F16)
     return launch<EPI, __half>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                               dev_err, s);
+                               dev_err, s, chain);
   return launch<EPI, __nv_bfloat16>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                                    dev_err, s);
+                                    dev_err, s, chain);
 }
 
 }  // namespace dec
@@ -478,13 +526,13 @@ bool grouped_gemm_decode_supported(int N, int K) {
 cudaError_t grouped_gemm_decode(const void* A, int A_rows, const uint8_t* packed,
                                 const float* absmax, const int32_t* offsets, int E, int N, int K,
                                 int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
-                                int32_t* dev_err, cudaStream_t s) {
+                                int32_t* dev_err, cudaStream_t s, bool chain) {
   using namespace moe::dec;
   return epi == MOE_EPI_SWIGLU
              ? launch_out<MOE_EPI_SWIGLU>(A, A_rows, packed, absmax, offsets, E, N, K, M_total,
-                                          out, out_dt, dev_err, s)
+                                          out, out_dt, dev_err, s, chain)
              : launch_out<MOE_EPI_NONE>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                                        out_dt, dev_err, s);
+                                        out_dt, dev_err, s, chain);
 }
 
 }  // namespace moe_launch

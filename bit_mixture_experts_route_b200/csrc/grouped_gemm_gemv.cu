@@ -194,6 +194,8 @@ __global__ void __launch_bounds__(32 * kWarps) gemv_nf4_kernel(
     const int32_t* __restrict__ offsets, int E, int N, int K, int M_total,
     OutT* __restrict__ out, int32_t* dev_err) {
   __shared__ uint32_t lut[256 * 32];
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.y;
   const int start = offsets[e], end = offsets[e + 1];
   if (threadIdx.x == 0 && blockIdx.x == 0 && e == 0 &&
@@ -259,15 +261,14 @@ cudaError_t launch_out(const void* A, int A_rows, const int32_t* gather, int k, 
   const dim3 grid(N / kRowsPerCta, E);
   const AT* a = reinterpret_cast<const AT*>(A);
   if (out_dt == MOE_DT_F32)
-    gemv_nf4_kernel<AT, EPI, float><<<grid, 32 * kWarps, 0, s>>>(
-        a, A_rows, gather, k, packed, absmax, offsets, E, N, K, M_total, (float*)out, dev_err);
-  else if (out_dt == MOE_DT_F16)
-    gemv_nf4_kernel<AT, EPI, __half><<<grid, 32 * kWarps, 0, s>>>(
-        a, A_rows, gather, k, packed, absmax, offsets, E, N, K, M_total, (__half*)out, dev_err);
-  else
-    gemv_nf4_kernel<AT, EPI, __nv_bfloat16><<<grid, 32 * kWarps, 0, s>>>(
-        a, A_rows, gather, k, packed, absmax, offsets, E, N, K, M_total, (__nv_bfloat16*)out, dev_err);
-  return cudaGetLastError();
+    return launch_pdl(gemv_nf4_kernel<AT, EPI, float>, grid, dim3(32 * kWarps), 0, s, a, A_rows,
+                      gather, k, packed, absmax, offsets, E, N, K, M_total, (float*)out, dev_err);
+  if (out_dt == MOE_DT_F16)
+    return launch_pdl(gemv_nf4_kernel<AT, EPI, __half>, grid, dim3(32 * kWarps), 0, s, a, A_rows,
+                      gather, k, packed, absmax, offsets, E, N, K, M_total, (__half*)out, dev_err);
+  return launch_pdl(gemv_nf4_kernel<AT, EPI, __nv_bfloat16>, grid, dim3(32 * kWarps), 0, s, a,
+                    A_rows, gather, k, packed, absmax, offsets, E, N, K, M_total,
+                    (__nv_bfloat16*)out, dev_err);
 }
 
 }  // namespace
@@ -280,11 +281,11 @@ cudaError_t grouped_gemm_gemv(const void* A, moe_dtype_t a_dt, int A_rows, const
                               const uint8_t* packed, const float* absmax,
                               const int32_t* offsets, int E, int N, int K, int M_total,
                               moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
-                              int32_t* dev_err, cudaStream_t s) {
+                              int32_t* dev_err, cudaStream_t s, bool chain) {
   if (M_total == 0) return cudaSuccess;
   if (!gather && a_dt == MOE_DT_F16 && grouped_gemm_decode_supported(N, K))
     return grouped_gemm_decode(A, A_rows, packed, absmax, offsets, E, N, K, M_total, epi, out,
-                               out_dt, dev_err, s);
+                               out_dt, dev_err, s, chain);
   using namespace moe;
   if (a_dt == MOE_DT_BF16) {
     return epi == MOE_EPI_SWIGLU

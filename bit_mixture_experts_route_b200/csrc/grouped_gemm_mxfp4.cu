@@ -156,25 +156,6 @@ __device__ __forceinline__ uint32_t mul_h2(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// E8M0 byte -> {2^(b-127), 2^(b-127)} as fp16 bits, exact for b in [103, 142]
-// (fp16 subnormals from 2^-24); 0 below.  *bad is set when b is not 0 and the
-// scaled E2M1 values would not all be exact in fp16 (b outside [104, 140]).
-__device__ __forceinline__ uint32_t scale_h2(uint32_t b, bool& bad) {
-  bad |= (b != 0u) && (b < 104u || b > 140u);
-  uint32_t h = 0;
-  if (b >= 113u && b <= 142u) h = (b - 112u) << 10;   // normal: exponent field b - 127 + 15
-  else if (b >= 103u && b < 113u) h = 1u << (b - 103u);  // subnormal: 2^-24 * 2^(b - 103)
-  return h * 0x00010001u;
-}
-
-// fp16 bits of an E2M1 code's value
-__device__ __forceinline__ uint32_t e2m1_h(uint32_t c) {
-  const uint32_t m = c & 7u;
-  const uint32_t mag = m == 0 ? 0u : m == 1 ? 0x3800u : m == 2 ? 0x3C00u : m == 3 ? 0x3E00u
-                     : m == 4 ? 0x4000u : m == 5 ? 0x4200u : m == 6 ? 0x4400u : 0x4600u;
-  return mag | ((c & 8u) << 12);
-}
-
 // One item's main loop and epilogue for one consumer warp, NT8 token tiles.
 template <int EPI, typename OutT, int NT8>
 __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, int K,
@@ -228,8 +209,8 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
       const int sbi = 2 * b + (t >> 1);
       const uint32_t bA = (mAv[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu;
       const uint32_t bB = (mBv[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu;
-      const uint32_t zA = scale_h2(bA, bad_scale);
-      const uint32_t zB = scale_h2(bB, bad_scale);
+      const uint32_t zA = mx_scale_h2(bA, bad_scale);
+      const uint32_t zB = mx_scale_h2(bB, bad_scale);
       uint32_t xf[NT8][8];
 #pragma unroll
       for (int j = 0; j < NT8; ++j) {

@@ -276,12 +276,33 @@ __device__ __forceinline__ TileInfo tile_info(const Smem& sm, int E, int n_tiles
   return ti;
 }
 
-template <int EPI, typename OutT>
+// A thread's scales of one 64-k stage of its weight row as fp16 pairs for the
+// two 32-element halves: NF4 one fp32 absmax (both halves; `bad` when its
+// fp16 is subnormal or not finite), MXFP4 two E8M0 bytes (`bad` outside the
+// range where every scaled value is exact in fp16).
+template <int FMT>
+__device__ __forceinline__ void stage_scales(uint32_t sc, uint32_t& h0, uint32_t& h1, bool& bad) {
+  if (FMT == kFmtNF4) {
+    const float a = __uint_as_float(sc);
+    bad |= a != 0.0f && !(a >= 6.103515625e-05f && a <= 65504.0f);
+    const __half2 ah = __float2half2_rn(a);
+    h0 = h1 = *reinterpret_cast<const uint32_t*>(&ah);
+  } else {
+    h0 = mx_scale_h2(sc & 0xFFu, bad);
+    h1 = mx_scale_h2((sc >> 8) & 0xFFu, bad);
+  }
+}
+
+template <int FMT, int EPI, typename OutT>
 __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
-    const float* __restrict__ absmax, const int32_t* __restrict__ offsets, int E, int N, int K,
-    int M_total, OutT* __restrict__ out, int32_t* dev_err) {
+    const void* __restrict__ scales, const int32_t* __restrict__ offsets, int E, int N, int K,
+    int M_total, OutT* __restrict__ out, int32_t* dev_err, int chain) {
   extern __shared__ uint8_t smem_raw[];
+  if (!chain) {  // nothing is read or written before the previous kernel is done
+    pdl_wait();
+    pdl_trigger();
+  }
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -306,11 +327,17 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int e = threadIdx.x; e <= E; e += THREADS) sm.off[e] = offsets[e];
+  // byte -> its two weights as an fp16 pair, the lower k in the low half:
+  // NF4 {L[high nibble], L[low nibble]}, MXFP4 {e2m1(low), e2m1(high)}
   for (int i = threadIdx.x; i < 256 * 32; i += THREADS) {
     const int b = i >> 5;
-    const __half2 h = __halves2half2(__float2half_rn(c_levels_tc[b >> 4]),
-                                     __float2half_rn(c_levels_tc[b & 15]));
-    sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+    if (FMT == kFmtNF4) {
+      const __half2 h = __halves2half2(__float2half_rn(c_levels_tc[b >> 4]),
+                                       __float2half_rn(c_levels_tc[b & 15]));
+      sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+      sm.lut[i] = e2m1_h((uint32_t)b & 15u) | (e2m1_h((uint32_t)b >> 4) << 16);
+    }
   }
   if (warp == W_MMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -356,6 +383,12 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   if (warp == W_BPROD) {
     // ---------------- TMA producer: activation tiles, stage S of the CTA
     if (lane == 0) {
+      // chain mode: the previous kernel writes A; the weight producer and the
+      // decoders started without waiting for it
+      if (chain) {
+        pdl_wait();
+        pdl_trigger();
+      }
       // slot S mod BSTAGES is free once the MMAs of stage S - BSTAGES are
       // done; their completion is the a_empty barrier of that stage's TMEM
       // slot (one commit per stage serves both rings)
@@ -450,9 +483,11 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     const int rrow = (EPI == MOE_EPI_SWIGLU) ? ((m & 1) ? BM / 2 + (m >> 1) : (m >> 1)) : m;
     const uint32_t* lut = sm.lut + lane;
     const uint32_t tlane = tmem_base + ((uint32_t)(32 * q) << 16);
-    // absmax of this thread's weight row, block ks of tile t (null past the
-    // CTA's last tile); walked one own stage ahead without divisions
-    auto row_absmax = [&](int t) -> const float* {
+    // scales of this thread's weight row in tile t (null past the CTA's last
+    // tile), stage ks at word ks: NF4 the fp32 absmax of block ks, MXFP4 the
+    // two E8M0 bytes of the stage; walked one own stage ahead without
+    // divisions
+    auto row_scales = [&](int t) -> const uint8_t* {
       if (t >= total) return nullptr;
       const TileId id = tile_id(sm, E, n_tiles, t);
       int row;
@@ -462,14 +497,20 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       } else {
         row = id.ntile * BM + m;
       }
-      return absmax + ((size_t)id.expert * N + row) * (size_t)KT;
+      const size_t r = (size_t)id.expert * N + row;
+      return reinterpret_cast<const uint8_t*>(scales) +
+             (FMT == kFmtNF4 ? r * (size_t)KT * 4 : r * (size_t)(K / 32));
+    };
+    auto fetch = [&](const uint8_t* row, int ks) -> uint32_t {
+      if (FMT == kFmtNF4) return __ldg(reinterpret_cast<const uint32_t*>(row) + ks);
+      return __ldg(reinterpret_cast<const uint16_t*>(row) + ks);
     };
     int n_ks = g, n_t = blockIdx.x;
     while (n_ks >= KT) { n_ks -= KT; n_t += gridDim.x; }
-    const float* n_row = row_absmax(n_t);
-    float a_cur = n_row ? __ldg(n_row + n_ks) : 0.0f;
+    const uint8_t* n_row = row_scales(n_t);
+    uint32_t sc_cur = n_row ? fetch(n_row, n_ks) : 0u;
     bool have = n_row != nullptr;
-    bool bad_scale = false;  // an absmax whose fp16 is subnormal or not finite
+    bool bad_scale = false;  // a scale the fp16 weights cannot carry exactly
     for (int S = g; have; S += GROUPS) {
       const int slot = S % RING, rslot = S % RAW_RING;
       const uint32_t ph = (uint32_t)(S / RING) & 1u, rph = (uint32_t)(S / RAW_RING) & 1u;
@@ -477,21 +518,22 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       while (n_ks >= KT && n_row) {
         n_ks -= KT;
         n_t += gridDim.x;
-        n_row = row_absmax(n_t);
+        n_row = row_scales(n_t);
       }
       const bool have_next = n_row != nullptr;
-      const float a_next = have_next ? __ldg(n_row + n_ks) : 0.0f;  // one stage ahead
+      const uint32_t sc_next = have_next ? fetch(n_row, n_ks) : 0u;  // one stage ahead
       // warp-uniform outcomes: tcgen05.st below is .aligned
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[rslot], rph, sm, dev_err))) break;
       const uint8_t* rp = sm.raw[rslot] + rrow * (BK / 2);
       const uint4 w0 = lds128(rp), w1 = lds128(rp + 16);
-      bad_scale |= a_cur != 0.0f && !(a_cur >= 6.103515625e-05f && a_cur <= 65504.0f);
-      const __half2 ah = __float2half2_rn(a_cur);
+      uint32_t sh[2];
+      stage_scales<FMT>(sc_cur, sh[0], sh[1], bad_scale);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.a_empty[slot], ph ^ 1, sm, dev_err))) break;
       tc_fence_after();
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
+        const __half2 ah = *reinterpret_cast<const __half2*>(&sh[half]);
         uint32_t hv[16];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -512,7 +554,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         mbar_arrive(&sm.ready[slot]);
         mbar_arrive(&sm.raw_empty[rslot]);  // its bytes are decoded
       }
-      a_cur = a_next;
+      sc_cur = sc_next;
       have = have_next;
     }
     // the loop exits are warp-uniform, so every lane takes part
@@ -613,10 +655,10 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
 
 int sm_count() { return device_sm_count(); }
 
-template <int EPI, typename OutT>
-cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
+template <int FMT, int EPI, typename OutT>
+cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
                    const int32_t* offsets, int E, int N, int K, int M_total, void* out,
-                   int32_t* dev_err, cudaStream_t s) {
+                   int32_t* dev_err, cudaStream_t s, bool chain) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
   CUtensorMap map, wmap;
@@ -643,16 +685,40 @@ cudaError_t launch(const void* A, const uint8_t* packed, const float* absmax,
       return cudaErrorInvalidValue;
   }
   const size_t smem = sizeof(Smem) + 1024;
-  auto kern = nf4_tc_kernel<EPI, OutT>;
+  auto kern = nf4_tc_kernel<FMT, EPI, OutT>;
   cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
   // Upper bound on tiles: every expert's rows rounded up to BN, plus one
   // partial tile per expert; the kernel derives the exact list itself.
   const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / BM);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-  kern<<<grid, THREADS, smem, s>>>(map, wmap, absmax, offsets, E, N, K, M_total,
-                                   reinterpret_cast<OutT*>(out), dev_err);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, wmap, scales, offsets, E, N, K,
+                    M_total, reinterpret_cast<OutT*>(out), dev_err, chain ? 1 : 0);
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const void* A, const uint8_t* packed, const void* scales,
+                       const int32_t* offsets, int E, int N, int K, int M_total,
+                       moe_epilogue_t epi, void* out, moe_dtype_t out_dt, int32_t* dev_err,
+                       cudaStream_t s, bool chain) {
+  if (epi == MOE_EPI_SWIGLU) {
+    if (out_dt == MOE_DT_F16)
+      return launch<FMT, MOE_EPI_SWIGLU, __half>(A, packed, scales, offsets, E, N, K, M_total,
+                                                 out, dev_err, s, chain);
+    if (out_dt == MOE_DT_BF16)
+      return launch<FMT, MOE_EPI_SWIGLU, __nv_bfloat16>(A, packed, scales, offsets, E, N, K,
+                                                        M_total, out, dev_err, s, chain);
+    return launch<FMT, MOE_EPI_SWIGLU, float>(A, packed, scales, offsets, E, N, K, M_total, out,
+                                              dev_err, s, chain);
+  }
+  if (out_dt == MOE_DT_F16)
+    return launch<FMT, MOE_EPI_NONE, __half>(A, packed, scales, offsets, E, N, K, M_total, out,
+                                             dev_err, s, chain);
+  if (out_dt == MOE_DT_BF16)
+    return launch<FMT, MOE_EPI_NONE, __nv_bfloat16>(A, packed, scales, offsets, E, N, K,
+                                                    M_total, out, dev_err, s, chain);
+  return launch<FMT, MOE_EPI_NONE, float>(A, packed, scales, offsets, E, N, K, M_total, out,
+                                          dev_err, s, chain);
 }
 
 }  // namespace tc
@@ -669,28 +735,20 @@ cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows, const i
                             int k, const uint8_t* packed, const float* absmax,
                             const int32_t* offsets, int E, int N, int K, int M_total,
                             moe_epilogue_t epi, void* out, moe_dtype_t out_dt, int32_t* dev_err,
-                            cudaStream_t s) {
+                            cudaStream_t s, bool chain) {
   (void)k;
   if (gather || a_dt != MOE_DT_F16 || A_rows < M_total) return cudaErrorNotSupported;
-  using namespace moe::tc;
-  if (epi == MOE_EPI_SWIGLU) {
-    if (out_dt == MOE_DT_F16)
-      return launch<MOE_EPI_SWIGLU, __half>(A, packed, absmax, offsets, E, N, K, M_total, out,
-                                            dev_err, s);
-    if (out_dt == MOE_DT_BF16)
-      return launch<MOE_EPI_SWIGLU, __nv_bfloat16>(A, packed, absmax, offsets, E, N, K,
-                                                   M_total, out, dev_err, s);
-    return launch<MOE_EPI_SWIGLU, float>(A, packed, absmax, offsets, E, N, K, M_total, out,
-                                         dev_err, s);
-  }
-  if (out_dt == MOE_DT_F16)
-    return launch<MOE_EPI_NONE, __half>(A, packed, absmax, offsets, E, N, K, M_total, out,
-                                        dev_err, s);
-  if (out_dt == MOE_DT_BF16)
-    return launch<MOE_EPI_NONE, __nv_bfloat16>(A, packed, absmax, offsets, E, N, K, M_total,
-                                               out, dev_err, s);
-  return launch<MOE_EPI_NONE, float>(A, packed, absmax, offsets, E, N, K, M_total, out,
-                                     dev_err, s);
+  return moe::tc::launch_fmt<moe::kFmtNF4>(A, packed, absmax, offsets, E, N, K, M_total, epi,
+                                           out, out_dt, dev_err, s, chain);
+}
+
+cudaError_t grouped_gemm_tc_mxfp4(const void* A, int A_rows, const uint8_t* packed,
+                                  const uint8_t* scales, const int32_t* offsets, int E, int N,
+                                  int K, int M_total, moe_epilogue_t epi, void* out,
+                                  moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s) {
+  if (A_rows < M_total) return cudaErrorNotSupported;
+  return moe::tc::launch_fmt<moe::kFmtMXFP4>(A, packed, scales, offsets, E, N, K, M_total, epi,
+                                             out, out_dt, dev_err, s, false);
 }
 
 }  // namespace moe_launch

@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kThreads) route_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     int32_t* __restrict__ rank, int32_t* __restrict__ tile_counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_eid[kTileTok * 32];
   __shared__ int s_cnt[1024];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -169,6 +171,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
     int32_t* __restrict__ inv_perm) {
+  pdl_wait();
+  pdl_trigger();
   // 16-bit fields: rows, ranks and counts are all < kSmallRows = 4096
   __shared__ int16_t s_eid[kSmallRows];
   __shared__ uint16_t s_rank[kSmallRows];
@@ -305,6 +309,8 @@ __global__ void __launch_bounds__(kThreads) permute_scatter_kernel(
     const int32_t* __restrict__ tile_counts, int T, int E, int k, int ntiles,
     int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
     int32_t* __restrict__ inv_perm) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_off[1024];
   __shared__ int s_before[1024];
   __shared__ int s_warp[kThreads / 32];
@@ -361,37 +367,34 @@ cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
                           cudaStream_t s) {
   if (T == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
   if ((int64_t)T * k <= moe::kSmallRows && E <= moe::kSmallE) {
-#define MOE_ROUTE_SMALL(NP)                                                           \
-  moe::route_small_kernel<NP><<<1, moe::kSmallThreads, 0, s>>>(logits, T, E, k, renorm, \
-                                                               topk_idx, topk_w, offsets, \
-                                                               sorted_rows, inv_perm)
-    if (E <= 32) MOE_ROUTE_SMALL(1);
-    else if (E <= 64) MOE_ROUTE_SMALL(2);
-    else if (E <= 128) MOE_ROUTE_SMALL(4);
-    else MOE_ROUTE_SMALL(8);
+#define MOE_ROUTE_SMALL(NP)                                                             \
+  moe::launch_pdl(moe::route_small_kernel<NP>, dim3(1), dim3(moe::kSmallThreads), 0, s, logits, \
+                  T, E, k, renorm, topk_idx, topk_w, offsets, sorted_rows, inv_perm)
+    if (E <= 32) return MOE_ROUTE_SMALL(1);
+    if (E <= 64) return MOE_ROUTE_SMALL(2);
+    if (E <= 128) return MOE_ROUTE_SMALL(4);
+    return MOE_ROUTE_SMALL(8);
 #undef MOE_ROUTE_SMALL
-    return cudaGetLastError();
   }
   const int ntiles = (T + moe::kTileTok - 1) / moe::kTileTok;
   int32_t* rank = reinterpret_cast<int32_t*>(ws);
   int32_t* tile_counts =
       reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + align256((size_t)T * k * 4));
-#define MOE_ROUTE_LAUNCH(NP)                                                          \
-  moe::route_tile_kernel<NP><<<ntiles, moe::kThreads, 0, s>>>(logits, T, E, k, renorm, \
-                                                              topk_idx, topk_w, rank,  \
-                                                              tile_counts)
-  if (E <= 32) MOE_ROUTE_LAUNCH(1);
-  else if (E <= 64) MOE_ROUTE_LAUNCH(2);
-  else if (E <= 128) MOE_ROUTE_LAUNCH(4);
-  else if (E <= 256) MOE_ROUTE_LAUNCH(8);
-  else if (E <= 512) MOE_ROUTE_LAUNCH(16);
-  else MOE_ROUTE_LAUNCH(32);
+#define MOE_ROUTE_LAUNCH(NP)                                                           \
+  moe::launch_pdl(moe::route_tile_kernel<NP>, dim3(ntiles), dim3(moe::kThreads), 0, s, logits, \
+                  T, E, k, renorm, topk_idx, topk_w, rank, tile_counts)
+  cudaError_t err;
+  if (E <= 32) err = MOE_ROUTE_LAUNCH(1);
+  else if (E <= 64) err = MOE_ROUTE_LAUNCH(2);
+  else if (E <= 128) err = MOE_ROUTE_LAUNCH(4);
+  else if (E <= 256) err = MOE_ROUTE_LAUNCH(8);
+  else if (E <= 512) err = MOE_ROUTE_LAUNCH(16);
+  else err = MOE_ROUTE_LAUNCH(32);
 #undef MOE_ROUTE_LAUNCH
-  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  moe::permute_scatter_kernel<<<ntiles, moe::kThreads, 0, s>>>(
-      topk_idx, rank, tile_counts, T, E, k, ntiles, offsets, sorted_rows, inv_perm);
-  return cudaGetLastError();
+  return moe::launch_pdl(moe::permute_scatter_kernel, dim3(ntiles), dim3(moe::kThreads), 0, s,
+                         topk_idx, rank, tile_counts, T, E, k, ntiles, offsets, sorted_rows,
+                         inv_perm);
 }
 
 // ---------------------------------------------------------------------------

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define MOE_NF4_ABI_VERSION 1
+#define MOE_NF4_ABI_VERSION 2
 
 typedef enum {
   MOE_OK = 0,
@@ -215,7 +215,7 @@ moe_status_t moe_mxfp4_quantize(const float* W, int E, int N, int K, uint8_t* pa
                                 uint8_t* scales, int32_t* dev_err, void* stream);
 
 /*
- * moe_mxfp4_grouped_gemm -- decode-shaped grouped GEMM on MXFP4 weights:
+ * moe_mxfp4_grouped_gemm -- grouped GEMM on MXFP4 weights:
  * out[p] = W[e(p)] @ A[p] for every row p in expert e's segment
  * [expert_offsets[e], expert_offsets[e+1]), W[e] = 2^(b - 127) * e2m1(code)
  * from (packed, scales) as written by moe_mxfp4_quantize or taken unchanged
@@ -224,21 +224,30 @@ moe_status_t moe_mxfp4_quantize(const float* W, int E, int N, int K, uint8_t* pa
  *   A        fp16 [A_rows >= M_total, K]  routed rows in permuted order
  *   packed   uint8 [E, N, K/2], scales uint8 [E, N, K/32]
  *   expert_offsets int32 [E+1] (device), monotone, offsets[E] == M_total
- *   N % 128 == 0, K % 256 == 0, E <= 1024
+ *   E <= 1024; GEMV kernel: N % 128 == 0, K % 256 == 0; tensor-core kernel:
+ *            N % 128 == 0, K % 64 == 0
  *   epilogue MOE_EPI_NONE: out [M_total, N]; MOE_EPI_SWIGLU: rows [0, N/2)
  *            are gate and [N/2, N) up, out [M_total, N/2] = silu(g) * u
  *   out      F32 / F16 / BF16
+ *   algo     AUTO takes the tensor-core kernel (tcgen05, TMEM accumulators)
+ *            from 36 routed rows per expert on average, as the NF4 call does,
+ *            else the decode GEMV; GEMV / TC force one
  *   dev_err  BAD_OFFSETS, TIMEOUT, LAYOUT as moe_nf4_grouped_gemm; RANGE when
  *            a scale byte is neither 0 nor in [104, 140], where the weights
- *            are not exact in fp16 (products then rounded or flushed)
- * The weights enter the MMA as exact fp16 values (E2M1 times the scale's power
- * of two); sums are fp32.  Streams every selected expert's bytes once.
+ *            are not exact in fp16 (products then rounded or flushed), or an
+ *            fp16 output overflowed
+ * Both kernels feed the weights to the tensor cores as exact fp16 values
+ * (E2M1 times the scale's power of two) with fp16 activations; sums are fp32.
+ * (Blackwell's block-scaled kind::mxf4 MMA would take the codes and scales
+ * directly, but it needs the activations in FP4 or FP8 as well, which puts
+ * the layer outside the parity tolerance; see the design notes.)
  * All pointers 16-byte aligned.
  */
 moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
                                     const uint8_t* scales, const int32_t* expert_offsets, int E,
                                     int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
-                                    moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
+                                    moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
+                                    void* stream);
 
 /*
  * Backward of the layer with the 4-bit experts frozen ("grouped-nf4-gemm &

@@ -48,8 +48,8 @@ int main(int argc, char** argv) {
     void* P = load("mx_P.bin", (size_t)E * N * K / 2); void* S = load("mx_S.bin", (size_t)E * N * K / 32);
     void* X = load("mx_X.bin", (size_t)M * K * 2); int32_t* off = (int32_t*)load("mx_off.bin", (E + 1) * 4);
     float* o1 = (float*)zeros((size_t)M * N * 4); float* o2 = (float*)zeros((size_t)M * N / 2 * 4);
-    ST(moe_mxfp4_grouped_gemm(X, M, (uint8_t*)P, (uint8_t*)S, off, E, N, K, M, MOE_EPI_NONE, o1, MOE_DT_F32, err, nullptr));
-    ST(moe_mxfp4_grouped_gemm(X, M, (uint8_t*)P, (uint8_t*)S, off, E, N, K, M, MOE_EPI_SWIGLU, o2, MOE_DT_F32, err, nullptr));
+    ST(moe_mxfp4_grouped_gemm(X, M, (uint8_t*)P, (uint8_t*)S, off, E, N, K, M, MOE_EPI_NONE, o1, MOE_DT_F32, MOE_ALGO_GEMV, err, nullptr));
+    ST(moe_mxfp4_grouped_gemm(X, M, (uint8_t*)P, (uint8_t*)S, off, E, N, K, M, MOE_EPI_SWIGLU, o2, MOE_DT_F32, MOE_ALGO_GEMV, err, nullptr));
     CK(cudaDeviceSynchronize());
     printf("mxfp4_gemm dev_err=%d\n", err_word(err));
     dump("mxg_none.bin", o1, (size_t)M * N * 4); dump("mxg_swiglu.bin", o2, (size_t)M * N / 2 * 4); }

@@ -27,15 +27,26 @@ def errors(y, ref):
 
 
 def assert_close_16bit(y, ref, dtype, what=""):
-    """A 16-bit output against the oracle, both ways.  The survey's reading
-    counts the output's own rounding as error, so ``y`` must meet the bar
-    against the unrounded oracle value; it must also meet it against that
-    value rounded once to ``dtype``, which isolates the kernel's arithmetic
-    from the final rounding."""
-    r1 = assert_close(y, ref, f"{what} (unrounded oracle)")
-    ref_rounded = torch.from_numpy(np.asarray(ref, dtype=np.float64)).to(dtype).double().numpy()
+    """A 16-bit output against the oracle, both ways.
+
+    Against the oracle value rounded once to ``dtype`` it must meet the full
+    bar: that isolates the kernel's arithmetic from the final rounding.
+    Against the unrounded oracle (the output's own rounding counted as error)
+    it must meet rel_max <= 1e-2, and mae <= 1e-3 * RMS for fp16; for bf16 the
+    rounding alone costs about 1e-3 * RMS on average (2^-9 of each value's
+    power of two), so there the bound is 1e-3 * RMS plus the mean error of
+    rounding the oracle itself to bf16."""
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    ref_rounded = torch.from_numpy(ref).to(dtype).double().numpy()
     r2 = assert_close(y, ref_rounded, f"{what} (oracle rounded to {dtype})")
-    return r1, r2
+    rel, mae = errors(y, ref)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    allowance = 0.0 if dtype == torch.float16 else float(np.mean(np.abs(ref_rounded - ref))) / rms
+    assert rel <= REL_MAX and mae <= MAE_RMS + allowance, (
+        f"{what} (unrounded oracle): rel_max={rel:.3e} mae/rms={mae:.3e} "
+        f"(bound {MAE_RMS + allowance:.3e})")
+    return (rel, mae), r2
 
 
 def assert_close(y, ref, what=""):

@@ -47,7 +47,7 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     for code, name in _lib.STATUS.items():
         assert lib.moe_status_string(code).decode() == name
 
@@ -158,15 +158,20 @@ def test_mxfp4_calls_reject_bad_arguments(lib):
     assert lib.moe_mxfp4_quantize(A, 1, 8, 48, A, A, None, None) == 1
     assert lib.moe_mxfp4_quantize(A, 1, 8, 64, A, None, None, None) == 1
     assert lib.moe_mxfp4_quantize(A, 1, 8, 64, A, M, None, None) == 2
-    # grouped GEMM: N % 128 or K % 256 -> unsupported; bad epilogue / dtype;
-    # A_rows < M_total; misaligned scales
+    # grouped GEMM (..., epilogue, out, out_dtype, algo, dev_err, stream):
+    # N % 128 or K % 64 -> unsupported by both kernels; K % 256 != 0 ->
+    # unsupported by the GEMV; bad epilogue / dtype / algo; A_rows < M_total;
+    # misaligned scales
     g = lib.moe_mxfp4_grouped_gemm
-    assert g(A, 8, A, A, A, 2, 64, 256, 8, 0, A, 0, None, None) == 3
-    assert g(A, 8, A, A, A, 2, 128, 288, 8, 0, A, 0, None, None) == 3
-    assert g(A, 8, A, A, A, 2, 128, 256, 8, 5, A, 0, None, None) == 1
-    assert g(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 4, None, None) == 1
-    assert g(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, None, None) == 1
-    assert g(A, 8, A, M, A, 2, 128, 256, 8, 0, A, 0, None, None) == 2
+    assert g(A, 8, A, A, A, 2, 64, 256, 8, 0, A, 0, 0, None, None) == 3
+    assert g(A, 8, A, A, A, 2, 128, 288, 8, 0, A, 0, 0, None, None) == 3
+    assert g(A, 8, A, A, A, 2, 128, 320, 8, 0, A, 0, 1, None, None) == 3
+    assert g(A, 8, A, A, A, 2, 64, 320, 8, 0, A, 0, 2, None, None) == 3
+    assert g(A, 8, A, A, A, 2, 128, 256, 8, 5, A, 0, 0, None, None) == 1
+    assert g(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 4, 0, None, None) == 1
+    assert g(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 0, 7, None, None) == 1
+    assert g(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, 0, None, None) == 1
+    assert g(A, 8, A, M, A, 2, 128, 256, 8, 0, A, 0, 0, None, None) == 2
 
 
 def test_backward_calls_reject_bad_arguments(lib):
