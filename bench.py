@@ -72,10 +72,10 @@ def parse_args():
                    help="time the headline (or --config) workload only")
     p.add_argument("--tokens", type=int, default=None, help="token batch T")
     p.add_argument("--layers", type=int, default=None)
-    p.add_argument("--algo", choices=["auto", "gemv", "tc"], default="auto")
+    p.add_argument("--algo", choices=["auto", "gemv", "tc", "tc_pair"], default="auto")
     p.add_argument("--weights", choices=["nf4", "int4", "mxfp4"], default="nf4",
                    help="expert weight format (int4: grouped GPTQ-style codes; mxfp4: e2m1 + "
-                        "e8m0 per 32; both run the decode GEMV only)")
+                        "e8m0 per 32)")
     p.add_argument("--backward", action="store_true",
                    help="time forward + backward of each layer (4-bit experts frozen)")
     p.add_argument("--lora", type=int, default=0, metavar="RANK",
@@ -335,7 +335,8 @@ class Workload:
 
     def _gemm(self, A, packed, scales, offsets, M, out, algo, epilogue="none"):
         if self.fmt == "int4":
-            self.moe.int4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out)
+            self.moe.int4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out,
+                                       algo=algo)
         elif self.fmt == "mxfp4":
             self.moe.mxfp4_grouped_gemm(A, packed, scales, offsets, M, epilogue=epilogue, out=out,
                                         algo=algo)
@@ -370,12 +371,29 @@ class Workload:
             moe.lora_delta(self.Hbuf, off, A_d, B_d, scale, self.Yp32, M_total=M)
         moe.unpermute_combine(self.Yp32, r["inv_perm"], r["topk_w"], out=self.Y)
         if self.backward:
-            dYp, dw = moe.combine_backward(self.dY, self.Yp32, r["inv_perm"], r["topk_w"])
-            dH = moe.nf4_grouped_gemm_t(dYp, p_d, a_d, off, M)
-            dGU = moe.swiglu_backward(self.GU, dH)
-            dXp = moe.nf4_grouped_gemm_t(dGU, p_gu, a_gu, off, M)
+            sh = self.shape
+            if self.tc_backward():
+                # tensor cores: fp16 row gradients, the transposed down GEMM
+                # and the SwiGLU backward in one launch, the transposed gate_up
+                dYp, dw = moe.combine_backward(self.dY, self.Yp32, r["inv_perm"], r["topk_w"],
+                                               dyp_dtype=torch.float16)
+                dGU = moe.nf4_down_backward(dYp, p_d, a_d, off, M, self.GU,
+                                            out_dtype=torch.float16)
+                dXp = moe.nf4_grouped_gemm_t(dGU, p_gu, a_gu, off, M, algo="tc")
+            else:
+                dYp, dw = moe.combine_backward(self.dY, self.Yp32, r["inv_perm"], r["topk_w"])
+                dH = moe.nf4_grouped_gemm_t(dYp, p_d, a_d, off, M, algo="gemv")
+                dGU = moe.swiglu_backward(self.GU, dH)
+                dXp = moe.nf4_grouped_gemm_t(dGU, p_gu, a_gu, off, M, algo="gemv")
             moe.unpermute_combine(dXp, r["inv_perm"], self.ones, out=self.dX)
-            moe.route_backward(logits, r["topk_idx"], r["topk_w"], dw, self.shape.renormalize)
+            moe.route_backward(logits, r["topk_idx"], r["topk_w"], dw, sh.renormalize)
+
+    def tc_backward(self):
+        """The backward runs on the tensor cores from 36 routed rows per expert
+        on average (the forward's rule) when the shapes allow it."""
+        sh = self.shape
+        return (self.T * sh.k >= 36 * sh.E and sh.H % 64 == 0 and sh.I % 256 == 0
+                and sh.H % 256 == 0 and (2 * sh.I) % 64 == 0)
 
     def lora_bytes(self, d):
         """Algorithmic bytes of the gate_up adapter launch: the distinct
@@ -558,6 +576,14 @@ def run_reference(args, shape, T, layers):
 
 # ----------------------------------------------------------------- one workload
 
+def _cuda_fault(exc):
+    """An exception that reports a fault on the device (the context is lost)
+    rather than a call that stream capture does not allow."""
+    msg = str(exc)
+    return any(m in msg for m in ("launch failure", "illegal", "misaligned", "Xid",
+                                   "device-side assert", "unspecified"))
+
+
 def graphed_replay(wl, algo, steps, warmup, world, local):
     """The layer steps captured as one CUDA graph and replayed ``steps``
     times (how a decode server issues a step): same kernels and work as the
@@ -580,6 +606,8 @@ def graphed_replay(wl, algo, steps, warmup, world, local):
         torch.cuda.synchronize()
         captured = 1.0
     except Exception as exc:  # noqa: BLE001
+        if _cuda_fault(exc):
+            raise  # a fault on the device is not a capture failure
         err = {"error": str(exc)[:200]}
         captured = 0.0
     # every rank takes the same collective steps: time only if all captured
@@ -758,15 +786,13 @@ def main():
     world, rank, local = dist_setup()
     import bit_mixture_experts_route_b200 as moe
     moe.load()
-    if args.weights == "int4" and T * shape.k >= 36 * shape.E:
-        raise SystemExit("int4 weights have the decode GEMV path only (fewer than 36 routed rows "
-                         "per expert)")
     if args.backward and args.weights != "nf4":
         raise SystemExit("--backward runs on NF4 weights (the transposed GEMM is NF4)")
     hbm, tf_burst, tf_sust, peak_kind = load_peaks()
     seed = rank_seed(args.seed, rank)
     wl = Workload(shape, T, layers, seed, weights=args.weights, lora=args.lora,
                   backward=args.backward)
+    wl_tc_backward = args.backward and wl.tc_backward()
     workload_name = (args.config + (f"/{args.weights}" if args.weights != "nf4" else "")
                      + (f"/lora-r{args.lora}" if args.lora else "")
                      + ("/fwd+bwd" if args.backward else ""))
@@ -831,6 +857,7 @@ def main():
                 torch.cuda.empty_cache()
                 current = (cfg, Workload(sh, t, nl, seed))
             w = current[1]
+            print(f"[bench] {cfg} T={t}", file=sys.stderr, flush=True)
             w.set_tokens(t)
             entry = run_workload(w, cfg, args, sweep_steps, world, local, hbm, tf_burst,
                                  tf_sust, peak_kind)
@@ -850,6 +877,8 @@ def main():
     # backward, scatter-add and routing backward
     launches_per_layer = (6 + (1 if (args.lora or args.backward) else 0) + (2 if args.lora else 0)
                           + (6 if args.backward else 0))
+    if args.backward and wl_tc_backward:
+        launches_per_layer -= 1     # the fused down + SwiGLU backward
     line = {
         "metric": "MoE layer tokens/s", "value": head["value"], "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

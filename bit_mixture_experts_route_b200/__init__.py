@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     int4_grouped_gemm,
     lora_delta,
     nf4_grouped_gemm_t,
+    nf4_down_backward,
     swiglu_backward,
     combine_backward,
     route_backward,

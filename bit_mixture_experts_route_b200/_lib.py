@@ -22,7 +22,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED",
           3: "MOE_ERR_UNSUPPORTED", 4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA"}
 DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EPI = {"none": 0, "swiglu": 1}
-ALGO = {"auto": 0, "gemv": 1, "tc": 2}
+ALGO = {"auto": 0, "gemv": 1, "tc": 2, "tc_pair": 3}
 DEVERR_NONFINITE, DEVERR_BAD_OFFSETS, DEVERR_BAD_INDEX, DEVERR_TIMEOUT = 1, 2, 4, 8
 DEVERR_LAYOUT, DEVERR_RANGE = 0x10, 0x20
 
@@ -41,11 +41,13 @@ SIGNATURES = {
     "moe_nf4_grouped_gemm": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P,
                                   _I, _I, _P, _S]),
     "moe_int4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
-    "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_int4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P, _S]),
     "moe_mxfp4_quantize": (_I, [_P, _I, _I, _I, _P, _P, _P, _S]),
     "moe_mxfp4_grouped_gemm": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P,
                                     _S]),
-    "moe_nf4_grouped_gemm_t": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _S]),
+    "moe_nf4_grouped_gemm_t": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P,
+                                    _S]),
+    "moe_nf4_down_backward": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _S]),
     "moe_swiglu_backward": (_I, [_P, _P, _I, _I, _I, _P, _I, _S]),
     "moe_combine_backward": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _P, _S]),
     "moe_route_backward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _S]),
@@ -243,9 +245,9 @@ def int4_quantize(W, packed=None, meta=None, dev_err=None):
 
 
 def int4_grouped_gemm(A, packed, meta, expert_offsets, M_total, epilogue="none",
-                      out_dtype=torch.float32, out=None, dev_err=None):
-    """Decode-shaped grouped GEMM on INT4 weights, all experts in one launch
-    (see the header); ``A`` fp16 rows in permuted order."""
+                      out_dtype=torch.float32, out=None, dev_err=None, algo="auto"):
+    """Grouped GEMM on INT4 weights, all experts in one launch (decode GEMV or
+    tensor-core kernel, see the header); ``A`` fp16 rows in permuted order."""
     _need(A, torch.float16, "A", 2)
     _need(packed, torch.uint8, "packed", 3)
     _need(meta, torch.int32, "meta", 3)
@@ -262,7 +264,7 @@ def int4_grouped_gemm(A, packed, meta, expert_offsets, M_total, epilogue="none",
     _room(out, M_total * n_out, "out", _F)
     _check(load().moe_int4_grouped_gemm(
         _ptr(A), A.shape[0], _ptr(packed), _ptr(meta), _ptr(expert_offsets), E, N, K, M_total,
-        EPI[epilogue], _ptr(out), DT[out.dtype], _ptr(dev_err), _stream(A.device)),
+        EPI[epilogue], _ptr(out), DT[out.dtype], ALGO[algo], _ptr(dev_err), _stream(A.device)),
         "moe_int4_grouped_gemm")
     return out
 
@@ -309,7 +311,7 @@ def mxfp4_grouped_gemm(A, packed, scales, expert_offsets, M_total, epilogue="non
 
 
 def nf4_grouped_gemm_t(G, packed, absmax, expert_offsets, M_total, out_dtype=torch.float32,
-                       out=None, dev_err=None):
+                       out=None, dev_err=None, algo="auto"):
     """Transposed grouped NF4 GEMM: ``out[p] = W[e(p)]^T @ G[p]`` -> ``[M_total, K]``;
     ``G`` fp32 or fp16 ``[>= M_total, N]`` (the backward of ``nf4_grouped_gemm``)."""
     if G.dtype not in (torch.float32, torch.float16):
@@ -329,8 +331,35 @@ def nf4_grouped_gemm_t(G, packed, absmax, expert_offsets, M_total, out_dtype=tor
     _room(out, M_total * K, "out", (torch.float32, torch.float16))
     _check(load().moe_nf4_grouped_gemm_t(_ptr(G), DT[G.dtype], G.shape[0], _ptr(packed),
                                          _ptr(absmax), _ptr(expert_offsets), E, N, K, M_total,
-                                         _ptr(out), DT[out.dtype], _ptr(dev_err),
+                                         _ptr(out), DT[out.dtype], ALGO[algo], _ptr(dev_err),
                                          _stream(G.device)), "moe_nf4_grouped_gemm_t")
+    return out
+
+
+def nf4_down_backward(dYp, packed, absmax, expert_offsets, M_total, gu, out_dtype=torch.float32,
+                      out=None, dev_err=None):
+    """Transposed down GEMM + SwiGLU backward in one tensor-core launch:
+    ``dYp`` fp16 ``[>= M_total, H]``, the down stack ``[E, H, I]``, ``gu`` fp32
+    ``[M_total, 2I]`` (the forward's pre-activations) -> ``dgu [M_total, 2I]``."""
+    _need(dYp, torch.float16, "dYp", 2)
+    _need(packed, torch.uint8, "packed", 3)
+    _need(absmax, torch.float32, "absmax")
+    _need(expert_offsets, torch.int32, "expert_offsets", 1)
+    _need(gu, torch.float32, "gu", 2)
+    E, H, half = packed.shape
+    I = 2 * half
+    if dYp.shape[1] != H or gu.shape[1] != 2 * I:
+        raise MoEError("dYp [*, H] and gu [*, 2I] must match the down stack [E, H, I]")
+    _room(absmax, E * H * (I // 64), "absmax")
+    _room(expert_offsets, E + 1, "expert_offsets")
+    _room(gu, M_total * 2 * I, "gu")
+    if out is None:
+        out = torch.empty((M_total, 2 * I), dtype=out_dtype, device=dYp.device)
+    _room(out, M_total * 2 * I, "out", (torch.float32, torch.float16))
+    _check(load().moe_nf4_down_backward(_ptr(dYp), dYp.shape[0], _ptr(packed), _ptr(absmax),
+                                        _ptr(expert_offsets), E, H, I, M_total, _ptr(gu),
+                                        _ptr(out), DT[out.dtype], _ptr(dev_err),
+                                        _stream(dYp.device)), "moe_nf4_down_backward")
     return out
 
 

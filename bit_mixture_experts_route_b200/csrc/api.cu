@@ -82,12 +82,19 @@ moe_status_t moe_int4_quantize(const float* W, int E, int N, int K, uint8_t* pac
 moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
                                    const uint32_t* meta, const int32_t* expert_offsets, int E,
                                    int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
-                                   moe_dtype_t out_dtype, int32_t* dev_err, void* stream) {
+                                   moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
+                                   void* stream) {
   if (E < 1 || E > 1024 || N < 1 || K < 1 || M_total < 0 || A_rows < M_total)
     return MOE_ERR_INVALID_ARG;
   if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (!valid_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
-  if (!moe_launch::grouped_gemm_int4_supported(N, K)) return MOE_ERR_UNSUPPORTED;
+  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC)
+    return MOE_ERR_INVALID_ARG;
+  const bool gemv_ok = moe_launch::grouped_gemm_int4_supported(N, K);
+  const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue) && K % 128 == 0;
+  const bool use_tc = algo == MOE_ALGO_TC ||
+                      (algo == MOE_ALGO_AUTO && tc_ok && ((int64_t)M_total >= 36LL * E || !gemv_ok));
+  if (use_tc ? !tc_ok : !gemv_ok) return MOE_ERR_UNSUPPORTED;
   if (!expert_offsets || !packed || !meta) return MOE_ERR_INVALID_ARG;
   if (M_total > 0 && (!A || !out)) return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {A, packed, meta, expert_offsets, out};
@@ -95,6 +102,10 @@ moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* pac
     if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
   if (moe_status_t st = check_device()) return st;
   if (M_total == 0) return MOE_OK;
+  if (use_tc)
+    return from_cuda(moe_launch::grouped_gemm_tc_int4(A, A_rows, packed, meta, expert_offsets, E,
+                                                      N, K, M_total, epilogue, out, out_dtype,
+                                                      dev_err, (cudaStream_t)stream));
   return from_cuda(moe_launch::grouped_gemm_int4(A, A_rows, packed, meta, expert_offsets, E, N,
                                                  K, M_total, epilogue, out, out_dtype, dev_err,
                                                  (cudaStream_t)stream));
@@ -119,12 +130,14 @@ moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* pa
     return MOE_ERR_INVALID_ARG;
   if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (!valid_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
-  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC)
+  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC &&
+      algo != MOE_ALGO_TC_PAIR)
     return MOE_ERR_INVALID_ARG;
   const bool gemv_ok = moe_launch::grouped_gemm_mxfp4_supported(N, K);
-  const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue);
+  const bool pair = algo == MOE_ALGO_TC_PAIR;
+  const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue) && (!pair || N % 256 == 0);
   bool use_tc;
-  if (algo == MOE_ALGO_TC) use_tc = true;
+  if (algo == MOE_ALGO_TC || pair) use_tc = true;
   else if (algo == MOE_ALGO_GEMV) use_tc = false;
   else use_tc = tc_ok && ((int64_t)M_total >= 36LL * E || !gemv_ok);  // the NF4 rule
   if (use_tc ? !tc_ok : !gemv_ok) return MOE_ERR_UNSUPPORTED;
@@ -138,7 +151,8 @@ moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* pa
   if (use_tc)
     return from_cuda(moe_launch::grouped_gemm_tc_mxfp4(A, A_rows, packed, scales, expert_offsets,
                                                        E, N, K, M_total, epilogue, out,
-                                                       out_dtype, dev_err, (cudaStream_t)stream));
+                                                       out_dtype, dev_err, (cudaStream_t)stream,
+                                                       pair));
   return from_cuda(moe_launch::grouped_gemm_mxfp4(A, A_rows, packed, scales, expert_offsets, E, N,
                                                   K, M_total, epilogue, out, out_dtype, dev_err,
                                                   (cudaStream_t)stream));
@@ -148,8 +162,10 @@ moe_status_t moe_nf4_grouped_gemm_t(const void* G, moe_dtype_t g_dtype, int G_ro
                                     const uint8_t* packed, const float* absmax,
                                     const int32_t* expert_offsets, int E, int N, int K,
                                     int M_total, void* out, moe_dtype_t out_dtype,
-                                    int32_t* dev_err, void* stream) {
+                                    moe_algo_t algo, int32_t* dev_err, void* stream) {
   if (!f32_or_f16(g_dtype) || !f32_or_f16(out_dtype)) return MOE_ERR_INVALID_ARG;
+  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC)
+    return MOE_ERR_INVALID_ARG;
   if (E < 1 || E > 1024 || N < 1 || K < 1 || K % moe::kBlock || M_total < 0 || G_rows < M_total)
     return MOE_ERR_INVALID_ARG;
   if (!expert_offsets || !packed || !absmax) return MOE_ERR_INVALID_ARG;
@@ -157,10 +173,40 @@ moe_status_t moe_nf4_grouped_gemm_t(const void* G, moe_dtype_t g_dtype, int G_ro
   const void* ptrs[] = {G, packed, absmax, expert_offsets, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  const bool tc_ok = g_dtype == MOE_DT_F16 && moe_launch::grouped_gemm_t_tc_supported(N, K);
+  if (algo == MOE_ALGO_TC && !tc_ok) return MOE_ERR_UNSUPPORTED;
+  const bool use_tc =
+      algo == MOE_ALGO_TC || (algo == MOE_ALGO_AUTO && tc_ok && (int64_t)M_total >= 36LL * E);
   if (moe_status_t st = check_device()) return st;
+  if (use_tc) {
+    if (M_total == 0) return MOE_OK;
+    return from_cuda(moe_launch::grouped_gemm_t_tc(G, G_rows, packed, absmax, expert_offsets, E,
+                                                   N, K, M_total, false, nullptr, out, out_dtype,
+                                                   dev_err, (cudaStream_t)stream));
+  }
   return from_cuda(moe_launch::grouped_gemm_t(G, g_dtype, packed, absmax, expert_offsets, E, N, K,
                                               M_total, out, out_dtype, dev_err,
                                               (cudaStream_t)stream));
+}
+
+moe_status_t moe_nf4_down_backward(const void* dYp, int G_rows, const uint8_t* packed,
+                                   const float* absmax, const int32_t* expert_offsets, int E,
+                                   int H, int I, int M_total, const float* gu, void* dgu,
+                                   moe_dtype_t dgu_dtype, int32_t* dev_err, void* stream) {
+  if (!f32_or_f16(dgu_dtype)) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 1024 || H < 1 || I < 1 || M_total < 0 || G_rows < M_total)
+    return MOE_ERR_INVALID_ARG;
+  if (!moe_launch::grouped_gemm_t_tc_supported(H, I)) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offsets || !packed || !absmax) return MOE_ERR_INVALID_ARG;
+  if (M_total > 0 && (!dYp || !gu || !dgu)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {dYp, packed, absmax, expert_offsets, gu, dgu};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (moe_status_t st = check_device()) return st;
+  if (M_total == 0) return MOE_OK;
+  return from_cuda(moe_launch::grouped_gemm_t_tc(dYp, G_rows, packed, absmax, expert_offsets, E, H,
+                                                 I, M_total, true, gu, dgu, dgu_dtype, dev_err,
+                                                 (cudaStream_t)stream));
 }
 
 moe_status_t moe_swiglu_backward(const void* gu, const void* dh, moe_dtype_t in_dtype, int M,
@@ -296,7 +342,8 @@ moe_status_t nf4_grouped_gemm_impl(const void* A, moe_dtype_t a_dtype, int A_row
   if (a_dtype != MOE_DT_BF16 && a_dtype != MOE_DT_F16) return MOE_ERR_INVALID_ARG;
   if (!valid_dtype(out_dtype)) return MOE_ERR_INVALID_ARG;
   if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
-  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC)
+  if (algo != MOE_ALGO_AUTO && algo != MOE_ALGO_GEMV && algo != MOE_ALGO_TC &&
+      algo != MOE_ALGO_TC_PAIR)
     return MOE_ERR_INVALID_ARG;
   if (E < 1 || E > 1024 || N < 1 || K < 1 || M_total < 0 || A_rows < 0 || (gather && k < 1))
     return MOE_ERR_INVALID_ARG;
@@ -312,9 +359,10 @@ moe_status_t nf4_grouped_gemm_impl(const void* A, moe_dtype_t a_dtype, int A_row
   const cudaStream_t s = (cudaStream_t)stream;
   const bool tc_ok = moe_launch::grouped_gemm_tc_supported(N, K, epilogue) && !gather &&
                      a_dtype == MOE_DT_F16;
+  const bool pair = algo == MOE_ALGO_TC_PAIR;
   bool use_tc;
-  if (algo == MOE_ALGO_TC) {
-    if (!tc_ok) return MOE_ERR_UNSUPPORTED;
+  if (algo == MOE_ALGO_TC || pair) {
+    if (!tc_ok || (pair && N % 256)) return MOE_ERR_UNSUPPORTED;
     use_tc = true;
   } else if (algo == MOE_ALGO_GEMV) {
     use_tc = false;
@@ -328,7 +376,7 @@ moe_status_t nf4_grouped_gemm_impl(const void* A, moe_dtype_t a_dtype, int A_row
   if (use_tc)
     return from_cuda(moe_launch::grouped_gemm_tc(A, a_dtype, A_rows, gather, k, packed, absmax,
                                                  expert_offsets, E, N, K, M_total, epilogue,
-                                                 out, out_dtype, dev_err, s, chain));
+                                                 out, out_dtype, dev_err, s, chain, pair));
   return from_cuda(moe_launch::grouped_gemm_gemv(A, a_dtype, A_rows, gather, k, packed, absmax,
                                                  expert_offsets, E, N, K, M_total, epilogue,
                                                  out, out_dtype, dev_err, s, chain));

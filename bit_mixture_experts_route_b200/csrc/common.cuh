@@ -151,7 +151,7 @@ __device__ __forceinline__ uint32_t mx_scale_h2(uint32_t b, bool& bad) {
 }
 
 // Weight formats of the tensor-core GEMM.
-enum WeightFormat { kFmtNF4 = 0, kFmtMXFP4 = 1 };
+enum WeightFormat { kFmtNF4 = 0, kFmtMXFP4 = 1, kFmtINT4 = 2 };
 
 // silu(g) * u with silu(g) = g / (1 + exp(-g)), IEEE division.
 __device__ __forceinline__ float swiglu_f32(float g, float u) {
@@ -336,14 +336,31 @@ cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows,
                             const int32_t* offsets, int E, int N, int K,
                             int M_total, moe_epilogue_t epi, void* out,
                             moe_dtype_t out_dt, int32_t* dev_err,
-                            cudaStream_t s, bool chain = false);
+                            cudaStream_t s, bool chain = false, bool pair = false);
 bool grouped_gemm_tc_supported(int N, int K, moe_epilogue_t epi);
+// The tensor-core kernel in its transposed form (the backward):
+// out[p, k] = sum_n W[e(p)][n, k] G[p, n], G fp16 [G_rows, N]; with
+// swiglu_bwd the result is the gradient of h and the epilogue writes the
+// gradient of the gate_up pre-activations gu (fp32 [M_total, 2K]) into out
+// [M_total, 2K].
+bool grouped_gemm_t_tc_supported(int N, int K);
+cudaError_t grouped_gemm_t_tc(const void* G, int G_rows, const uint8_t* packed,
+                              const float* absmax, const int32_t* offsets, int E, int N, int K,
+                              int M_total, bool swiglu_bwd, const float* gu, void* out,
+                              moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);
+// The same tensor-core kernel on INT4 weights (meta uint32 [E, N, K/128]:
+// fp16 scale | zero << 16); A fp16 rows in permuted order.
+cudaError_t grouped_gemm_tc_int4(const void* A, int A_rows, const uint8_t* packed,
+                                 const uint32_t* meta, const int32_t* offsets, int E, int N,
+                                 int K, int M_total, moe_epilogue_t epi, void* out,
+                                 moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);
 // The same tensor-core kernel on MXFP4 weights (scales uint8 [E, N, K/32]);
 // A fp16 rows in permuted order.
 cudaError_t grouped_gemm_tc_mxfp4(const void* A, int A_rows, const uint8_t* packed,
                                   const uint8_t* scales, const int32_t* offsets, int E, int N,
                                   int K, int M_total, moe_epilogue_t epi, void* out,
-                                  moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s);
+                                  moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s,
+                                  bool pair = false);
 cudaError_t int4_quantize(const float* W, int64_t rows, int K, uint8_t* packed, uint32_t* meta,
                           int32_t* dev_err, cudaStream_t s);
 bool grouped_gemm_int4_supported(int N, int K);

@@ -41,6 +41,20 @@
 // Every mbarrier wait is bounded; on expiry the kernel sets
 // MOE_DEVERR_TIMEOUT, every role leaves its loop, TMEM is freed and the
 // kernel returns.
+//
+// Pair form (PAIR = 2, used when N % 256 == 0): the CTAs run as clusters of
+// two on two SMs and every tile is 256 weight rows.  Each CTA decodes its
+// 128 rows into its own tensor memory and loads half of the tile's routed
+// rows (B) into its own shared memory; the leader CTA (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256, which reads A and B from both CTAs
+// and writes each CTA's 128 x N block of D into that CTA's tensor memory.
+// One MMA instruction then does twice the work of the single-CTA form, and
+// each routed-row tile crosses L2 -> SM once per 256 weight rows instead of
+// per 128.  The peer's decoders and its B loads signal the leader's `ready`
+// barriers directly (remote mbarrier arrive, and TMA with .cta_group::2);
+// the leader's commits arrive on both CTAs' barriers (.multicast::cluster);
+// the peer's epilogue hands the accumulator back with remote arrives.  No
+// TMA load uses multicast.
 #include "common.cuh"
 
 namespace moe {
@@ -49,12 +63,18 @@ namespace tc {
 constexpr int BM = 128;          // weight rows per tile (MMA M)
 constexpr int BN = 256;          // routed rows per tile (max MMA N)
 constexpr int BK = 64;           // k per stage = one NF4 block
-constexpr int BSTAGES = 3;       // activation ring
-constexpr int B_STAGE = BN * BK * 2;   // 32 KB
+constexpr int BSTAGES = 3;       // activation ring (shared memory)
 constexpr int B_BOX_ROWS = 128;        // TMA box: 64 k x 128 rows
+constexpr int B_BOX_BYTES = B_BOX_ROWS * BK * 2;  // 16 KB
+constexpr int B_STAGE = BN * BK * 2;   // 32 KB: a tile's routed rows, two boxes
+
 constexpr int RAW_RING = 8;            // packed-row ring (shared memory)
 constexpr int RING = 8;                // decoded-weight ring (tensor memory)
 constexpr int RAW_STAGE = BM * BK / 2; // 4 KB
+// transposed (backward) form: 64 weight rows x 128 columns of packed bytes
+// (4 KB) and their absmax, 4 fp32 per row (1 KB), per stage
+constexpr int RAW_STAGE_T = RAW_STAGE + 64 * 16;
+constexpr int EPI_SWIGLU_BWD = 2;       // transposed down GEMM + SwiGLU backward
 constexpr int GROUPS = 4;              // decoder groups (stages in flight)
 constexpr int DEC_WARPS = 4 * GROUPS;
 constexpr int W_BPROD = 0, W_MMA = 1, W_RPROD = 2, W_DEC = 3, W_EPI = W_DEC + DEC_WARPS;
@@ -68,7 +88,7 @@ constexpr int STG_BYTES = 32 * 32 * 4; // epilogue transpose buffer per warp
 constexpr uint32_t kWaitLimit = 1u << 20;  // suspended tries before a wait gives up
 constexpr uint32_t kSuspendNs = 1000;       // longest sleep of one try
 static_assert(A_COL + RING * A_SLOT_COLS <= TMEM_COLS, "tensor memory budget");
-static_assert(BSTAGES * B_STAGE + RAW_RING * RAW_STAGE + EPI_WARPS * STG_BYTES + 256 * 32 * 4 +
+static_assert(BSTAGES * B_STAGE + RAW_RING * RAW_STAGE_T + EPI_WARPS * STG_BYTES + 256 * 32 * 4 +
                       2 * 1025 * 4 + 1024 <
                   227 * 1024,
               "shared memory budget");
@@ -78,7 +98,7 @@ static_assert(RING % GROUPS == 0 && RAW_RING % GROUPS == 0,
 
 struct __align__(8) Smem {
   uint8_t b[BSTAGES][B_STAGE];  // 1024-aligned (struct placed at 1024)
-  uint8_t raw[RAW_RING][RAW_STAGE];
+  uint8_t raw[RAW_RING][RAW_STAGE_T];
   uint8_t stg[EPI_WARPS][STG_BYTES];
   uint32_t lut[256 * 32];
   uint64_t raw_full[RAW_RING], raw_empty[RAW_RING];
@@ -86,6 +106,7 @@ struct __align__(8) Smem {
   // activation tile (producer arrival + TMA bytes); a_empty[s]: its MMAs done
   uint64_t ready[RING], a_empty[RING];
   uint64_t acc_full, acc_empty;
+  uint64_t drain;  // pair form: the leader's MMAs all complete
   uint32_t tmem_base;
   int abort_flag;
   int ntiles_total;
@@ -137,19 +158,94 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// The same two waits with acquire at cluster scope, for barriers that the
+// other CTA of a pair arrives on.
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_suspend_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of a phase (the MMA issuer polls with it: a thread woken
+// from a suspended try_wait resumes later than one that polls).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kPollLimit = 1u << 26;  // polls before a polled wait gives up (~1 s)
+
+// Bounded polled wait (see mbar_wait), for the single MMA-issuing thread.
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, Smem& sm,
+                                          int32_t* dev_err) {
+  for (uint32_t i = 0; i < kPollLimit; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && *reinterpret_cast<volatile int*>(&sm.abort_flag)) return false;
+  }
+  *reinterpret_cast<volatile int*>(&sm.abort_flag) = 1;
+  set_dev_err(dev_err, MOE_DEVERR_TIMEOUT);
+  return false;
+}
+
 // Bounded wait: false (and the abort flag set) if the phase never completes
 // (kWaitLimit suspended tries, well under a second each way) or another role
-// already aborted.
+// already aborted.  CLUSTER: acquire at cluster scope.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem& sm,
                                           int32_t* dev_err) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (CLUSTER ? mbar_try_wait_cl(bar, parity) : mbar_try_wait(bar, parity)) return true;
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (CLUSTER ? mbar_try_wait_suspend_cl(bar, parity) : mbar_try_wait_suspend(bar, parity))
+      return true;
     if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) return false;
   }
   *reinterpret_cast<volatile int*>(&sm.abort_flag) = 1;
   set_dev_err(dev_err, MOE_DEVERR_TIMEOUT);
   return false;
+}
+
+// ---- pair form (clusters of two CTAs)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async() {
@@ -162,6 +258,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// The same load issued for the pair: the destination is this CTA's shared
+// memory, the barrier may be the other CTA's (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t cluster_bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y)
       : "memory");
 }
 
@@ -184,14 +291,29 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: D fp32, A/B fp16, both K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_f16(int n) {
-  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptor: D fp32, A/B fp16, both K-major, M = m, N = n.
+__device__ __forceinline__ uint32_t idesc_f16(int m, int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// Pair form: the leader's MMAs so far done -> one arrival on the barrier at
+// this offset in both CTAs of the pair.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_pair_local(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
       : "memory");
 }
@@ -226,15 +348,26 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// D (TMEM) += A (TMEM) * B (shared memory descriptor)
+// D (TMEM) += A (TMEM) * B (shared memory descriptor); PAIR = 2 issues the
+// two-SM form (M = 256: A and D halves in each CTA's TMEM, B halves in each
+// CTA's shared memory at the same offset).
+template <int PAIR>
 __device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if (PAIR == 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 __device__ __forceinline__ uint4 lds128(const void* p) {
@@ -279,25 +412,40 @@ __device__ __forceinline__ TileInfo tile_info(const Smem& sm, int E, int n_tiles
 // A thread's scales of one 64-k stage of its weight row as fp16 pairs for the
 // two 32-element halves: NF4 one fp32 absmax (both halves; `bad` when its
 // fp16 is subnormal or not finite), MXFP4 two E8M0 bytes (`bad` outside the
-// range where every scaled value is exact in fp16).
+// range where every scaled value is exact in fp16), INT4 the group's fp16
+// scale (both halves; `bad` when not finite) and its zero as an fp16 pair.
 template <int FMT>
-__device__ __forceinline__ void stage_scales(uint32_t sc, uint32_t& h0, uint32_t& h1, bool& bad) {
+__device__ __forceinline__ void stage_scales(uint32_t sc, uint32_t& h0, uint32_t& h1, uint32_t& zp,
+                                             bool& bad) {
   if (FMT == kFmtNF4) {
     const float a = __uint_as_float(sc);
     bad |= a != 0.0f && !(a >= 6.103515625e-05f && a <= 65504.0f);
     const __half2 ah = __float2half2_rn(a);
     h0 = h1 = *reinterpret_cast<const uint32_t*>(&ah);
-  } else {
+  } else if (FMT == kFmtMXFP4) {
     h0 = mx_scale_h2(sc & 0xFFu, bad);
     h1 = mx_scale_h2((sc >> 8) & 0xFFu, bad);
+  } else {
+    bad |= (sc & 0x7C00u) == 0x7C00u;
+    h0 = h1 = (sc & 0xFFFFu) * 0x00010001u;
+    const __half z = __uint2half_rn((sc >> 16) & 15u);
+    zp = (uint32_t)(*reinterpret_cast<const uint16_t*>(&z)) * 0x00010001u;
   }
 }
 
-template <int FMT, int EPI, typename OutT>
+// TR = false: out[p, n] = sum_k W[e(p)][n, k] A[p, k] (the forward grouped
+// GEMM; tiles of output rows n = weight rows).  TR = true: the transposed
+// GEMM of the backward, out[p, k] = sum_n W[e(p)][n, k] A[p, n] (tiles of
+// output columns k; A = the upstream gradient), NF4 only, single CTA; with
+// EPI_SWIGLU_BWD its epilogue applies the SwiGLU backward to the result (the
+// gradient of h) and writes the gradient of gate_up's pre-activations.
+template <int FMT, int EPI, typename OutT, int PAIR, bool TR>
 __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
-    const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
+    const __grid_constant__ CUtensorMap bmap,
+    const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
     const void* __restrict__ scales, const int32_t* __restrict__ offsets, int E, int N, int K,
-    int M_total, OutT* __restrict__ out, int32_t* dev_err, int chain) {
+    int M_total, OutT* __restrict__ out, const float* __restrict__ gu, int32_t* dev_err,
+    int chain) {
   extern __shared__ uint8_t smem_raw[];
   if (!chain) {  // nothing is read or written before the previous kernel is done
     pdl_wait();
@@ -306,23 +454,33 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = N / BM;
-  const int KT = K / BK;
+  // tiles of BM * PAIR output rows (weight rows; transposed: weight
+  // columns); this CTA's 128-row part of tile ntile is sub-tile
+  // ntile * PAIR + rank.  KT stages of BK along the reduction.
+  const int n_tiles = (TR ? K : N) / (BM * PAIR);
+  const int KT = (TR ? N : K) / BK;
+  const int rank = PAIR == 1 ? 0 : (int)cluster_rank();
+  const bool leader = rank == 0;
+  const int t0 = blockIdx.x / PAIR, tstep = gridDim.x / PAIR;  // this pair's tiles
+
+  // MMA N for a tile's routed rows: a multiple of 16 (one CTA) or of 32 (the
+  // pair's M = 256 form, each CTA holding N / 2 rows of B)
+  auto mma_n = [](int rows) { return PAIR == 1 ? (rows + 15) & ~15 : (rows + 31) & ~31; };
 
   // ---- setup: barriers, offsets, decode table, tile list, TMEM
   if (threadIdx.x == 0) {
-    for (int s = 0; s < BSTAGES; ++s) {
-    }
     for (int s = 0; s < RAW_RING; ++s) {
       mbar_init(&sm.raw_full[s], 1);
       mbar_init(&sm.raw_empty[s], 4);   // the four warps of the decoding group
     }
     for (int s = 0; s < RING; ++s) {
-      mbar_init(&sm.ready[s], 4 + 1);
+      // the decoder warps of every CTA of the pair + the (leader's) B producer
+      mbar_init(&sm.ready[s], 4 * PAIR + 1);
       mbar_init(&sm.a_empty[s], 1);     // MMA completion (tcgen05.commit)
     }
     mbar_init(&sm.acc_full, 1);
-    mbar_init(&sm.acc_empty, 32 * EPI_WARPS);
+    mbar_init(&sm.acc_empty, 32 * EPI_WARPS * PAIR);
+    mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -335,15 +493,26 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       const __half2 h = __halves2half2(__float2half_rn(c_levels_tc[b >> 4]),
                                        __float2half_rn(c_levels_tc[b & 15]));
       sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
-    } else {
+    } else if (FMT == kFmtMXFP4) {
       sm.lut[i] = e2m1_h((uint32_t)b & 15u) | (e2m1_h((uint32_t)b >> 4) << 16);
+    } else {  // INT4: the codes as exact fp16 integers {q(high nibble), q(low)}
+      const __half2 h = __halves2half2(__uint2half_rn((unsigned)(b >> 4)),
+                                       __uint2half_rn((unsigned)(b & 15)));
+      sm.lut[i] = *reinterpret_cast<const uint32_t*>(&h);
     }
   }
   if (warp == W_MMA) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&sm.tmem_base)),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if (PAIR == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&sm.tmem_base)),
+                   "r"(TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    } else {  // same warp, same destination in both CTAs of the pair
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&sm.tmem_base)),
+                   "r"(TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
   }
   __syncthreads();
   if (warp == W_BPROD) {
@@ -376,6 +545,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync();  // both CTAs' barriers and TMEM exist
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
   const int total = sm.ntiles_total;
@@ -389,62 +559,86 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         pdl_wait();
         pdl_trigger();
       }
-      // slot S mod BSTAGES is free once the MMAs of stage S - BSTAGES are
-      // done; their completion is the a_empty barrier of that stage's TMEM
-      // slot (one commit per stage serves both rings)
+      // Activation slot S mod BSTAGES is free once the MMAs of stage
+      // S - BSTAGES are done: the a_empty barrier of that stage's TMEM slot
+      // (one commit per stage serves both rings).  A stage is the tile's
+      // routed rows in whole 128-row boxes (rows past the tile are loaded and
+      // never read).  Pair form: each CTA loads its half of the routed rows
+      // into its own slot; both halves are counted on the leader's ready
+      // barrier.
       int bs = 0, S = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = t0; t < total && ok; t += tstep) {
         const TileInfo ti = tile_info(sm, E, n_tiles, t);
-        const int nmma = (ti.nrows + 15) & ~15;
-        const int boxes = (nmma + B_BOX_ROWS - 1) / B_BOX_ROWS;
+        const int rows_b = mma_n(ti.nrows) / PAIR;
+        const int boxes = (rows_b + B_BOX_ROWS - 1) / B_BOX_ROWS;
+        const int brow0 = ti.row0 + rank * rows_b;
         for (int ks = 0; ks < KT; ++ks, ++S) {
           if (S >= BSTAGES) {
             const int P = S - BSTAGES;
-            if (!(ok = mbar_wait(&sm.a_empty[P % RING], (uint32_t)(P / RING) & 1u, sm, dev_err)))
+            if (!(ok = mbar_wait<PAIR == 2>(&sm.a_empty[P % RING], (uint32_t)(P / RING) & 1u, sm,
+                                            dev_err)))
               break;
           }
           uint64_t* rdy = &sm.ready[S % RING];
-          mbar_arrive_expect_tx(rdy, boxes * B_BOX_ROWS * BK * 2);
-          for (int b = 0; b < boxes; ++b)
-            tma_load_2d(sm.b[bs] + b * (B_BOX_ROWS * BK * 2), &bmap, rdy, ks * BK,
-                        ti.row0 + b * B_BOX_ROWS);
+          // leader: its own barrier; the pair's peer: the leader's
+          const uint32_t bar = leader ? smem_u32(rdy) : cluster_addr(rdy, 0);
+          if (leader) mbar_arrive_expect_tx(rdy, PAIR * boxes * B_BOX_BYTES);
+          for (int b = 0; b < boxes; ++b) {
+            if (PAIR == 1)
+              tma_load_2d(sm.b[bs] + b * B_BOX_BYTES, &bmap, rdy, ks * BK,
+                          brow0 + b * B_BOX_ROWS);
+            else
+              tma_load_2d_pair(sm.b[bs] + b * B_BOX_BYTES, &bmap, bar, ks * BK,
+                               brow0 + b * B_BOX_ROWS);
+          }
           if (++bs == BSTAGES) bs = 0;
         }
       }
     }
   } else if (warp == W_MMA) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
+    // ---------------- MMA issuer (the leader CTA's, in the pair form)
+    if (lane == 0 && leader) {
       const uint64_t bdesc0 = sw128_desc(smem_u32(sm.b[0]));
-      int bs = 0, as = 0;
+      int bs = 0, as = 0;  // activation slot (as the producer's), TMEM slot
       uint32_t aph = 0;
       bool ok = true;
       int lt = 0;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+      for (int t = t0; t < total && ok; t += tstep, ++lt) {
         const TileInfo ti = tile_info(sm, E, n_tiles, t);
-        const int nmma = (ti.nrows + 15) & ~15;
-        // the single accumulator must have been drained by the epilogue
-        if (!(ok = mbar_wait(&sm.acc_empty, (lt & 1) ^ 1, sm, dev_err))) break;
+        const int nmma = mma_n(ti.nrows);
+        // the single accumulator must have been drained by the epilogue(s)
+        if (!(ok = mbar_poll(&sm.acc_empty, (lt & 1) ^ 1, sm, dev_err))) break;
         tc_fence_after();
-        const uint32_t idesc = idesc_f16(nmma);
+        const uint32_t idesc = idesc_f16(BM * PAIR, nmma);
         const uint32_t dcol = tmem_base + ACC_COL;
         for (int ks = 0; ks < KT; ++ks) {
-          if (!(ok = mbar_wait(&sm.ready[as], aph, sm, dev_err))) break;
+          if (!(ok = mbar_poll(&sm.ready[as], aph, sm, dev_err))) break;
           tc_fence_after();
           // K slice kk: 8 more TMEM columns of A; 32 bytes further into the
           // swizzled activation rows (+2 in the descriptor's address field)
           const uint32_t acol = tmem_base + A_COL + as * A_SLOT_COLS;
-          const uint64_t bd = bdesc0 + (uint64_t)(bs * (B_STAGE >> 4));
-          mma_ts(dcol, acol, bd, idesc, ks != 0);
-          mma_ts(dcol, acol + 8, bd + 2, idesc, 1u);
-          mma_ts(dcol, acol + 16, bd + 4, idesc, 1u);
-          mma_ts(dcol, acol + 24, bd + 6, idesc, 1u);
-          mma_commit(&sm.a_empty[as]);  // frees TMEM slot as and activation slot bs
+          const uint64_t bd = bdesc0 + (uint64_t)((bs * B_STAGE) >> 4);
+          mma_ts<PAIR>(dcol, acol, bd, idesc, ks != 0);
+          mma_ts<PAIR>(dcol, acol + 8, bd + 2, idesc, 1u);
+          mma_ts<PAIR>(dcol, acol + 16, bd + 4, idesc, 1u);
+          mma_ts<PAIR>(dcol, acol + 24, bd + 6, idesc, 1u);
+          // frees TMEM slot as and the stage's activation bytes (in both CTAs)
+          if (PAIR == 1) mma_commit(&sm.a_empty[as]); else mma_commit_pair(&sm.a_empty[as]);
           if (++bs == BSTAGES) bs = 0;
           if (++as == RING) { as = 0; aph ^= 1; }
         }
-        if (ok) mma_commit(&sm.acc_full);
+        if (ok) {
+          if (PAIR == 1) mma_commit(&sm.acc_full); else mma_commit_pair(&sm.acc_full);
+        }
+      }
+      if (PAIR == 2) {
+        // every MMA this thread issued has finished reading both CTAs'
+        // shared and tensor memory before either CTA leaves
+        // (bounded, and not cut short by an abort of another role)
+        mma_commit_pair_local(&sm.drain);
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait_suspend_cl(&sm.drain, 0); ++i) {
+        }
       }
     }
   } else if (warp == W_RPROD) {
@@ -453,21 +647,33 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       int rs = 0;
       uint32_t rph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = t0; t < total && ok; t += tstep) {
         const TileId id = tile_id(sm, E, n_tiles, t);
+        const int wt = id.ntile * PAIR + rank;  // this CTA's 128-row weight sub-tile
         int y0, y1;  // first weight row of each 64-row box
         if (EPI == MOE_EPI_SWIGLU) {
-          y0 = id.expert * N + id.ntile * (BM / 2);  // gate rows
-          y1 = y0 + N / 2;                           // matching up rows
+          y0 = id.expert * N + wt * (BM / 2);  // gate rows
+          y1 = y0 + N / 2;                     // matching up rows
         } else {
-          y0 = id.expert * N + id.ntile * BM;
+          y0 = id.expert * N + wt * BM;
           y1 = y0 + BM / 2;
         }
         for (int ks = 0; ks < KT; ++ks) {
           if (!(ok = mbar_wait(&sm.raw_empty[rs], rph ^ 1, sm, dev_err))) break;
-          mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE);
-          tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], ks * (BK / 2), y0);
-          tma_load_2d(sm.raw[rs] + (BM / 2) * (BK / 2), &wmap, &sm.raw_full[rs], ks * (BK / 2), y1);
+          if (TR) {
+            // weight rows n = 64 ks .. 64 ks + 63 of the expert, the packed
+            // bytes of columns 128 wt .. 128 wt + 127, and the absmax of their
+            // two 64-blocks (4 per row from a 16-byte-aligned block index)
+            const int yr = id.expert * N + ks * BK;
+            mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE_T);
+            tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], wt * (BM / 2), yr);
+            tma_load_2d(sm.raw[rs] + RAW_STAGE, &amap, &sm.raw_full[rs], (2 * wt) & ~3, yr);
+          } else {
+            mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE);
+            tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], ks * (BK / 2), y0);
+            tma_load_2d(sm.raw[rs] + (BM / 2) * (BK / 2), &wmap, &sm.raw_full[rs],
+                        ks * (BK / 2), y1);
+          }
           if (++rs == RAW_RING) { rs = 0; rph ^= 1; }
         }
       }
@@ -483,6 +689,60 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     const int rrow = (EPI == MOE_EPI_SWIGLU) ? ((m & 1) ? BM / 2 + (m >> 1) : (m >> 1)) : m;
     const uint32_t* lut = sm.lut + lane;
     const uint32_t tlane = tmem_base + ((uint32_t)(32 * q) << 16);
+    if constexpr (TR) {
+      // Transposed form: this thread's TMEM lane is output column
+      // k = 128 wt + m; a stage's 32 columns of fp16 pairs are its weights in
+      // rows n = 64 ks + 2c, 2c + 1, decoded from the byte of column k in each
+      // row (high nibble for even k) through the byte table, times each row's
+      // absmax of k's 64-block (fp16 products, as in the forward form).
+      const uint32_t* lutl = sm.lut + lane;
+      const int byte = m >> 1;
+      // a table entry is {L[high nibble] (low half), L[low nibble] (high
+      // half)}; even k takes the low halves of rows n and n + 1, odd k the
+      // high halves
+      const uint32_t sel = (m & 1) ? 0x7632u : 0x5410u;
+      bool bad_scale = false;
+      for (int S = g; ; S += GROUPS) {
+        const int lt_ = S / KT, ks = S - lt_ * KT;
+        const int t = t0 + lt_ * tstep;
+        if (t >= total) break;
+        const TileId id = tile_id(sm, E, n_tiles, t);
+        const int si = ((2 * id.ntile) & 3) + (m >> 6);  // absmax word of k's block
+        const int slot = S % RING, rslot = S % RAW_RING;
+        const uint32_t ph = (uint32_t)(S / RING) & 1u, rph = (uint32_t)(S / RAW_RING) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[rslot], rph, sm, dev_err))) break;
+        const uint8_t* rp = sm.raw[rslot];
+        const float* sc = reinterpret_cast<const float*>(rp + RAW_STAGE);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.a_empty[slot], ph ^ 1, sm, dev_err))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t hv[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int n = 32 * half + 2 * c;
+            const uint32_t p0 = lutl[(uint32_t)rp[n * 64 + byte] << 5];
+            const uint32_t p1 = lutl[(uint32_t)rp[(n + 1) * 64 + byte] << 5];
+            const float a0 = sc[n * 4 + si], a1 = sc[(n + 1) * 4 + si];
+            bad_scale |= (a0 != 0.0f && !(a0 >= 6.103515625e-05f && a0 <= 65504.0f)) ||
+                         (a1 != 0.0f && !(a1 >= 6.103515625e-05f && a1 <= 65504.0f));
+            const uint32_t lv = __byte_perm(p0, p1, sel);  // {L(row n), L(row n + 1)}
+            const __half2 ah = __floats2half2_rn(a0, a1);
+            const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&lv), ah);
+            hv[c] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          tmem_st16(tlane + A_COL + slot * A_SLOT_COLS + 16 * half, hv);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sm.ready[slot]);
+          mbar_arrive(&sm.raw_empty[rslot]);
+        }
+      }
+      if (__any_sync(0xffffffffu, bad_scale) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
+    } else {
     // scales of this thread's weight row in tile t (null past the CTA's last
     // tile), stage ks at word ks: NF4 the fp32 absmax of block ks, MXFP4 the
     // two E8M0 bytes of the stage; walked one own stage ahead without
@@ -490,23 +750,26 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     auto row_scales = [&](int t) -> const uint8_t* {
       if (t >= total) return nullptr;
       const TileId id = tile_id(sm, E, n_tiles, t);
+      const int wt = id.ntile * PAIR + rank;
       int row;
       if (EPI == MOE_EPI_SWIGLU) {
-        const int j = id.ntile * (BM / 2) + (m >> 1);
+        const int j = wt * (BM / 2) + (m >> 1);
         row = (m & 1) ? (N / 2 + j) : j;
       } else {
-        row = id.ntile * BM + m;
+        row = wt * BM + m;
       }
       const size_t r = (size_t)id.expert * N + row;
       return reinterpret_cast<const uint8_t*>(scales) +
-             (FMT == kFmtNF4 ? r * (size_t)KT * 4 : r * (size_t)(K / 32));
+             (FMT == kFmtNF4 ? r * (size_t)KT * 4
+              : FMT == kFmtMXFP4 ? r * (size_t)(K / 32) : r * (size_t)(K / 128) * 4);
     };
     auto fetch = [&](const uint8_t* row, int ks) -> uint32_t {
       if (FMT == kFmtNF4) return __ldg(reinterpret_cast<const uint32_t*>(row) + ks);
-      return __ldg(reinterpret_cast<const uint16_t*>(row) + ks);
+      if (FMT == kFmtMXFP4) return __ldg(reinterpret_cast<const uint16_t*>(row) + ks);
+      return __ldg(reinterpret_cast<const uint32_t*>(row) + (ks >> 1));  // 128-k group
     };
-    int n_ks = g, n_t = blockIdx.x;
-    while (n_ks >= KT) { n_ks -= KT; n_t += gridDim.x; }
+    int n_ks = g, n_t = t0;
+    while (n_ks >= KT) { n_ks -= KT; n_t += tstep; }
     const uint8_t* n_row = row_scales(n_t);
     uint32_t sc_cur = n_row ? fetch(n_row, n_ks) : 0u;
     bool have = n_row != nullptr;
@@ -517,7 +780,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       n_ks += GROUPS;
       while (n_ks >= KT && n_row) {
         n_ks -= KT;
-        n_t += gridDim.x;
+        n_t += tstep;
         n_row = row_scales(n_t);
       }
       const bool have_next = n_row != nullptr;
@@ -526,9 +789,10 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[rslot], rph, sm, dev_err))) break;
       const uint8_t* rp = sm.raw[rslot] + rrow * (BK / 2);
       const uint4 w0 = lds128(rp), w1 = lds128(rp + 16);
-      uint32_t sh[2];
-      stage_scales<FMT>(sc_cur, sh[0], sh[1], bad_scale);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.a_empty[slot], ph ^ 1, sm, dev_err))) break;
+      uint32_t sh[2], zp = 0;
+      stage_scales<FMT>(sc_cur, sh[0], sh[1], zp, bad_scale);
+      if (!__all_sync(0xffffffffu, mbar_wait<PAIR == 2>(&sm.a_empty[slot], ph ^ 1, sm, dev_err)))
+        break;
       tc_fence_after();
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
@@ -541,7 +805,9 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
             const uint32_t raw = lut[__byte_perm(w, 0, 0x4440u | b) << 5];
-            __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&raw), ah);
+            __half2 lv = *reinterpret_cast<const __half2*>(&raw);
+            if (FMT == kFmtINT4) lv = __hsub2(lv, *reinterpret_cast<const __half2*>(&zp));
+            __half2 v = __hmul2(lv, ah);
             hv[4 * c + b] = *reinterpret_cast<uint32_t*>(&v);
           }
         }
@@ -551,7 +817,9 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sm.ready[slot]);
+        // the slot is ready on the MMA-issuing CTA's barrier
+        if (leader) mbar_arrive(&sm.ready[slot]);
+        else mbar_arrive_remote(cluster_addr(&sm.ready[slot], 0));
         mbar_arrive(&sm.raw_empty[rslot]);  // its bytes are decoded
       }
       sc_cur = sc_next;
@@ -559,6 +827,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     }
     // the loop exits are warp-uniform, so every lane takes part
     if (__any_sync(0xffffffffu, bad_scale) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
+    }
   } else {
     // ---------------- epilogue: warp (q, hc) reads TMEM lanes 32q .. 32q+31,
     // columns of half hc of each 64-column block (two warps per lane quarter)
@@ -574,14 +843,40 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     bool ok = true;
     bool ovf = false;  // an fp16 output that overflowed
     int lt = 0;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+    // the accumulator goes back to the MMA-issuing CTA
+    auto release_acc = [&]() {
+      tc_fence_before();
+      if (leader) mbar_arrive(&sm.acc_empty);
+      else mbar_arrive_remote(cluster_addr(&sm.acc_empty, 0));
+    };
+    for (int t = t0; t < total && ok; t += tstep, ++lt) {
       const TileInfo ti = tile_info(sm, E, n_tiles, t);
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full, lt & 1, sm, dev_err)))) break;
+      if (!(ok = __all_sync(0xffffffffu,
+                            mbar_wait<PAIR == 2>(&sm.acc_full, lt & 1, sm, dev_err))))
+        break;
       tc_fence_after();
-      const int ncols = (ti.nrows + 15) & ~15;
+      const int ncols = mma_n(ti.nrows);
       // first output column of this warp's rows
-      const int col0 = (EPI == MOE_EPI_SWIGLU) ? ti.ntile * (BM / 2) + 16 * q : ti.ntile * BM + 32 * q;
-      const int ldo = (EPI == MOE_EPI_SWIGLU) ? N / 2 : N;
+      const int wt = ti.ntile * PAIR + rank;
+      const int col0 = (EPI == MOE_EPI_SWIGLU) ? wt * (BM / 2) + 16 * q : wt * BM + 32 * q;
+      // row pitch of out: SwiGLU N/2; transposed K, or 2K with the SwiGLU
+      // backward (gate gradients at col, up gradients at K + col)
+      const int ldo = (EPI == MOE_EPI_SWIGLU) ? N / 2
+                      : TR ? (EPI == EPI_SWIGLU_BWD ? 2 * K : K) : N;
+      // staged rows -> global, 16 bytes per lane, at column offset cofs
+      auto store_staged = [&](int c0, int cofs) {
+        __syncwarp();
+#pragma unroll
+        for (int idx = lane; idx < 32 * V; idx += 32) {
+          const int tok = idx / V, piece = idx - tok * V;
+          if (c0 + tok < ti.nrows) {
+            const uint4 val = lds128(stg + tok * ROWB + piece * 16);
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(
+                out + (size_t)(ti.row0 + c0 + tok) * ldo + cofs) + piece * 16) = val;
+          }
+        }
+        __syncwarp();
+      };
       bool released = false;
       for (int c0 = 32 * hc; c0 < ncols; c0 += 64) {
         uint32_t v[32];
@@ -589,8 +884,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         if (c0 + 64 >= ncols) {
           // this warp's last read of the accumulator: hand it back to the
           // MMA before the math and the stores
-          tc_fence_before();
-          mbar_arrive(&sm.acc_empty);
+          release_acc();
           released = true;
         }
         if (EPI == MOE_EPI_SWIGLU) {
@@ -611,6 +905,30 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
             ovf |= c0 + tok < ti.nrows && overflows_out<OutT>(h);
             reinterpret_cast<OutT*>(stg + tok * ROWB)[p] = from_f32<OutT>(h);
           }
+        } else if (EPI == EPI_SWIGLU_BWD) {
+          // v[i] = dh of token c0 + i at column col0 + lane; with s =
+          // sigmoid(g): d gate = dh u s (1 + g (1 - s)), d up = dh g s, from
+          // the forward's pre-activations gu [M, 2K] (fp32)
+          float du[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const bool live = c0 + i < ti.nrows;
+            const size_t gp = (size_t)(ti.row0 + c0 + i) * (2 * (size_t)K) + col0 + lane;
+            const float gv = live ? __ldg(gu + gp) : 0.0f;
+            const float uv = live ? __ldg(gu + gp + K) : 0.0f;
+            const float sg = __fdiv_rn(1.0f, 1.0f + expf(-gv));
+            const float dh = __uint_as_float(v[i]);
+            const float dgate = dh * uv * sg * (1.0f + gv * (1.0f - sg));
+            du[i] = dh * gv * sg;
+            ovf |= live && (overflows_out<OutT>(dgate) || overflows_out<OutT>(du[i]));
+            reinterpret_cast<OutT*>(stg + i * ROWB)[lane] = from_f32<OutT>(dgate);
+          }
+          store_staged(c0, col0);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            reinterpret_cast<OutT*>(stg + i * ROWB)[lane] = from_f32<OutT>(du[i]);
+          store_staged(c0, K + col0);
+          continue;
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -619,43 +937,70 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
             reinterpret_cast<OutT*>(stg + i * ROWB)[lane] = from_f32<OutT>(y);
           }
         }
-        __syncwarp();
-        // staged rows -> global, 16 bytes per lane
-#pragma unroll
-        for (int idx = lane; idx < 32 * V; idx += 32) {
-          const int tok = idx / V, piece = idx - tok * V;
-          if (c0 + tok < ti.nrows) {
-            const uint4 val = lds128(stg + tok * ROWB + piece * 16);
-            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(
-                out + (size_t)(ti.row0 + c0 + tok) * ldo + col0) + piece * 16) = val;
-          }
-        }
-        __syncwarp();
+        store_staged(c0, col0);
       }
-      if (!released) {  // no columns for this warp in this tile
-        tc_fence_before();
-        mbar_arrive(&sm.acc_empty);
-      }
+      if (!released) release_acc();  // no columns for this warp in this tile
     }
     // the loop exits are warp-uniform, so every lane takes part
     if (__any_sync(0xffffffffu, ovf) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
   }
 
   // single-lane roles (producers, MMA issuer) rejoin their warp before the
-  // CTA-wide barrier
+  // CTA-wide barrier; in the pair form neither CTA frees its tensor memory or
+  // leaves (its shared memory holds barriers the other CTA arrives on) before
+  // both are done
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync();
   if (warp == W_MMA) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(TMEM_COLS));
+    if (PAIR == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(TMEM_COLS));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(TMEM_COLS));
   }
 }
 
 int sm_count() { return device_sm_count(); }
 
-template <int FMT, int EPI, typename OutT>
+// Clusters of two of `kern` that fit on the device at once, once per kernel
+// and device (the GPCs' SM counts decide it); SMs / 2 if the query fails.
+inline int max_pair_clusters(const void* kern, size_t smem) {
+  static std::mutex mu;
+  static std::unordered_map<uint64_t, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return std::max(1, sm_count() / 2);
+  const uint64_t key = (reinterpret_cast<uint64_t>(kern) << 6) ^ (uint64_t)dev;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * std::max(1, sm_count() / 2));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = std::max(1, sm_count() / 2);
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = n;
+  return n;
+}
+
+template <int FMT, int EPI, typename OutT, int PAIR>
 cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
                    const int32_t* offsets, int E, int N, int K, int M_total, void* out,
                    int32_t* dev_err, cudaStream_t s, bool chain) {
@@ -667,8 +1012,8 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M_total};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
     const cuuint32_t box[2] = {BK, B_BOX_ROWS};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -685,40 +1030,131 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
       return cudaErrorInvalidValue;
   }
   const size_t smem = sizeof(Smem) + 1024;
-  auto kern = nf4_tc_kernel<FMT, EPI, OutT>;
+  auto kern = nf4_tc_kernel<FMT, EPI, OutT, PAIR, false>;
   cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
   // Upper bound on tiles: every expert's rows rounded up to BN, plus one
   // partial tile per expert; the kernel derives the exact list itself.
-  const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / BM);
+  const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / (BM * PAIR));
+  if (PAIR == 1) {
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
+    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, wmap, wmap, scales,
+                      offsets, E, N, K, M_total, reinterpret_cast<OutT*>(out),
+                      static_cast<const float*>(nullptr), dev_err, chain ? 1 : 0);
+  }
+  const int clusters = (int)std::max<int64_t>(
+      1, std::min<int64_t>(max_pair_clusters(reinterpret_cast<const void*>(kern), smem),
+                           max_tiles));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, map, wmap, wmap, scales, offsets, E, N, K, M_total,
+                            reinterpret_cast<OutT*>(out), static_cast<const float*>(nullptr),
+                            dev_err, chain ? 1 : 0);
+}
+
+// The transposed (backward) form: out[p, k] = sum_n W[e(p)][n, k] G[p, n],
+// G fp16 [G_rows, N] in permuted order; EPI_SWIGLU_BWD applies the SwiGLU
+// backward with gu fp32 [M_total, 2K] and writes out [M_total, 2K].
+template <int EPI, typename OutT>
+cudaError_t launch_t(const void* G, int G_rows, const uint8_t* packed, const float* absmax,
+                     const int32_t* offsets, int E, int N, int K, int M_total, void* out,
+                     const float* gu, int32_t* dev_err, cudaStream_t s) {
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  const auto enc = encode_tiled_cached;
+  CUtensorMap map, wmap, amap;
+  const cuuint32_t estr[2] = {1, 1};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    const cuuint32_t box[2] = {BK, B_BOX_ROWS};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(G),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // packed rows [E*N, K/2]; box = 64 bytes (128 columns) x 64 rows
+    const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)E * N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t box[2] = {BM / 2, BK};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // absmax [E*N, K/64]; box = 4 blocks x 64 rows
+    const cuuint64_t dims[2] = {(cuuint64_t)K / kBlock, (cuuint64_t)E * N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K / kBlock * 4};
+    const cuuint32_t box[2] = {4, BK};
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(absmax), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const size_t smem = sizeof(Smem) + 1024;
+  auto kern = nf4_tc_kernel<kFmtNF4, EPI, OutT, 1, true>;
+  cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
+  if (err != cudaSuccess) return err;
+  const int64_t max_tiles = ((int64_t)M_total / BN + E) * (K / BM);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, wmap, scales, offsets, E, N, K,
-                    M_total, reinterpret_cast<OutT*>(out), dev_err, chain ? 1 : 0);
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, wmap, amap,
+                    static_cast<const void*>(absmax), offsets, E, N, K, M_total,
+                    reinterpret_cast<OutT*>(out), gu, dev_err, 0);
+}
+
+template <int FMT, int EPI, typename OutT>
+cudaError_t launch_pair_or_not(const void* A, const uint8_t* packed, const void* scales,
+                               const int32_t* offsets, int E, int N, int K, int M_total,
+                               void* out, int32_t* dev_err, cudaStream_t s, bool chain,
+                               bool pair) {
+  // the pair form needs whole 256-row weight tiles
+  if (pair && N % (2 * BM) == 0)
+    return launch<FMT, EPI, OutT, 2>(A, packed, scales, offsets, E, N, K, M_total, out, dev_err,
+                                     s, chain);
+  return launch<FMT, EPI, OutT, 1>(A, packed, scales, offsets, E, N, K, M_total, out, dev_err, s,
+                                   chain);
 }
 
 template <int FMT>
 cudaError_t launch_fmt(const void* A, const uint8_t* packed, const void* scales,
                        const int32_t* offsets, int E, int N, int K, int M_total,
                        moe_epilogue_t epi, void* out, moe_dtype_t out_dt, int32_t* dev_err,
-                       cudaStream_t s, bool chain) {
+                       cudaStream_t s, bool chain, bool pair) {
   if (epi == MOE_EPI_SWIGLU) {
     if (out_dt == MOE_DT_F16)
-      return launch<FMT, MOE_EPI_SWIGLU, __half>(A, packed, scales, offsets, E, N, K, M_total,
-                                                 out, dev_err, s, chain);
+      return launch_pair_or_not<FMT, MOE_EPI_SWIGLU, __half>(A, packed, scales, offsets, E, N, K,
+                                                             M_total, out, dev_err, s, chain, pair);
     if (out_dt == MOE_DT_BF16)
-      return launch<FMT, MOE_EPI_SWIGLU, __nv_bfloat16>(A, packed, scales, offsets, E, N, K,
-                                                        M_total, out, dev_err, s, chain);
-    return launch<FMT, MOE_EPI_SWIGLU, float>(A, packed, scales, offsets, E, N, K, M_total, out,
-                                              dev_err, s, chain);
+      return launch_pair_or_not<FMT, MOE_EPI_SWIGLU, __nv_bfloat16>(
+          A, packed, scales, offsets, E, N, K, M_total, out, dev_err, s, chain, pair);
+    return launch_pair_or_not<FMT, MOE_EPI_SWIGLU, float>(A, packed, scales, offsets, E, N, K,
+                                                          M_total, out, dev_err, s, chain, pair);
   }
   if (out_dt == MOE_DT_F16)
-    return launch<FMT, MOE_EPI_NONE, __half>(A, packed, scales, offsets, E, N, K, M_total, out,
-                                             dev_err, s, chain);
+    return launch_pair_or_not<FMT, MOE_EPI_NONE, __half>(A, packed, scales, offsets, E, N, K,
+                                                         M_total, out, dev_err, s, chain, pair);
   if (out_dt == MOE_DT_BF16)
-    return launch<FMT, MOE_EPI_NONE, __nv_bfloat16>(A, packed, scales, offsets, E, N, K,
-                                                    M_total, out, dev_err, s, chain);
-  return launch<FMT, MOE_EPI_NONE, float>(A, packed, scales, offsets, E, N, K, M_total, out,
-                                          dev_err, s, chain);
+    return launch_pair_or_not<FMT, MOE_EPI_NONE, __nv_bfloat16>(A, packed, scales, offsets, E, N,
+                                                                K, M_total, out, dev_err, s,
+                                                                chain, pair);
+  return launch_pair_or_not<FMT, MOE_EPI_NONE, float>(A, packed, scales, offsets, E, N, K,
+                                                      M_total, out, dev_err, s, chain, pair);
 }
 
 }  // namespace tc
@@ -735,20 +1171,56 @@ cudaError_t grouped_gemm_tc(const void* A, moe_dtype_t a_dt, int A_rows, const i
                             int k, const uint8_t* packed, const float* absmax,
                             const int32_t* offsets, int E, int N, int K, int M_total,
                             moe_epilogue_t epi, void* out, moe_dtype_t out_dt, int32_t* dev_err,
-                            cudaStream_t s, bool chain) {
+                            cudaStream_t s, bool chain, bool pair) {
   (void)k;
   if (gather || a_dt != MOE_DT_F16 || A_rows < M_total) return cudaErrorNotSupported;
   return moe::tc::launch_fmt<moe::kFmtNF4>(A, packed, absmax, offsets, E, N, K, M_total, epi,
-                                           out, out_dt, dev_err, s, chain);
+                                           out, out_dt, dev_err, s, chain, pair);
+}
+
+bool grouped_gemm_t_tc_supported(int N, int K) {
+  // 128-column output tiles, 64-row reduction stages, and an absmax row
+  // pitch that is a multiple of 16 bytes (the TMA stride rule)
+  return N % moe::tc::BK == 0 && N >= moe::tc::BK && K % 256 == 0;
+}
+
+cudaError_t grouped_gemm_t_tc(const void* G, int G_rows, const uint8_t* packed,
+                              const float* absmax, const int32_t* offsets, int E, int N, int K,
+                              int M_total, bool swiglu_bwd, const float* gu, void* out,
+                              moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s) {
+  using namespace moe::tc;
+  if (G_rows < M_total) return cudaErrorNotSupported;
+  if (swiglu_bwd) {
+    if (out_dt == MOE_DT_F16)
+      return launch_t<EPI_SWIGLU_BWD, __half>(G, G_rows, packed, absmax, offsets, E, N, K,
+                                              M_total, out, gu, dev_err, s);
+    return launch_t<EPI_SWIGLU_BWD, float>(G, G_rows, packed, absmax, offsets, E, N, K, M_total,
+                                           out, gu, dev_err, s);
+  }
+  if (out_dt == MOE_DT_F16)
+    return launch_t<MOE_EPI_NONE, __half>(G, G_rows, packed, absmax, offsets, E, N, K, M_total,
+                                          out, nullptr, dev_err, s);
+  return launch_t<MOE_EPI_NONE, float>(G, G_rows, packed, absmax, offsets, E, N, K, M_total, out,
+                                       nullptr, dev_err, s);
+}
+
+cudaError_t grouped_gemm_tc_int4(const void* A, int A_rows, const uint8_t* packed,
+                                 const uint32_t* meta, const int32_t* offsets, int E, int N,
+                                 int K, int M_total, moe_epilogue_t epi, void* out,
+                                 moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s) {
+  if (A_rows < M_total) return cudaErrorNotSupported;
+  return moe::tc::launch_fmt<moe::kFmtINT4>(A, packed, meta, offsets, E, N, K, M_total, epi, out,
+                                            out_dt, dev_err, s, false, false);
 }
 
 cudaError_t grouped_gemm_tc_mxfp4(const void* A, int A_rows, const uint8_t* packed,
                                   const uint8_t* scales, const int32_t* offsets, int E, int N,
                                   int K, int M_total, moe_epilogue_t epi, void* out,
-                                  moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s) {
+                                  moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s,
+                                  bool pair) {
   if (A_rows < M_total) return cudaErrorNotSupported;
   return moe::tc::launch_fmt<moe::kFmtMXFP4>(A, packed, scales, offsets, E, N, K, M_total, epi,
-                                             out, out_dt, dev_err, s, false);
+                                             out, out_dt, dev_err, s, false, pair);
 }
 
 }  // namespace moe_launch

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define MOE_NF4_ABI_VERSION 2
+#define MOE_NF4_ABI_VERSION 3
 
 typedef enum {
   MOE_OK = 0,
@@ -78,8 +78,13 @@ typedef enum { MOE_EPI_NONE = 0, MOE_EPI_SWIGLU = 1 } moe_epilogue_t;
  * tensor-memory (tcgen05) kernel otherwise; the others force one path. */
 typedef enum {
   MOE_ALGO_AUTO = 0,
-  MOE_ALGO_GEMV = 1, /* decode: streams weights, warp MMA per 16 rows      */
-  MOE_ALGO_TC = 2    /* prefill: tcgen05.mma with TMEM accumulators        */
+  MOE_ALGO_GEMV = 1,    /* decode: streams weights, warp MMA per 16 rows    */
+  MOE_ALGO_TC = 2,      /* prefill: tcgen05.mma with TMEM accumulators, one
+                           CTA per 128-weight-row tile                      */
+  MOE_ALGO_TC_PAIR = 3  /* the same on CTA pairs (cta_group::2, M = 256, two
+                           SMs per 256-weight-row tile); needs N % 256 == 0.
+                           Measured slower than MOE_ALGO_TC on the Qwen3
+                           shapes, so AUTO does not pick it                 */
 } moe_algo_t;
 
 /* Bits the kernels OR into the caller's device error word. */
@@ -167,7 +172,7 @@ moe_status_t moe_int4_quantize(const float* W, int E, int N, int K, uint8_t* pac
                                uint32_t* meta, int32_t* dev_err, void* stream);
 
 /*
- * moe_int4_grouped_gemm -- decode-shaped grouped GEMM on INT4 weights:
+ * moe_int4_grouped_gemm -- grouped GEMM on INT4 weights:
  * out[p] = W[e(p)] @ A[p] for every row p in expert e's segment
  * [expert_offsets[e], expert_offsets[e+1]), W[e] = (q - z) * s from
  * (packed, meta) as written by moe_int4_quantize, all experts in one launch.
@@ -176,20 +181,26 @@ moe_status_t moe_int4_quantize(const float* W, int E, int N, int K, uint8_t* pac
  *            (e.g. moe_permute_rows output); no gather
  *   packed   uint8 [E, N, K/2], meta uint32 [E, N, K/128]
  *   expert_offsets int32 [E+1] (device), monotone, offsets[E] == M_total
- *   N % 128 == 0, K % 256 == 0, E <= 1024
+ *   E <= 1024; decode GEMV: N % 128 == 0, K % 256 == 0; tensor-core kernel:
+ *            N % 128 == 0, K % 128 == 0
  *   epilogue MOE_EPI_NONE: out [M_total, N]; MOE_EPI_SWIGLU: rows [0, N/2)
  *            are gate and [N/2, N) up, out [M_total, N/2] = silu(g) * u
  *   out      F32 / F16 / BF16
- *   dev_err  as moe_nf4_grouped_gemm (BAD_OFFSETS, TIMEOUT, LAYOUT)
- * The weights enter the MMA as the exact integers q - z (fp16); each 64-k
- * block's fp32 partial sum is scaled by its group's s.  Streams every
- * selected expert's bytes once (HBM-bound at decode sizes).
+ *   algo     AUTO: the tensor-core kernel from 36 routed rows per expert on
+ *            average (as the NF4 call), else the decode GEMV; GEMV / TC force
+ *   dev_err  as moe_nf4_grouped_gemm (BAD_OFFSETS, TIMEOUT, LAYOUT, RANGE)
+ * Decode GEMV: the weights enter the MMA as the exact integers q - z (fp16);
+ * each 64-k block's fp32 partial sum is scaled by its group's s.  Streams
+ * every selected expert's bytes once (HBM-bound at decode sizes).
+ * Tensor-core kernel (tcgen05): weights enter as fp16((q - z) * s), one
+ * rounding of the exact value; sums fp32 in TMEM.
  * All pointers 16-byte aligned.
  */
 moe_status_t moe_int4_grouped_gemm(const void* A, int A_rows, const uint8_t* packed,
                                    const uint32_t* meta, const int32_t* expert_offsets, int E,
                                    int N, int K, int M_total, moe_epilogue_t epilogue, void* out,
-                                   moe_dtype_t out_dtype, int32_t* dev_err, void* stream);
+                                   moe_dtype_t out_dtype, moe_algo_t algo, int32_t* dev_err,
+                                   void* stream);
 
 /*
  * moe_mxfp4_quantize -- MXFP4 quantization of a fused expert stack, the format
@@ -264,13 +275,41 @@ moe_status_t moe_mxfp4_grouped_gemm(const void* A, int A_rows, const uint8_t* pa
  *   expert_offsets int32 [E+1] (device), monotone, offsets[E] == M_total,
  *            else MOE_DEVERR_BAD_OFFSETS and no output
  *   out      F32 or F16 [M_total, K]
- *   E <= 1024, K % 64 == 0.  fp32 sums.  All pointers 16-byte aligned.
+ *   algo     MOE_ALGO_GEMV: CUDA-core kernel (any G dtype, K % 64 == 0);
+ *            MOE_ALGO_TC: the tcgen05 kernel in its transposed form (G F16,
+ *            N % 64 == 0, K % 256 == 0): each thread decodes one output
+ *            column's weights down 64 rows into tensor memory, weights enter
+ *            as fp16(fp16(level) * fp16(absmax)) as in the forward TC kernel;
+ *            AUTO: TC when it applies and M_total >= 36 * E, else GEMV
+ *   E <= 1024.  fp32 sums.  All pointers 16-byte aligned.
  */
 moe_status_t moe_nf4_grouped_gemm_t(const void* G, moe_dtype_t g_dtype, int G_rows,
                                     const uint8_t* packed, const float* absmax,
                                     const int32_t* expert_offsets, int E, int N, int K,
                                     int M_total, void* out, moe_dtype_t out_dtype,
-                                    int32_t* dev_err, void* stream);
+                                    moe_algo_t algo, int32_t* dev_err, void* stream);
+
+/*
+ * moe_nf4_down_backward -- the down projection's backward and the SwiGLU
+ * backward in one tensor-core launch: with dh[p] = W_d[e(p)]^T @ dYp[p]
+ * (the transposed grouped GEMM over the down stack [E, H, I]) and the
+ * forward's gate_up pre-activations gu[p] = [g | u] (I each), s = sigmoid(g):
+ *   dgu[p, i] = dh u s (1 + g (1 - s)),  dgu[p, I + i] = dh g s.
+ * dh never reaches memory.  ("grouped-nf4-gemm & experts-4bit", fourth
+ * bullet: the backward computes on the packed weights, fused.)
+ *   dYp      F16 [G_rows >= M_total, H]   routed rows' output gradients
+ *   packed   uint8 [E, H, I/2], absmax fp32 [E, H*I/64]  (the down stack)
+ *   expert_offsets int32 [E+1], as above
+ *   gu       fp32 [M_total, 2I]            (the forward's, gate | up)
+ *   dgu      F32 or F16 [M_total, 2I]      output
+ *   H % 64 == 0, I % 256 == 0, E <= 1024; other shapes MOE_ERR_UNSUPPORTED
+ *   (use moe_nf4_grouped_gemm_t and moe_swiglu_backward).
+ * All pointers 16-byte aligned.
+ */
+moe_status_t moe_nf4_down_backward(const void* dYp, int G_rows, const uint8_t* packed,
+                                   const float* absmax, const int32_t* expert_offsets, int E,
+                                   int H, int I, int M_total, const float* gu, void* dgu,
+                                   moe_dtype_t dgu_dtype, int32_t* dev_err, void* stream);
 
 /*
  * moe_swiglu_backward -- for gu [M, 2I] (gate | up pre-activations) and

@@ -117,9 +117,11 @@ def route_backward(logits: np.ndarray, idx: np.ndarray, dw: np.ndarray,
 
 
 def moe_layer_backward(x: np.ndarray, logits: np.ndarray, stack: ExpertStack, k: int,
-                       renormalize: bool, dY: np.ndarray):
+                       renormalize: bool, dY: np.ndarray, with_dw: bool = False):
     """``(dx [T, H], dlogits [T, E])`` of ``oracle.moe_layer`` for the output
-    gradient ``dY [T, H]``, one token and one routed expert at a time."""
+    gradient ``dY [T, H]``, one token and one routed expert at a time.
+    ``with_dw``: also return ``(idx [T, k], dw [T, k])``, the selection and
+    the gradient w.r.t. its routing weights."""
     x = np.asarray(x, dtype=np.float64)
     dY = np.asarray(dY, dtype=np.float64)
     idx, w = route_topk(np.asarray(logits, dtype=np.float32), k, renormalize)
@@ -137,7 +139,8 @@ def moe_layer_backward(x: np.ndarray, logits: np.ndarray, stack: ExpertStack, k:
             dh = Wd.T @ (w[t, j] * dY[t])
             dgu = swiglu_backward(gu[None], dh[None])[0]
             dx[t] += Wgu.T @ dgu
-    return dx, route_backward(logits, idx, dw, renormalize)
+    dl = route_backward(logits, idx, dw, renormalize)
+    return (dx, dl, idx, dw) if with_dw else (dx, dl)
 
 
 def moe_layer_backward_permuted(x, logits, stack: ExpertStack, k: int, renormalize: bool,

@@ -58,13 +58,13 @@ int main(int argc, char** argv) {
     void* P = load("gt_P.bin", (size_t)E * N * K / 2); void* A = load("gt_A.bin", (size_t)E * N * K / 64 * 4);
     void* G = load("gt_G.bin", (size_t)(M + 2) * N * 4); int32_t* off = (int32_t*)load("gt_off.bin", (E + 1) * 4);
     float* o = (float*)zeros((size_t)M * K * 4);
-    ST(moe_nf4_grouped_gemm_t(G, MOE_DT_F32, M + 2, (uint8_t*)P, (float*)A, off, E, N, K, M, o, MOE_DT_F32, err, nullptr));
+    ST(moe_nf4_grouped_gemm_t(G, MOE_DT_F32, M + 2, (uint8_t*)P, (float*)A, off, E, N, K, M, o, MOE_DT_F32, MOE_ALGO_GEMV, err, nullptr));
     CK(cudaDeviceSynchronize()); printf("gemm_t dev_err=%d\n", err_word(err)); dump("gt_out.bin", o, (size_t)M * K * 4); }
   { const int E = 4, N = 70, K = 320, M = 13;
     void* P = load("gt2_P.bin", (size_t)E * N * K / 2); void* A = load("gt2_A.bin", (size_t)E * N * K / 64 * 4);
     void* G = load("gt2_G.bin", (size_t)M * N * 4); int32_t* off = (int32_t*)load("gt2_off.bin", (E + 1) * 4);
     float* o = (float*)zeros((size_t)M * K * 4);
-    ST(moe_nf4_grouped_gemm_t(G, MOE_DT_F32, M, (uint8_t*)P, (float*)A, off, E, N, K, M, o, MOE_DT_F32, err, nullptr));
+    ST(moe_nf4_grouped_gemm_t(G, MOE_DT_F32, M, (uint8_t*)P, (float*)A, off, E, N, K, M, o, MOE_DT_F32, MOE_ALGO_GEMV, err, nullptr));
     CK(cudaDeviceSynchronize()); printf("gemm_t2 dev_err=%d\n", err_word(err)); dump("gt2_out.bin", o, (size_t)M * K * 4); }
   // 4. SwiGLU backward [37, 96]
   { const int M = 37, I = 96;

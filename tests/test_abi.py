@@ -47,7 +47,7 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
     for code, name in _lib.STATUS.items():
         assert lib.moe_status_string(code).decode() == name
 
@@ -129,12 +129,17 @@ def test_int4_calls_reject_bad_arguments(lib):
     assert lib.moe_int4_quantize(A, 1, 8, 256, M, A, None, None) == 2
     # grouped GEMM: N % 128 or K % 256 -> unsupported; bad epilogue / dtype;
     # A_rows < M_total; misaligned output
-    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 64, 256, 8, 0, A, 0, None, None) == 3
-    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 384, 8, 0, A, 0, None, None) == 3
-    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 7, A, 0, None, None) == 1
-    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 9, None, None) == 1
-    assert lib.moe_int4_grouped_gemm(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, None, None) == 1
-    assert lib.moe_int4_grouped_gemm(A, 8, A, A, A, 2, 128, 256, 8, 0, M, 0, None, None) == 2
+    # (..., epilogue, out, out_dtype, algo, dev_err, stream); K = 384 has no
+    # GEMV form (K % 256) but a tensor-core one (K % 128)
+    g4 = lib.moe_int4_grouped_gemm
+    assert g4(A, 8, A, A, A, 2, 64, 256, 8, 0, A, 0, 0, None, None) == 3
+    assert g4(A, 8, A, A, A, 2, 128, 384, 8, 0, A, 0, 1, None, None) == 3
+    assert g4(A, 8, A, A, A, 2, 128, 192, 8, 0, A, 0, 2, None, None) == 3
+    assert g4(A, 8, A, A, A, 2, 128, 256, 8, 7, A, 0, 0, None, None) == 1
+    assert g4(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 9, 0, None, None) == 1
+    assert g4(A, 8, A, A, A, 2, 128, 256, 8, 0, A, 0, 5, None, None) == 1
+    assert g4(A, 4, A, A, A, 2, 128, 256, 8, 0, A, 0, 0, None, None) == 1
+    assert g4(A, 8, A, A, A, 2, 128, 256, 8, 0, M, 0, 0, None, None) == 2
 
 
 def test_lora_delta_rejects_bad_arguments(lib):
@@ -177,12 +182,22 @@ def test_mxfp4_calls_reject_bad_arguments(lib):
 def test_backward_calls_reject_bad_arguments(lib):
     A, M = ALIGNED, MISALIGNED
     # transposed GEMM: (G, g_dtype, G_rows, packed, absmax, offsets, E, N, K, M_total, out,
-    # out_dtype, dev_err, stream): bf16 G, K % 64, G_rows < M_total, misaligned out
+    # out_dtype, algo, dev_err, stream): bf16 G, K % 64, G_rows < M_total, misaligned out,
+    # bad algo; the tensor-core form needs fp16 G and K % 256
     t = lib.moe_nf4_grouped_gemm_t
-    assert t(A, 1, 8, A, A, A, 2, 128, 256, 8, A, 0, None, None) == 1
-    assert t(A, 0, 8, A, A, A, 2, 128, 96, 8, A, 0, None, None) == 1
-    assert t(A, 0, 4, A, A, A, 2, 128, 256, 8, A, 0, None, None) == 1
-    assert t(A, 0, 8, A, A, A, 2, 128, 256, 8, M, 0, None, None) == 2
+    assert t(A, 1, 8, A, A, A, 2, 128, 256, 8, A, 0, 0, None, None) == 1
+    assert t(A, 0, 8, A, A, A, 2, 128, 96, 8, A, 0, 0, None, None) == 1
+    assert t(A, 0, 4, A, A, A, 2, 128, 256, 8, A, 0, 0, None, None) == 1
+    assert t(A, 0, 8, A, A, A, 2, 128, 256, 8, M, 0, 0, None, None) == 2
+    assert t(A, 0, 8, A, A, A, 2, 128, 256, 8, A, 0, 9, None, None) == 1
+    assert t(A, 0, 8, A, A, A, 2, 128, 256, 8, A, 0, 2, None, None) == 3
+    assert t(A, 2, 8, A, A, A, 2, 128, 192, 8, A, 0, 2, None, None) == 3
+    # fused down backward (dYp, G_rows, packed, absmax, offsets, E, H, I, M_total, gu, dgu,
+    # dgu_dtype, dev_err, stream): I % 256, bf16 output, null gu
+    d = lib.moe_nf4_down_backward
+    assert d(A, 8, A, A, A, 2, 128, 192, 8, A, A, 0, None, None) == 3
+    assert d(A, 8, A, A, A, 2, 128, 256, 8, A, A, 1, None, None) == 1
+    assert d(A, 8, A, A, A, 2, 128, 256, 8, None, A, 0, None, None) == 1
     # SwiGLU backward: bf16 inputs, null dh
     assert lib.moe_swiglu_backward(A, A, 1, 4, 8, A, 0, None) == 1
     assert lib.moe_swiglu_backward(A, None, 0, 4, 8, A, 0, None) == 1

@@ -99,3 +99,27 @@ def test_int4_grouped_gemm_flags_bad_offsets():
     moe.int4_grouped_gemm(X, packed, meta, bad, 8, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) & moe.DEVERR_BAD_OFFSETS
+
+
+@pytest.mark.parametrize("epi", ["none", "swiglu"])
+@pytest.mark.parametrize("counts", [[1, 0, 15, 16, 17, 300], [0, 0, 513, 0, 2, 256]])
+def test_int4_tc_grouped_gemm_ragged(epi, counts):
+    # the tcgen05 kernel on INT4 weights, fp16((q - z) s) in tensor memory;
+    # K = 384 has no decode-GEMV form
+    off = _ragged(counts)
+    E, M = len(counts), int(off[-1])
+    g = torch.Generator().manual_seed(sum(counts) + 13 * len(epi))
+    N, K = (512, 384) if epi == "swiglu" else (256, 640)
+    W = torch.randn((E, N, K), generator=g) * 0.03
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    packed, meta = moe.int4_quantize(W.cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.int4_grouped_gemm(X.cuda(), packed, meta, torch.from_numpy(off).cuda(), M,
+                                epilogue=epi, out_dtype=torch.float32, algo="tc", dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    p_ref, m_ref = oracle.quantize_int4_grouped(W.numpy())
+    ref = oracle.grouped_gemm_int4(X.float().numpy(), p_ref, m_ref, off)
+    if epi == "swiglu":
+        ref = oracle.swiglu(ref)
+    assert_close(out.cpu().numpy(), ref, f"int4 tc {epi} {counts}")

@@ -40,12 +40,13 @@ def _ragged(E, counts):
     return off
 
 
+@pytest.mark.parametrize("algo", ["tc", "tc_pair"])
 @pytest.mark.parametrize("epi", ["none", "swiglu"])
 @pytest.mark.parametrize("counts", [
     [1, 0, 15, 16, 17, 300],          # partial N tiles, an empty expert, two token tiles
     [0, 0, 513, 0, 2, 256],           # three token tiles, exact 256 tile
 ])
-def test_tc_grouped_gemm_ragged(epi, counts):
+def test_tc_grouped_gemm_ragged(epi, counts, algo):
     E = len(counts)
     counts = np.array(counts)
     off = _ragged(E, counts)
@@ -57,14 +58,14 @@ def test_tc_grouped_gemm_ragged(epi, counts):
     p, a = moe.nf4_quantize(W.cuda())
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
-                               out_dtype=torch.float32, algo="tc", dev_err=err)
+                               out_dtype=torch.float32, algo=algo, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     pr, ar = oracle.quantize_blockwise(W.numpy())
     ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
     if epi == "swiglu":
         ref = oracle.swiglu(ref)
-    assert_close(_np(out), ref, f"tc {epi}")
+    assert_close(_np(out), ref, f"{algo} {epi}")
 
 
 @pytest.mark.parametrize("K", [64, 192, 320])
@@ -92,9 +93,10 @@ def test_tc_short_and_odd_k(K):
         assert_close(_np(out), ref, f"tc K={K} {epi}")
 
 
+@pytest.mark.parametrize("algo", ["tc", "tc_pair"])
 @pytest.mark.parametrize("epi,N,K", [("swiglu", 3072, 4096), ("none", 4096, 1536)],
                          ids=["gate_up", "down"])
-def test_tc_grouped_gemm_qwen3_235b_dims(epi, N, K):
+def test_tc_grouped_gemm_qwen3_235b_dims(epi, N, K, algo):
     # The Qwen3-235B-A22B expert projections (gate_up 4096 -> 2*1536 with the
     # SwiGLU epilogue, down 1536 -> 4096) on four experts with ragged row
     # counts: an empty expert, partial and full 256-row token tiles, weights
@@ -112,7 +114,7 @@ def test_tc_grouped_gemm_qwen3_235b_dims(epi, N, K):
     p, a = moe.nf4_quantize(W.cuda())
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
-                               out_dtype=torch.float32, algo="tc", dev_err=err)
+                               out_dtype=torch.float32, algo=algo, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     pr, ar = oracle.quantize_blockwise(W.numpy())
@@ -151,3 +153,55 @@ def test_layer_qwen3_prefill_tc_sampled():
     ref = oracle.moe_layer(X.float().numpy(), lg.numpy(), stack, shape.k, shape.renormalize,
                            tokens=toks)
     assert_close(_np(Y)[toks], ref, "qwen3 prefill (tensor cores)")
+
+
+@pytest.mark.parametrize("epi,N,K", [("none", 384, 256), ("swiglu", 640, 192)])
+def test_tc_single_cta_form(epi, N, K):
+    # N not a multiple of 256 (the pair form's tile): single-CTA tiles of 128
+    # weight rows, and the pair form is refused
+    counts = np.array([33, 0, 300, 7])
+    E = len(counts)
+    off = _ragged(E, counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(N + K + 1)
+    W = torch.randn((E, N, K), generator=g) * 0.05
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    p, a = moe.nf4_quantize(W.cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
+                               out_dtype=torch.float32, algo="tc", dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    pr, ar = oracle.quantize_blockwise(W.numpy())
+    ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
+    if epi == "swiglu":
+        ref = oracle.swiglu(ref)
+    assert_close(_np(out), ref, f"tc single-CTA {epi}")
+    with pytest.raises(moe.MoEError, match="UNSUPPORTED"):
+        moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
+                             algo="tc_pair")
+
+
+@pytest.mark.parametrize("counts", [[1, 2, 3, 31, 32, 33], [255, 257, 1, 0, 0, 64]])
+def test_tc_pair_form_small_and_odd_tiles(counts):
+    # the pair form rounds a tile's routed rows up to 32 and splits them
+    # between the two CTAs: tiles of 1..33 rows and tiles straddling 256
+    E = len(counts)
+    counts = np.array(counts)
+    off = _ragged(E, counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(int(counts.sum()) + 5)
+    N, K = 512, 320
+    W = torch.randn((E, N, K), generator=g) * 0.05
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    p, a = moe.nf4_quantize(W.cuda())
+    pr, ar = oracle.quantize_blockwise(W.numpy())
+    ref = oracle.grouped_gemm(X.float().numpy(), pr, ar.reshape(E, -1), off)
+    for epi in ("none", "swiglu"):
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = moe.nf4_grouped_gemm(X.cuda(), p, a, torch.from_numpy(off).cuda(), M, epilogue=epi,
+                                   out_dtype=torch.float32, algo="tc_pair", dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        r = oracle.swiglu(ref) if epi == "swiglu" else ref
+        assert_close(_np(out), r, f"tc pair {epi} {counts.tolist()}")
