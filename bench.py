@@ -241,8 +241,8 @@ def rank_seed(seed, rank):
 # bytes per weight: the 4-bit code plus its share of the scales (NF4: fp32
 # absmax per 64; INT4: fp16 scale + zero in 4 B per 128; MXFP4: 1 B per 32)
 BYTES_PER_WEIGHT = {"nf4": 0.5625, "int4": 0.53125, "mxfp4": 0.53125}
-DECODE_KERNEL_SOURCE = {"nf4": "grouped_gemm_decode.cu", "int4": "grouped_gemm_int4.cu",
-                        "mxfp4": "grouped_gemm_mxfp4.cu"}
+DECODE_KERNEL_SOURCE = {"nf4": "grouped_gemm_decode.cu", "int4": "grouped_gemm_decode.cu",
+                        "mxfp4": "grouped_gemm_decode.cu"}
 
 class Workload:
     """One configuration's NF4 (or INT4, MXFP4) layer stacks on the device,

@@ -116,19 +116,27 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const InT* __restrict
     if (!ok && lane == 0) set_dev_err(dev_err, MOE_DEVERR_BAD_INDEX);
     const InT* src = X + (size_t)(ok ? f / k : 0) * K;
     __half* dst = Xp + (size_t)p * K;
-    for (int c = lane * 8; c < K; c += 256) {
-      uint4 o;
-      if (!ok) {
-        o = make_uint4(0, 0, 0, 0);
-      } else if constexpr (sizeof(InT) == 2 && !std::is_same<InT, __half>::value) {
-        const uint4 u = *reinterpret_cast<const uint4*>(src + c);
-        o = make_uint4(bf16x2_to_f16x2(u.x), bf16x2_to_f16x2(u.y), bf16x2_to_f16x2(u.z),
-                       bf16x2_to_f16x2(u.w));
-        ovf |= any_f16x8_nonfinite(o);
-      } else {
-        o = *reinterpret_cast<const uint4*>(src + c);
+    // eight 16-byte loads in flight per lane before the first store: a row
+    // costs about one memory latency even when the grid is a single CTA
+    for (int c0 = lane * 8; c0 < K; c0 += 8 * 256) {
+      uint4 u[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + i * 256;
+        u[i] = (ok && c < K) ? *reinterpret_cast<const uint4*>(src + c) : make_uint4(0, 0, 0, 0);
       }
-      *reinterpret_cast<uint4*>(dst + c) = o;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + i * 256;
+        if (c >= K) break;
+        uint4 o = u[i];
+        if constexpr (sizeof(InT) == 2 && !std::is_same<InT, __half>::value) {
+          o = make_uint4(bf16x2_to_f16x2(o.x), bf16x2_to_f16x2(o.y), bf16x2_to_f16x2(o.z),
+                         bf16x2_to_f16x2(o.w));
+          ovf |= any_f16x8_nonfinite(o);
+        }
+        *reinterpret_cast<uint4*>(dst + c) = o;
+      }
     }
   }
   // every lane of the warp leaves the row loop together (warp-uniform p)

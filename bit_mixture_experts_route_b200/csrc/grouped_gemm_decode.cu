@@ -1,32 +1,49 @@
-// Grouped NF4 GEMM, decode path with TMA-staged weights (few rows per
-// expert; HBM-bound).
+// Grouped 4-bit GEMM, decode path (few routed rows per expert; HBM-bound):
+// one pipeline for the three weight formats.
 //
 // "grouped-nf4-gemm & experts-4bit" (jordananderson-pages.pages.dev), first
-// bullet: one launch for all active experts, the 16-entry codebook decoded in
-// registers, no dequantized weight copy.  At decode sizes the whole cost is
-// streaming the NF4 bytes of every expert that received a token, so the
-// kernel is built to keep HBM busy with as few instructions per weight as
-// possible:
+// bullet: one launch for all active experts, the codebook decoded in
+// registers, no dequantized weight copy; third bullet: the same kernel runs on
+// the released MXFP4 bytes and on GPTQ-style INT4 experts.  At decode sizes
+// the whole cost is streaming the packed bytes of every expert that received
+// a token, so the kernel is built to keep HBM busy.
+//
+// Formats (FMT):
+//   NF4    two codes per byte (even element in the HIGH nibble), fp32 absmax
+//          per 64 along K; w = L[code] * absmax.
+//   MXFP4  two E2M1 codes per byte (even element in the LOW nibble), one E8M0
+//          byte b per 32 along K; w = 2^(b - 127) * e2m1(code).
+//   INT4   two codes per byte (even element in the high nibble), per 128 along
+//          K an fp16 scale s and a 4-bit zero z (meta word s | z << 16);
+//          w = (q - z) * s.
 //
 // * Persistent CTAs (one per SM) walk a list of work items built on the
 //   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
 //   rows; an expert with more routed rows yields one item per 16).
 // * One producer thread streams each item through a 5-stage ring with TMA
-//   tile loads, 256 k per stage and six copies per stage: the packed rows
-//   (one 3-D box of 2 x 64 rows x 128 bytes), their absmax (one 3-D box of
-//   2 x 64 rows x 4 fp32) and the routed activation rows (one box of 8 or 16
-//   rows per 64-k block), with 128-byte swizzle.
-// * Eight consumer warps each own 16 weight rows and run mma.sync.m16n8k16
-//   with the weights as the M side and the routed rows as N (swap-AB).  A
-//   lane turns each packed byte into an fp16 pair {L[hi], L[lo]} with ONE
+//   tile loads, 256 k per stage: the packed rows (one 3-D box of 2 x 64 rows x
+//   128 bytes), for NF4 their absmax (one 3-D box of 2 x 64 rows x 4 fp32) and
+//   the routed activation rows (one box of 8 or 16 rows per 64-k block), with
+//   128-byte swizzle.
+// * Eight consumer warps each own 16 weight rows of the item and run
+//   mma.sync.m16n8k16 with the weights as the M side and the routed rows as N
+//   (swap-AB); the four 64-k blocks of a stage run as four interleaved MMA
+//   chains.  A lane turns each packed byte into an fp16 pair through ONE
 //   byte_perm (which assembles the shared address of the byte's entry in a
-//   per-lane table: 0x10000 | byte << 8 | lane << 2) and one shared load.
-//   The table sits at shared address 64 KB, one 256-byte row per byte value,
-//   so the lookups never conflict.  The four 64-k blocks of a stage run as
-//   four interleaved MMA chains, and each block's fp32 absmax scales its
-//   fp32 partial sums (the only weight rounding is the levels' fp16 one).
+//   per-lane table: 0x10000 | byte << 8 | lane << 2) and one shared load; the
+//   table sits at shared address 64 KB, one 256-byte row per byte value, so
+//   the lookups never conflict.
+// * Scales: NF4 scales each 64-k block's fp32 partial sum by the row's fp32
+//   absmax (the only weight rounding is the levels' fp16 one); INT4 subtracts
+//   the zero in fp16 (exact) and scales the block's fp32 partial sum by s;
+//   MXFP4 multiplies the fp16 pairs by the block's power of two (exact while
+//   2^(b - 127) lies in [2^-23, 2^13]; scale bytes outside that range, other
+//   than 0, set MOE_DEVERR_RANGE).  INT4 and MXFP4 scales come from global
+//   memory, one stage ahead.
 // * MMA row g of a warp maps to weight row sigma(g) = 2(g mod 4) + g div 4,
-//   which makes the swizzled 8-byte reads of the packed rows conflict-free.
+//   which makes the swizzled 8-byte reads of the packed rows conflict-free;
+//   the k order inside a block is permuted the same way on both operands (a
+//   lane's 8 packed bytes are 16 consecutive k).
 // * The SwiGLU epilogue pairs gate row j and up row I + j in the same lane.
 // Every wait is bounded; on expiry MOE_DEVERR_TIMEOUT is set and all roles
 // leave their loops.
@@ -40,27 +57,30 @@ constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int SB = SK / 2;      // packed bytes per row per stage
 constexpr int STAGES = 5;
-constexpr int CWARPS = 8;
+constexpr int CWARPS = 8;       // two row groups x four k blocks
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr int XBOX = 8 * 64 * 2;                 // one 8-row x 64-k fp16 box
 constexpr int XKBOX = (TOK / 8) * XBOX;          // 16 rows x 64 k
 constexpr uint32_t kWBytes = ROWS * SB;          // packed rows per stage
 constexpr uint32_t kXBytes = 4 * XKBOX;          // activations per stage (max)
-constexpr uint32_t kABytes = ROWS * 16;          // absmax per stage
-constexpr uint32_t kStageBytes = kWBytes + kXBytes + kABytes;  // 26 KB, 1 KB multiple
+constexpr uint32_t kABytes = ROWS * 16;          // NF4 absmax per stage
+constexpr int MX_BLK = 32;                       // MXFP4: k per scale byte
+constexpr int I4_GROUP = 128;                    // INT4: k per scale / zero
 
-// Absolute shared-memory layout.  The dynamic window must start at or below
-// 1 KB (checked at run time).  Stages need 1 KB alignment (128-byte swizzle).
-constexpr uint32_t kStage0 = 1024;                        // stages 0-1
-constexpr uint32_t kMisc = kStage0 + 2 * kStageBytes;     // barriers, item list
-constexpr uint32_t kLut = 65536;                          // table: 256 x 256 B
-constexpr uint32_t kStage2 = 2 * 65536;                   // stages 2-4
-constexpr uint32_t kEnd = kStage2 + (STAGES - 2) * kStageBytes;
-
-__device__ __forceinline__ uint32_t stage_addr(int s) {
-  return s < 2 ? kStage0 + s * kStageBytes : kStage2 + (s - 2) * kStageBytes;
-}
+template <int FMT>
+struct Layout {
+  static constexpr uint32_t kA = FMT == kFmtNF4 ? kABytes : 0;
+  static constexpr uint32_t kStageBytes = kWBytes + kXBytes + kA;  // 1 KB multiple
+  // Absolute shared-memory layout.  The dynamic window must start at or
+  // below 1 KB (checked at run time).  Stages need 1 KB alignment (128-byte
+  // swizzle).
+  static constexpr uint32_t kStage0 = 1024;                      // stages 0-1
+  static constexpr uint32_t kMisc = kStage0 + 2 * kStageBytes;   // barriers, item list
+  static constexpr uint32_t kLut = 65536;                        // table: 256 x 256 B
+  static constexpr uint32_t kStage2 = 2 * 65536;                 // stages 2-4
+  static constexpr uint32_t kEnd = kStage2 + (STAGES - 2) * kStageBytes;
+};
 
 struct Misc {
   uint64_t full[STAGES], empty[STAGES];
@@ -68,7 +88,9 @@ struct Misc {
   int nitems;
   int item_prefix[1025];
 };
-static_assert(kMisc + sizeof(Misc) <= kLut, "shared layout overlap");
+static_assert(Layout<kFmtNF4>::kMisc + sizeof(Misc) <= Layout<kFmtNF4>::kLut,
+              "shared layout overlap");
+static_assert(Layout<kFmtNF4>::kEnd <= 227 * 1024 + 1024, "shared layout too large");
 
 __constant__ float c_levels_dec[16] = {MOE_NF4_LEVEL_LIST};
 
@@ -139,6 +161,14 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
@@ -181,11 +211,24 @@ __device__ __forceinline__ Item item_info(const Misc& ms, const int32_t* offsets
   return r;
 }
 
-// One item's main loop and epilogue for one consumer warp, NT8 token tiles.
-template <int EPI, typename OutT, int NT8>
+// Weight row (within the expert's N rows) of stage-local row r of rtile.
+template <int EPI>
+__device__ __forceinline__ int weight_row(int r, int rtile, int N) {
+  if (EPI == MOE_EPI_SWIGLU)
+    return r < ROWS / 2 ? rtile * (ROWS / 2) + r : N / 2 + rtile * (ROWS / 2) + (r - ROWS / 2);
+  return rtile * ROWS + r;
+}
+
+// One item for one consumer warp, NT8 token tiles.  Warp w owns 16 weight
+// rows of the item (SwiGLU: gate rows 8 w .. 8 w + 7 and the matching up
+// rows) and all four 64-k blocks of every stage: four independent MMA chains
+// per token tile.  Returns false if a wait gave up.
+template <int FMT, int EPI, typename OutT, int NT8>
 __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, int K,
+                                             const void* __restrict__ gscales,
                                              OutT* __restrict__ out, int32_t* dev_err,
                                              int& stage, uint32_t& phase) {
+  using LY = Layout<FMT>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int sg = ((g & 3) << 1) | (g >> 2);  // sigma(g)
@@ -197,10 +240,26 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
   // row index is congruent to sg (mod 8): chunk (2b + t/2) ^ sg, half t & 1
   uint32_t woff[4];
 #pragma unroll
-  for (int b = 0; b < 4; ++b)
-    woff[b] = ((((2 * b + (t >> 1)) ^ sg) << 4) | ((t & 1) << 3));
-  // activation rows 8j + g: chunks 2t and 2t+1 of the 128-byte line, swizzled
+  for (int b = 0; b < 4; ++b) woff[b] = ((((2 * b + (t >> 1)) ^ sg) << 4) | ((t & 1) << 3));
+  // activation rows 8j + g: chunks 2t and 2t+1 of a block's 128-byte line
   const uint32_t xo0 = (uint32_t)(((2 * t) ^ g) << 4), xo1 = (uint32_t)(((2 * t + 1) ^ g) << 4);
+
+  // INT4 / MXFP4 scales of rows rA and rB from global memory, one stage
+  // ahead: INT4 the meta words of the stage's two 128-k groups, MXFP4 the
+  // stage's eight scale bytes
+  const size_t gA = (size_t)it.expert * N + weight_row<EPI>(rA, it.rtile, N);
+  const size_t gB = (size_t)it.expert * N + weight_row<EPI>(rB, it.rtile, N);
+  auto fetch = [&](int s, uint2& mA, uint2& mB) {
+    if (FMT == kFmtINT4) {
+      const uint2* p = reinterpret_cast<const uint2*>(static_cast<const uint32_t*>(gscales));
+      mA = __ldg(p + gA * (K / I4_GROUP / 2) + s);
+      mB = __ldg(p + gB * (K / I4_GROUP / 2) + s);
+    } else if (FMT == kFmtMXFP4) {
+      const uint2* p = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(gscales));
+      mA = __ldg(p + gA * (K / MX_BLK / 8) + s);
+      mB = __ldg(p + gB * (K / MX_BLK / 8) + s);
+    }
+  };
 
   float acc[NT8][4];
 #pragma unroll
@@ -208,16 +267,47 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[j][q] = 0.0f;
 
+  bool bad_scale = false;
   const int KS = K / SK;
+  uint2 cA = make_uint2(0, 0), cB = make_uint2(0, 0);
+  if (FMT != kFmtNF4) fetch(0, cA, cB);
   for (int s = 0; s < KS; ++s) {
-    const uint32_t base = stage_addr(stage);
+    uint2 nA = make_uint2(0, 0), nB = make_uint2(0, 0);
+    if (FMT != kFmtNF4 && s + 1 < KS) fetch(s + 1, nA, nB);
+    const uint32_t base = stage < 2 ? LY::kStage0 + stage * LY::kStageBytes
+                                    : LY::kStage2 + (stage - 2) * LY::kStageBytes;
     if (!mbar_wait(smem_u32(&ms.full[stage]), phase, ms, dev_err)) return false;
     const uint32_t wst = base, xst = base + kWBytes, ast = base + kWBytes + kXBytes;
-    const uint4 sa = lds128(ast + rA * 16), sb = lds128(ast + rB * 16);
-    const float sav[4] = {__uint_as_float(sa.x), __uint_as_float(sa.y), __uint_as_float(sa.z),
-                          __uint_as_float(sa.w)};
-    const float sbv[4] = {__uint_as_float(sb.x), __uint_as_float(sb.y), __uint_as_float(sb.z),
-                          __uint_as_float(sb.w)};
+    // per block b: the fp32 factor of its partial sums (NF4 absmax, INT4 s)
+    // and the fp16-pair operand transform (INT4 {1024 + z}, MXFP4 2^(e-127))
+    float fA[4] = {1.f, 1.f, 1.f, 1.f}, fB[4] = {1.f, 1.f, 1.f, 1.f};
+    uint32_t zA[4] = {0, 0, 0, 0}, zB[4] = {0, 0, 0, 0};
+    if (FMT == kFmtNF4) {
+      const uint4 sa = lds128(ast + rA * 16), sb = lds128(ast + rB * 16);
+      fA[0] = __uint_as_float(sa.x); fA[1] = __uint_as_float(sa.y);
+      fA[2] = __uint_as_float(sa.z); fA[3] = __uint_as_float(sa.w);
+      fB[0] = __uint_as_float(sb.x); fB[1] = __uint_as_float(sb.y);
+      fB[2] = __uint_as_float(sb.z); fB[3] = __uint_as_float(sb.w);
+    } else if (FMT == kFmtINT4) {
+      const uint32_t mA[2] = {cA.x, cA.y}, mB[2] = {cB.x, cB.y};
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t a = mA[b >> 1], c = mB[b >> 1];  // group of this 64-k block
+        fA[b] = __half2float(__ushort_as_half((unsigned short)(a & 0xFFFFu)));
+        fB[b] = __half2float(__ushort_as_half((unsigned short)(c & 0xFFFFu)));
+        zA[b] = 0x64006400u | ((a >> 16) & 0xFu) * 0x00010001u;
+        zB[b] = 0x64006400u | ((c >> 16) & 0xFu) * 0x00010001u;
+      }
+    } else {
+      const uint32_t mA[2] = {cA.x, cA.y}, mB[2] = {cB.x, cB.y};
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        // a lane's 16 k of block b lie in scale block 2b + t/2 of the stage
+        const int sbi = 2 * b + (t >> 1);
+        zA[b] = mx_scale_h2((mA[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu, bad_scale);
+        zB[b] = mx_scale_h2((mB[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu, bad_scale);
+      }
+    }
     uint32_t xf[4][NT8][8];
     uint2 wa[4], wb[4];
 #pragma unroll
@@ -246,29 +336,42 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
         af[1] = lds32(__byte_perm(vB, lb, s0));
         af[2] = lds32(__byte_perm(vA, lb, s1));
         af[3] = lds32(__byte_perm(vB, lb, s1));
+        if (FMT == kFmtINT4) {
+          af[0] = hsub2_u(af[0], zA[b]); af[2] = hsub2_u(af[2], zA[b]);
+          af[1] = hsub2_u(af[1], zB[b]); af[3] = hsub2_u(af[3], zB[b]);
+        } else if (FMT == kFmtMXFP4) {
+          af[0] = hmul2_u(af[0], zA[b]); af[2] = hmul2_u(af[2], zA[b]);
+          af[1] = hmul2_u(af[1], zB[b]); af[3] = hmul2_u(af[3], zB[b]);
+        }
 #pragma unroll
         for (int j = 0; j < NT8; ++j) {
-          if (i == 0)
+          if (FMT == kFmtMXFP4)
+            mma_16816(acc[j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
+          else if (i == 0)
             mma_16816_z(tmp[b][j], af, xf[b][j][0], xf[b][j][1]);
           else
             mma_16816(tmp[b][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
         }
       }
     }
+    if (FMT != kFmtMXFP4) {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+      for (int b = 0; b < 4; ++b)
 #pragma unroll
-      for (int j = 0; j < NT8; ++j) {
-        acc[j][0] = fmaf(sav[b], tmp[b][j][0], acc[j][0]);
-        acc[j][1] = fmaf(sav[b], tmp[b][j][1], acc[j][1]);
-        acc[j][2] = fmaf(sbv[b], tmp[b][j][2], acc[j][2]);
-        acc[j][3] = fmaf(sbv[b], tmp[b][j][3], acc[j][3]);
-      }
+        for (int j = 0; j < NT8; ++j) {
+          acc[j][0] = fmaf(fA[b], tmp[b][j][0], acc[j][0]);
+          acc[j][1] = fmaf(fA[b], tmp[b][j][1], acc[j][1]);
+          acc[j][2] = fmaf(fB[b], tmp[b][j][2], acc[j][2]);
+          acc[j][3] = fmaf(fB[b], tmp[b][j][3], acc[j][3]);
+        }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&ms.empty[stage]));
     if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    cA = nA;
+    cB = nB;
   }
+  if (bad_scale) set_dev_err(dev_err, MOE_DEVERR_RANGE);
 
   // acc[j][q]: row rA (q < 2) or rB (q >= 2), routed row 8j + 2t + (q & 1)
 #pragma unroll
@@ -279,37 +382,36 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
       if (tok >= it.cnt) continue;
       const size_t p = (size_t)(it.start + tok);
       if (EPI == MOE_EPI_SWIGLU) {
-        const int I = N / 2;
-        const int col = it.rtile * (ROWS / 2) + 8 * warp + sg;
-        store_checked(out, p * I + col, swiglu_f32(acc[j][q], acc[j][q + 2]), dev_err);
+        store_checked(out, p * (N / 2) + it.rtile * (ROWS / 2) + rA,
+                      swiglu_f32(acc[j][q], acc[j][q + 2]), dev_err);
       } else {
-        const int col = it.rtile * ROWS + 16 * warp + sg;
-        store_checked(out, p * N + col, acc[j][q], dev_err);
-        store_checked(out, p * N + col + 8, acc[j][q + 2], dev_err);
+        store_checked(out, p * N + it.rtile * ROWS + rA, acc[j][q], dev_err);
+        store_checked(out, p * N + it.rtile * ROWS + rB, acc[j][q + 2], dev_err);
       }
     }
   }
   return true;
 }
 
-template <int EPI, typename OutT>
-__global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
+template <int FMT, int EPI, typename OutT>
+__global__ void __launch_bounds__(THREADS, 1) decode_kernel(
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
     const __grid_constant__ CUtensorMap xmap8, const __grid_constant__ CUtensorMap xmap16,
-    const int32_t* __restrict__ offsets, int E, int N, int K, int M_total,
-    OutT* __restrict__ out, int32_t* dev_err, int chain) {
+    const void* __restrict__ gscales, const int32_t* __restrict__ offsets, int E, int N, int K,
+    int M_total, OutT* __restrict__ out, int32_t* dev_err, int chain) {
+  using LY = Layout<FMT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (!chain) {  // nothing is read or written before the previous kernel is done
     pdl_wait();
     pdl_trigger();
   }
   const uint32_t base = smem_u32(smem_raw);
-  if (base > kStage0) {  // layout assumption broken: do nothing, say so
+  if (base > LY::kStage0) {  // layout assumption broken: do nothing, say so
     if (threadIdx.x == 0) set_dev_err(dev_err, MOE_DEVERR_LAYOUT);
     return;
   }
-  Misc& ms = *reinterpret_cast<Misc*>(smem_raw + (kMisc - base));
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem_raw + (kLut - base));
+  Misc& ms = *reinterpret_cast<Misc*>(smem_raw + (LY::kMisc - base));
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem_raw + (LY::kLut - base));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rtiles = N / ROWS;
 
@@ -321,14 +423,24 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
     ms.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // byte b -> {fp16 L[b >> 4] (low half), fp16 L[b & 15] (high half)}, one
-  // 256-byte row per byte value, lane l's copy at 4 l (the upper 128 bytes of
-  // each row are unused)
+  // byte b -> its two weights as an fp16 pair, the lower k in the low half:
+  // NF4 {L[b >> 4], L[b & 15]}, MXFP4 {e2m1(b & 15), e2m1(b >> 4)}, INT4
+  // {1024 + (b >> 4), 1024 + (b & 15)} (0x6400 is fp16 1024, whose mantissa
+  // then holds the code).  One 256-byte row per byte value, lane l's copy at
+  // 4 l (the upper 128 bytes of each row are unused).
   for (int i = threadIdx.x; i < 256 * 32; i += THREADS) {
-    const int b = i >> 5, l = i & 31;
-    const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
-                                     __float2half_rn(c_levels_dec[b & 15]));
-    lut[b * 64 + l] = *reinterpret_cast<const uint32_t*>(&h);
+    const uint32_t b = (uint32_t)(i >> 5), l = (uint32_t)(i & 31);
+    uint32_t v;
+    if (FMT == kFmtNF4) {
+      const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
+                                       __float2half_rn(c_levels_dec[b & 15]));
+      v = *reinterpret_cast<const uint32_t*>(&h);
+    } else if (FMT == kFmtMXFP4) {
+      v = e2m1_h(b & 15u) | (e2m1_h(b >> 4) << 16);
+    } else {
+      v = (0x6400u | (b >> 4)) | ((0x6400u | (b & 15u)) << 16);
+    }
+    lut[b * 64 + l] = v;
   }
   if (warp == CWARPS) {
     // item_prefix[e] = sum over e' < e of ceil(count / TOK) * rtiles
@@ -361,12 +473,15 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
   __syncthreads();
   const int total = ms.nitems;
   const int KS = K / SK;
+  auto stage_addr = [](int s) -> uint32_t {
+    return s < 2 ? LY::kStage0 + s * LY::kStageBytes : LY::kStage2 + (s - 2) * LY::kStageBytes;
+  };
 
   if (warp == CWARPS) {
     // ---------------- producer
     if (lane == 0) {
       // the item's 128 weight rows as two 64-row halves (y, z .. z+1) of the
-      // 3-D weight and absmax maps: SwiGLU items take the gate rows and the
+      // 3-D weight (and absmax) maps: SwiGLU items take the gate rows and the
       // matching up rows (z = 2e + half), plain items 128 consecutive rows
       auto rows_of = [&](const Item& it, int& wy, int& wz) {
         if (EPI == MOE_EPI_SWIGLU) {
@@ -377,7 +492,12 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
           wz = it.expert * (N / (ROWS / 2)) + 2 * it.rtile;
         }
       };
-      // Chain mode: the weights and absmax of the first ring's worth of
+      auto issue_weights = [&](uint32_t sb, uint32_t full, int s, int wy, int wz, int nr8) {
+        mbar_arrive_expect_tx(full, kWBytes + LY::kA + nr8 * 4 * XBOX);
+        tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
+        if (FMT == kFmtNF4) tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
+      };
+      // Chain mode: the weights (and absmax) of the first ring's worth of
       // stages are requested before the previous kernel (which writes A) has
       // finished; their barriers already expect the activation bytes too.
       int pre = 0;
@@ -387,18 +507,13 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
           int wy, wz;
           rows_of(it, wy, wz);
           const int nr8 = (it.cnt + 7) / 8;
-          for (int s = 0; s < KS && pre < STAGES; ++s, ++pre) {
-            const uint32_t full = smem_u32(&ms.full[pre]);
-            const uint32_t sb = stage_addr(pre);
-            mbar_arrive_expect_tx(full, kWBytes + kABytes + nr8 * 4 * XBOX);
-            tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
-            tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
-          }
+          for (int s = 0; s < KS && pre < STAGES; ++s, ++pre)
+            issue_weights(stage_addr(pre), smem_u32(&ms.full[pre]), s, wy, wz, nr8);
         }
         pdl_wait();
         pdl_trigger();
       }
-      int stage = 0, g = 0;
+      int stage = 0, gi = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
@@ -407,14 +522,12 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
         rows_of(it, wy, wz);
         const int nr8 = (it.cnt + 7) / 8;
         const CUtensorMap* xmap = nr8 > 1 ? &xmap16 : &xmap8;
-        for (int s = 0; s < KS; ++s, ++g) {
+        for (int s = 0; s < KS; ++s, ++gi) {
           const uint32_t full = smem_u32(&ms.full[stage]);
           const uint32_t sb = stage_addr(stage);
-          if (g >= pre) {  // stages g < pre are slot g, phase 0, weights already requested
+          if (gi >= pre) {  // stages gi < pre are slot gi, phase 0, weights already requested
             if (!(ok = mbar_wait(smem_u32(&ms.empty[stage]), phase ^ 1, ms, dev_err))) break;
-            mbar_arrive_expect_tx(full, kWBytes + kABytes + nr8 * 4 * XBOX);
-            tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
-            tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
+            issue_weights(sb, full, s, wy, wz, nr8);
           }
           for (int b = 0; b < 4; ++b)
             tma_load_2d(sb + kWBytes + b * XKBOX, xmap, full, s * SK + b * kBlock, it.start);
@@ -430,9 +543,9 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
       const Item it = item_info(ms, offsets, E, rtiles, i);
       bool ok;
       if (it.cnt > 8)
-        ok = consume_item<EPI, OutT, 2>(ms, it, N, K, out, dev_err, stage, phase);
+        ok = consume_item<FMT, EPI, OutT, 2>(ms, it, N, K, gscales, out, dev_err, stage, phase);
       else
-        ok = consume_item<EPI, OutT, 1>(ms, it, N, K, out, dev_err, stage, phase);
+        ok = consume_item<FMT, EPI, OutT, 1>(ms, it, N, K, gscales, out, dev_err, stage, phase);
       if (!ok) break;
     }
   }
@@ -442,10 +555,11 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_decode_kernel(
 
 int sm_count() { return device_sm_count(); }
 
-template <int EPI, typename OutT>
-cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
+template <int FMT, int EPI, typename OutT>
+cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const void* scales,
                    const int32_t* offsets, int E, int N, int K, int M_total, void* out,
                    int32_t* dev_err, cudaStream_t s, bool chain) {
+  using LY = Layout<FMT>;
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
   CUtensorMap wmap, amap, xmap8, xmap16;
@@ -465,17 +579,20 @@ cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  {
+  if (FMT == kFmtNF4) {
     // the absmax of the same rows, 4 blocks (one stage) per row; the L2
     // fetches whole 128-byte lines, so later stages of a row hit in L2
     const cuuint64_t dims[3] = {(cuuint64_t)K / kBlock, ry, rz};
     const cuuint64_t strides[2] = {(cuuint64_t)K / kBlock * 4, ry * (K / kBlock) * 4};
     const cuuint32_t box[3] = {SK / kBlock, ROWS / 2, 2};
-    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(absmax), dims, strides,
-            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+            const_cast<float*>(static_cast<const float*>(scales)), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+  } else {
+    amap = wmap;  // unused
   }
   for (int rows : {8, 16}) {
     // routed activation rows: one 64-k block of 8 or 16 rows per box
@@ -488,28 +605,41 @@ cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const float
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t smem = kEnd;  // absolute layout; the window starts at or below 1 KB
-  auto kern = nf4_decode_kernel<EPI, OutT>;
+  const size_t smem = LY::kEnd;  // absolute layout; the window starts at or below 1 KB
+  auto kern = decode_kernel<FMT, EPI, OutT>;
   cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
   const int64_t max_items = ((int64_t)M_total / TOK + E) * (N / ROWS);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_items));
-  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, wmap, amap, xmap8, xmap16, offsets,
-                    E, N, K, M_total, reinterpret_cast<OutT*>(out), dev_err, chain ? 1 : 0);
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, wmap, amap, xmap8, xmap16, scales,
+                    offsets, E, N, K, M_total, reinterpret_cast<OutT*>(out), dev_err,
+                    chain ? 1 : 0);
 }
 
-template <int EPI>
-cudaError_t launch_out(const void* A, int A_rows, const uint8_t* packed, const float* absmax,
+template <int FMT, int EPI>
+cudaError_t launch_out(const void* A, int A_rows, const uint8_t* packed, const void* scales,
                        const int32_t* offsets, int E, int N, int K, int M_total, void* out,
                        moe_dtype_t out_dt, int32_t* dev_err, cudaStream_t s, bool chain) {
   if (out_dt == MOE_DT_F32)
-    return launch<EPI, float>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                              dev_err, s, chain);
+    return launch<FMT, EPI, float>(A, A_rows, packed, scales, offsets, E, N, K, M_total, out,
+                                   dev_err, s, chain);
   if (out_dt == MOE_DT_F16)
-    return launch<EPI, __half>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                               dev_err, s, chain);
-  return launch<EPI, __nv_bfloat16>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
+    return launch<FMT, EPI, __half>(A, A_rows, packed, scales, offsets, E, N, K, M_total, out,
                                     dev_err, s, chain);
+  return launch<FMT, EPI, __nv_bfloat16>(A, A_rows, packed, scales, offsets, E, N, K, M_total,
+                                         out, dev_err, s, chain);
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const void* A, int A_rows, const uint8_t* packed, const void* scales,
+                       const int32_t* offsets, int E, int N, int K, int M_total,
+                       moe_epilogue_t epi, void* out, moe_dtype_t out_dt, int32_t* dev_err,
+                       cudaStream_t s, bool chain) {
+  return epi == MOE_EPI_SWIGLU
+             ? launch_out<FMT, MOE_EPI_SWIGLU>(A, A_rows, packed, scales, offsets, E, N, K,
+                                               M_total, out, out_dt, dev_err, s, chain)
+             : launch_out<FMT, MOE_EPI_NONE>(A, A_rows, packed, scales, offsets, E, N, K, M_total,
+                                             out, out_dt, dev_err, s, chain);
 }
 
 }  // namespace dec
@@ -527,12 +657,32 @@ cudaError_t grouped_gemm_decode(const void* A, int A_rows, const uint8_t* packed
                                 const float* absmax, const int32_t* offsets, int E, int N, int K,
                                 int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
                                 int32_t* dev_err, cudaStream_t s, bool chain) {
-  using namespace moe::dec;
-  return epi == MOE_EPI_SWIGLU
-             ? launch_out<MOE_EPI_SWIGLU>(A, A_rows, packed, absmax, offsets, E, N, K, M_total,
-                                          out, out_dt, dev_err, s, chain)
-             : launch_out<MOE_EPI_NONE>(A, A_rows, packed, absmax, offsets, E, N, K, M_total, out,
-                                        out_dt, dev_err, s, chain);
+  return moe::dec::launch_fmt<moe::kFmtNF4>(A, A_rows, packed, absmax, offsets, E, N, K, M_total,
+                                            epi, out, out_dt, dev_err, s, chain);
+}
+
+bool grouped_gemm_int4_supported(int N, int K) {
+  return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
+}
+
+cudaError_t grouped_gemm_int4(const void* A, int A_rows, const uint8_t* packed,
+                              const uint32_t* meta, const int32_t* offsets, int E, int N, int K,
+                              int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
+                              int32_t* dev_err, cudaStream_t s) {
+  return moe::dec::launch_fmt<moe::kFmtINT4>(A, A_rows, packed, meta, offsets, E, N, K, M_total,
+                                             epi, out, out_dt, dev_err, s, false);
+}
+
+bool grouped_gemm_mxfp4_supported(int N, int K) {
+  return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
+}
+
+cudaError_t grouped_gemm_mxfp4(const void* A, int A_rows, const uint8_t* packed,
+                               const uint8_t* scales, const int32_t* offsets, int E, int N, int K,
+                               int M_total, moe_epilogue_t epi, void* out, moe_dtype_t out_dt,
+                               int32_t* dev_err, cudaStream_t s) {
+  return moe::dec::launch_fmt<moe::kFmtMXFP4>(A, A_rows, packed, scales, offsets, E, N, K,
+                                              M_total, epi, out, out_dt, dev_err, s, false);
 }
 
 }  // namespace moe_launch

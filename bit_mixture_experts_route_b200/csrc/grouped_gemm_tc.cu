@@ -644,27 +644,35 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   } else if (warp == W_RPROD) {
     // ---------------- TMA producer: packed NF4 rows of the tile
     if (lane == 0) {
-      int rs = 0;
-      uint32_t rph = 0;
-      bool ok = true;
-      for (int t = t0; t < total && ok; t += tstep) {
+      // tile t's 128-row weight sub-tile of this CTA (wt) and the first weight
+      // row of each 64-row box (forward: gate and up rows with SwiGLU,
+      // consecutive rows without; transposed: the expert's first row)
+      auto tile_rows = [&](int t, int& wt, int& y0, int& y1) {
         const TileId id = tile_id(sm, E, n_tiles, t);
-        const int wt = id.ntile * PAIR + rank;  // this CTA's 128-row weight sub-tile
-        int y0, y1;  // first weight row of each 64-row box
-        if (EPI == MOE_EPI_SWIGLU) {
+        wt = id.ntile * PAIR + rank;
+        if (TR) {
+          y0 = y1 = id.expert * N;
+        } else if (EPI == MOE_EPI_SWIGLU) {
           y0 = id.expert * N + wt * (BM / 2);  // gate rows
           y1 = y0 + N / 2;                     // matching up rows
         } else {
           y0 = id.expert * N + wt * BM;
           y1 = y0 + BM / 2;
         }
+      };
+      int rs = 0;
+      uint32_t rph = 0;
+      bool ok = true;
+      for (int t = t0; t < total && ok; t += tstep) {
+        int wt, y0, y1;
+        tile_rows(t, wt, y0, y1);
         for (int ks = 0; ks < KT; ++ks) {
           if (!(ok = mbar_wait(&sm.raw_empty[rs], rph ^ 1, sm, dev_err))) break;
           if (TR) {
             // weight rows n = 64 ks .. 64 ks + 63 of the expert, the packed
             // bytes of columns 128 wt .. 128 wt + 127, and the absmax of their
             // two 64-blocks (4 per row from a 16-byte-aligned block index)
-            const int yr = id.expert * N + ks * BK;
+            const int yr = y0 + ks * BK;
             mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE_T);
             tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], wt * (BM / 2), yr);
             tma_load_2d(sm.raw[rs] + RAW_STAGE, &amap, &sm.raw_full[rs], (2 * wt) & ~3, yr);
@@ -703,7 +711,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       const uint32_t sel = (m & 1) ? 0x7632u : 0x5410u;
       bool bad_scale = false;
       for (int S = g; ; S += GROUPS) {
-        const int lt_ = S / KT, ks = S - lt_ * KT;
+        const int lt_ = S / KT;
         const int t = t0 + lt_ * tstep;
         if (t >= total) break;
         const TileId id = tile_id(sm, E, n_tiles, t);
