@@ -252,6 +252,14 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {
   asm volatile(
@@ -441,7 +449,7 @@ __device__ __forceinline__ void stage_scales(uint32_t sc, uint32_t& h0, uint32_t
 // gradient of h) and writes the gradient of gate_up's pre-activations.
 template <int FMT, int EPI, typename OutT, int PAIR, bool TR>
 __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
-    const __grid_constant__ CUtensorMap bmap,
+    const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap bmap2,
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
     const void* __restrict__ scales, const int32_t* __restrict__ offsets, int E, int N, int K,
     int M_total, OutT* __restrict__ out, const float* __restrict__ gu, int32_t* dev_err,
@@ -584,14 +592,12 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
           // leader: its own barrier; the pair's peer: the leader's
           const uint32_t bar = leader ? smem_u32(rdy) : cluster_addr(rdy, 0);
           if (leader) mbar_arrive_expect_tx(rdy, PAIR * boxes * B_BOX_BYTES);
-          for (int b = 0; b < boxes; ++b) {
-            if (PAIR == 1)
-              tma_load_2d(sm.b[bs] + b * B_BOX_BYTES, &bmap, rdy, ks * BK,
-                          brow0 + b * B_BOX_ROWS);
-            else
-              tma_load_2d_pair(sm.b[bs] + b * B_BOX_BYTES, &bmap, bar, ks * BK,
-                               brow0 + b * B_BOX_ROWS);
-          }
+          // one copy per stage: a 128-row box, or a 256-row box (bmap2)
+          const CUtensorMap* bm = boxes == 2 ? &bmap2 : &bmap;
+          if (PAIR == 1)
+            tma_load_2d(sm.b[bs], bm, rdy, ks * BK, brow0);
+          else
+            tma_load_2d_pair(sm.b[bs], bm, bar, ks * BK, brow0);
           if (++bs == BSTAGES) bs = 0;
         }
       }
@@ -644,20 +650,21 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
   } else if (warp == W_RPROD) {
     // ---------------- TMA producer: packed NF4 rows of the tile
     if (lane == 0) {
-      // tile t's 128-row weight sub-tile of this CTA (wt) and the first weight
-      // row of each 64-row box (forward: gate and up rows with SwiGLU,
-      // consecutive rows without; transposed: the expert's first row)
+      // tile t's 128-row weight sub-tile of this CTA (wt) and the box
+      // coordinates of its rows: forward SwiGLU y1 = z of the expert's gate
+      // half; forward plain y0 = the first of 128 consecutive rows;
+      // transposed y0 = the expert's first row
       auto tile_rows = [&](int t, int& wt, int& y0, int& y1) {
         const TileId id = tile_id(sm, E, n_tiles, t);
         wt = id.ntile * PAIR + rank;
         if (TR) {
           y0 = y1 = id.expert * N;
         } else if (EPI == MOE_EPI_SWIGLU) {
-          y0 = id.expert * N + wt * (BM / 2);  // gate rows
-          y1 = y0 + N / 2;                     // matching up rows
+          y0 = 0;
+          y1 = 2 * id.expert;  // z of the expert's gate half
         } else {
           y0 = id.expert * N + wt * BM;
-          y1 = y0 + BM / 2;
+          y1 = 0;
         }
       };
       int rs = 0;
@@ -676,11 +683,15 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
             mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE_T);
             tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], wt * (BM / 2), yr);
             tma_load_2d(sm.raw[rs] + RAW_STAGE, &amap, &sm.raw_full[rs], (2 * wt) & ~3, yr);
+          } else if (EPI == MOE_EPI_SWIGLU) {
+            // one 3-D box: the 64 gate rows, then the 64 matching up rows
+            // (weight rows as [2E][N/2][K/2]: z = 2 expert + half)
+            mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE);
+            tma_load_3d(sm.raw[rs], &wmap, &sm.raw_full[rs], ks * (BK / 2), wt * (BM / 2), y1);
           } else {
+            // one box of the tile's 128 consecutive rows
             mbar_arrive_expect_tx(&sm.raw_full[rs], RAW_STAGE);
             tma_load_2d(sm.raw[rs], &wmap, &sm.raw_full[rs], ks * (BK / 2), y0);
-            tma_load_2d(sm.raw[rs] + (BM / 2) * (BK / 2), &wmap, &sm.raw_full[rs],
-                        ks * (BK / 2), y1);
           }
           if (++rs == RAW_RING) { rs = 0; rph ^= 1; }
         }
@@ -1014,23 +1025,35 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
                    int32_t* dev_err, cudaStream_t s, bool chain) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
-  CUtensorMap map, wmap;
-  const cuuint32_t estr[2] = {1, 1};
-  {
+  CUtensorMap map, map2, wmap;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  for (int rows : {B_BOX_ROWS, 2 * B_BOX_ROWS}) {
+    // routed activation rows: boxes of 64 k x 128 or 256 rows
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M_total};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {BK, B_BOX_ROWS};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(A),
-            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const cuuint32_t box[2] = {BK, (cuuint32_t)rows};
+    if (enc(rows == B_BOX_ROWS ? &map : &map2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  if (EPI == MOE_EPI_SWIGLU) {
+    // packed rows as [2E][N/2][K/2] (z = 2 expert + half); box = 32 bytes x
+    // 64 rows x 2 halves: a stage's gate rows and their up rows in one copy
+    const cuuint64_t dims[3] = {(cuuint64_t)K / 2, (cuuint64_t)N / 2, (cuuint64_t)2 * E};
+    const cuuint64_t strides[2] = {(cuuint64_t)K / 2, (cuuint64_t)(N / 2) * (K / 2)};
+    const cuuint32_t box[3] = {BK / 2, BM / 2, 2};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-  }
-  {
-    // packed rows as a 2-D byte tensor [E*N, K/2]; box = 32 bytes x 64 rows
+  } else {
+    // packed rows as a 2-D byte tensor [E*N, K/2]; box = 32 bytes x 128 rows
     const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)E * N};
     const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
-    const cuuint32_t box[2] = {BK / 2, BM / 2};
+    const cuuint32_t box[2] = {BK / 2, BM};
     if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
@@ -1046,7 +1069,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
   const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / (BM * PAIR));
   if (PAIR == 1) {
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, wmap, wmap, scales,
+    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, map2, wmap, wmap, scales,
                       offsets, E, N, K, M_total, reinterpret_cast<OutT*>(out),
                       static_cast<const float*>(nullptr), dev_err, chain ? 1 : 0);
   }
@@ -1067,7 +1090,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map, wmap, wmap, scales, offsets, E, N, K, M_total,
+  return cudaLaunchKernelEx(&cfg, kern, map, map2, wmap, wmap, scales, offsets, E, N, K, M_total,
                             reinterpret_cast<OutT*>(out), static_cast<const float*>(nullptr),
                             dev_err, chain ? 1 : 0);
 }
@@ -1081,16 +1104,16 @@ cudaError_t launch_t(const void* G, int G_rows, const uint8_t* packed, const flo
                      const float* gu, int32_t* dev_err, cudaStream_t s) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
-  CUtensorMap map, wmap, amap;
+  CUtensorMap map, map2, wmap, amap;
   const cuuint32_t estr[2] = {1, 1};
-  {
+  for (int rows : {B_BOX_ROWS, 2 * B_BOX_ROWS}) {
     const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G_rows};
     const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
-    const cuuint32_t box[2] = {BK, B_BOX_ROWS};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(G),
-            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-        CUDA_SUCCESS)
+    const cuuint32_t box[2] = {BK, (cuuint32_t)rows};
+    if (enc(rows == B_BOX_ROWS ? &map : &map2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(G), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   {
@@ -1121,7 +1144,7 @@ cudaError_t launch_t(const void* G, int G_rows, const uint8_t* packed, const flo
   if (err != cudaSuccess) return err;
   const int64_t max_tiles = ((int64_t)M_total / BN + E) * (K / BM);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, wmap, amap,
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, map2, wmap, amap,
                     static_cast<const void*>(absmax), offsets, E, N, K, M_total,
                     reinterpret_cast<OutT*>(out), gu, dev_err, 0);
 }
