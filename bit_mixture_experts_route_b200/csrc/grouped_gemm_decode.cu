@@ -23,8 +23,8 @@
 // * One producer thread streams each item through a 5-stage ring with TMA
 //   tile loads, 256 k per stage: the packed rows (one 3-D box of 2 x 64 rows x
 //   128 bytes), for NF4 their absmax (one 3-D box of 2 x 64 rows x 4 fp32) and
-//   the routed activation rows (one box of 8 or 16 rows per 64-k block), with
-//   128-byte swizzle.
+//   the routed activation rows (one 3-D box of the stage's four 64-k blocks x
+//   8 or 16 rows), with 128-byte swizzle: three copies per stage.
 // * Eight consumer warps each own 16 weight rows of the item and run
 //   mma.sync.m16n8k16 with the weights as the M side and the routed rows as N
 //   (swap-AB); the four 64-k blocks of a stage run as four interleaved MMA
@@ -57,7 +57,7 @@ constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int SB = SK / 2;      // packed bytes per row per stage
 constexpr int STAGES = 5;
-constexpr int CWARPS = 8;       // two row groups x four k blocks
+constexpr int CWARPS = 8;       // consumer warps, 16 weight rows each
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr int XBOX = 8 * 64 * 2;                 // one 8-row x 64-k fp16 box
@@ -314,7 +314,7 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
     for (int b = 0; b < 4; ++b) {
 #pragma unroll
       for (int j = 0; j < NT8; ++j) {
-        const uint32_t line = xst + b * XKBOX + (8 * j + g) * 128;
+        const uint32_t line = xst + b * (NT8 * XBOX) + (8 * j + g) * 128;
         const uint4 u = lds128(line + xo0), v = lds128(line + xo1);
         xf[b][j][0] = u.x; xf[b][j][1] = u.y; xf[b][j][2] = u.z; xf[b][j][3] = u.w;
         xf[b][j][4] = v.x; xf[b][j][5] = v.y; xf[b][j][6] = v.z; xf[b][j][7] = v.w;
@@ -529,8 +529,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
             if (!(ok = mbar_wait(smem_u32(&ms.empty[stage]), phase ^ 1, ms, dev_err))) break;
             issue_weights(sb, full, s, wy, wz, nr8);
           }
-          for (int b = 0; b < 4; ++b)
-            tma_load_2d(sb + kWBytes + b * XKBOX, xmap, full, s * SK + b * kBlock, it.start);
+          // the stage's four 64-k blocks of the routed rows in one 3-D box
+          tma_load_3d(sb + kWBytes, xmap, full, 0, it.start, s * (SK / kBlock));
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -595,11 +595,13 @@ cudaError_t launch(const void* A, int A_rows, const uint8_t* packed, const void*
     amap = wmap;  // unused
   }
   for (int rows : {8, 16}) {
-    // routed activation rows: one 64-k block of 8 or 16 rows per box
-    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)A_rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {kBlock, (cuuint32_t)rows};
-    if (enc(rows == 8 ? &xmap8 : &xmap16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+    // routed activation rows as [K/64 blocks][rows][64 k]: one box of 4
+    // blocks x 8 or 16 rows x 64 k is a stage's activations, laid out block
+    // after block (8 or 16 swizzled 128-byte rows each)
+    const cuuint64_t dims[3] = {(cuuint64_t)kBlock, (cuuint64_t)A_rows, (cuuint64_t)K / kBlock};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)kBlock * 2};
+    const cuuint32_t box[3] = {kBlock, (cuuint32_t)rows, SK / kBlock};
+    if (enc(rows == 8 ? &xmap8 : &xmap16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
             const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
