@@ -799,38 +799,71 @@ def main():
     head = run_workload(wl, workload_name, args, args.steps, world, local, hbm, tf_burst,
                         tf_sust, peak_kind)
 
-    # ---- end to end through the one-call C API with host buffers
+    # ---- end to end through the one-call C API with host buffers: every
+    # step copies its inputs from pinned host memory and its output back.
+    # The plain NF4 layer runs two steps in flight (double-buffered inputs and
+    # output; uploads and downloads on two more streams, so PCIe runs both
+    # directions at once), as a serving loop overlaps the next batch's upload
+    # and the last batch's download with the current compute; the other paths
+    # copy and compute on one stream.
     X_h = wl.X.cpu().pin_memory()
     L_h = wl.logits.cpu().pin_memory()
-    Y_h = torch.empty((T, shape.H), dtype=torch.float32).pin_memory()
-    X_d, L_d = torch.empty_like(wl.X), torch.empty_like(wl.logits)
+    pipelined = wl.fmt == "nf4" and not (wl.lora or wl.backward)
+    nbuf = 2 if pipelined else 1
+    Y_h = [torch.empty((T, shape.H), dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    X_d = [torch.empty_like(wl.X) for _ in range(nbuf)]
+    L_d = [torch.empty_like(wl.logits) for _ in range(nbuf)]
+    Y_d = [torch.empty((T, shape.H), dtype=torch.float32, device=wl.X.device)
+           for _ in range(nbuf)]
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_free = [torch.cuda.Event() for _ in range(nbuf)]
 
-    def e2e_step():
-        X_d.copy_(X_h, non_blocking=True)
-        L_d.copy_(L_h, non_blocking=True)
+    def e2e_step(s):
+        b = s % nbuf
+        if not pipelined:  # the calls one by one, copies on the compute stream
+            X_d[0].copy_(X_h, non_blocking=True)
+            L_d[0].copy_(L_h, non_blocking=True)
+            for layer in range(layers):
+                wl.layer(layer, args.algo, X=X_d[0], logits=L_d[0][layer])
+            Y_h[0].copy_(wl.Y, non_blocking=True)
+            return
+        with torch.cuda.stream(up):
+            up.wait_event(ev_free[b])  # step s - 2 is done with buffer b
+            X_d[b].copy_(X_h, non_blocking=True)
+            L_d[b].copy_(L_h, non_blocking=True)
+            ev_in[b].record(up)
+        comp.wait_event(ev_in[b])
         for layer in range(layers):
-            if wl.fmt != "nf4" or wl.lora or wl.backward:  # the calls one by one
-                wl.layer(layer, args.algo, X=X_d, logits=L_d[layer])
-            else:
-                moe.layer_forward(X_d, L_d[layer], shape.k, shape.renormalize,
-                                  *wl.stacks[layer], workspace=wl.lws, out=wl.Y)
-        Y_h.copy_(wl.Y, non_blocking=True)
+            moe.layer_forward(X_d[b], L_d[b][layer], shape.k, shape.renormalize,
+                              *wl.stacks[layer], workspace=wl.lws, out=Y_d[b])
+        ev_out[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_out[b])
+            Y_h[b].copy_(Y_d[b], non_blocking=True)
+            ev_free[b].record(down)
 
-    for _ in range(3):
-        e2e_step()
+    for s in range(3):
+        e2e_step(s)
     torch.cuda.synchronize()
     es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
-    es.record()
-    for _ in range(args.steps):
-        e2e_step()
-    ee.record()
+    es.record(comp)
+    for s in range(args.steps):
+        e2e_step(3 + s)
+    comp.wait_stream(down)  # the last step's output is on the host
+    ee.record(comp)
     torch.cuda.synchronize()
     ems = max_over_ranks(es.elapsed_time(ee), world)
     e2e = {"value": world * T * layers * args.steps / (ems / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": X_h.numel() * 2 + L_h.numel() * 4,
-           "d2h_bytes_per_step": Y_h.numel() * 4,
-           "path": "moe_layer_forward per layer (C ABI), pinned host X and logits in, Y out"}
+           "d2h_bytes_per_step": Y_h[0].numel() * 4,
+           "path": ("moe_layer_forward per layer (C ABI), pinned host X and logits in, Y out; "
+                    + ("two steps in flight, uploads and downloads on their own streams"
+                       if pipelined
+                       else "copies and compute on one stream"))}
     del wl
     torch.cuda.empty_cache()
 

@@ -108,3 +108,13 @@ def test_gate_up_bytes_accounting(weights, lora, backward):
         M = T * sh.k
         want = 64 * lora * (sh.H + 2 * sh.I) * 2 + M * sh.H * 2 + 2 * M * 2 * sh.I * 4
         assert wl.lora_bytes(64) == want
+
+
+def test_a_device_fault_is_not_taken_for_a_capture_failure():
+    # graph capture failures are recorded and the eager timing is reported;
+    # a fault on the device must surface instead (the context is lost)
+    assert bench._cuda_fault(RuntimeError("CUDA error: unspecified launch failure"))
+    assert bench._cuda_fault(RuntimeError("CUDA error: an illegal memory access was encountered"))
+    assert bench._cuda_fault(RuntimeError("CUDA error: misaligned address"))
+    assert not bench._cuda_fault(RuntimeError("operation not permitted when stream is capturing"))
+    assert not bench._cuda_fault(RuntimeError("moe_layer_forward: workspace too small"))
