@@ -584,8 +584,11 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
         for (int ks = 0; ks < KT; ++ks, ++S) {
           if (S >= BSTAGES) {
             const int P = S - BSTAGES;
-            if (!(ok = mbar_wait<PAIR == 2>(&sm.a_empty[P % RING], (uint32_t)(P / RING) & 1u, sm,
-                                            dev_err)))
+            // this thread paces the ring: it polls (single CTA) rather than
+            // sleep in the barrier unit
+            const uint32_t par = (uint32_t)(P / RING) & 1u;
+            if (!(ok = PAIR == 1 ? mbar_poll(&sm.a_empty[P % RING], par, sm, dev_err)
+                                 : mbar_wait<true>(&sm.a_empty[P % RING], par, sm, dev_err)))
               break;
           }
           uint64_t* rdy = &sm.ready[S % RING];
