@@ -123,3 +123,29 @@ def test_int4_tc_grouped_gemm_ragged(epi, counts):
     if epi == "swiglu":
         ref = oracle.swiglu(ref)
     assert_close(out.cpu().numpy(), ref, f"int4 tc {epi} {counts}")
+
+
+@pytest.mark.parametrize("N,K,epi", [(1536, 2048, "swiglu"), (2048, 768, "none")],
+                         ids=["gate_up", "down"])
+def test_int4_decode_at_qwen3_30b_projection_sizes(N, K, epi):
+    # the decode pipeline's INT4 form at the Qwen3-30B-A3B projection sizes
+    # (12 and 16 row tiles, 8 and 3 stages per item), three experts with 1, 0
+    # and 19 routed rows (two items for the last)
+    counts = [1, 0, 19]
+    E = len(counts)
+    off = _ragged(counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(N + K)
+    W = torch.randn((E, N, K), generator=g) * 0.02
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    packed, meta = moe.int4_quantize(W.cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.int4_grouped_gemm(X.cuda(), packed, meta, torch.from_numpy(off).cuda(), M,
+                                epilogue=epi, out_dtype=torch.float32, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    p_ref, m_ref = oracle.quantize_int4_grouped(W.numpy())
+    ref = oracle.grouped_gemm_int4(X.float().numpy(), p_ref, m_ref, off)
+    if epi == "swiglu":
+        ref = oracle.swiglu(ref)
+    assert_close(_np(out), ref, f"int4 30b {epi}")

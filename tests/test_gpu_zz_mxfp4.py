@@ -200,3 +200,29 @@ def test_mxfp4_layer_qwen3_30b_prefill_tc_sampled():
     ref = oracle.moe_layer(X.float().numpy(), lg.numpy(), stack, shape.k, shape.renormalize,
                            tokens=toks)
     assert_close(_np(Y)[toks], ref, "mxfp4 qwen3-30b prefill (tensor cores)")
+
+
+@pytest.mark.parametrize("N,K,epi", [(1536, 2048, "swiglu"), (2048, 768, "none")],
+                         ids=["gate_up", "down"])
+def test_mxfp4_decode_at_qwen3_30b_projection_sizes(N, K, epi):
+    # the decode pipeline's MXFP4 form at the Qwen3-30B-A3B projection sizes
+    # (12 and 16 row tiles, 8 and 3 stages per item), three experts with 1, 0
+    # and 19 routed rows (two items for the last)
+    counts = [1, 0, 19]
+    E = len(counts)
+    off = _ragged(counts)
+    M = int(off[-1])
+    g = torch.Generator().manual_seed(N + K + 1)
+    W = torch.randn((E, N, K), generator=g) * 0.02
+    X = torch.randn((M, K), generator=g).to(torch.float16)
+    packed, scales = moe.mxfp4_quantize(W.cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.mxfp4_grouped_gemm(X.cuda(), packed, scales, torch.from_numpy(off).cuda(), M,
+                                 epilogue=epi, out_dtype=torch.float32, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    p_ref, s_ref = oracle.quantize_mxfp4(W.numpy())
+    ref = oracle.grouped_gemm_mxfp4(X.float().numpy(), p_ref, s_ref, off)
+    if epi == "swiglu":
+        ref = oracle.swiglu(ref)
+    assert_close(_np(out), ref, f"mxfp4 30b {epi}")
