@@ -55,6 +55,8 @@
 // the leader's commits arrive on both CTAs' barriers (.multicast::cluster);
 // the peer's epilogue hands the accumulator back with remote arrives.  No
 // TMA load uses multicast.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace moe {
@@ -63,7 +65,6 @@ namespace tc {
 constexpr int BM = 128;          // weight rows per tile (MMA M)
 constexpr int BN = 256;          // routed rows per tile (max MMA N)
 constexpr int BK = 64;           // k per stage = one NF4 block
-constexpr int BSTAGES = 3;       // activation ring (shared memory)
 constexpr int B_BOX_ROWS = 128;        // TMA box: 64 k x 128 rows
 constexpr int B_BOX_BYTES = B_BOX_ROWS * BK * 2;  // 16 KB
 constexpr int B_STAGE = BN * BK * 2;   // 32 KB: a tile's routed rows, two boxes
@@ -84,22 +85,25 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;             // accumulator: columns [0, 256)
 constexpr int A_COL = BN;              // decoded-weight slot a: columns 256 + 32 a
 constexpr int A_SLOT_COLS = BK / 2;
-constexpr int STG_BYTES = 32 * 32 * 4; // epilogue transpose buffer per warp
+constexpr int STG_BYTES = 32 * 32 * 4; // epilogue transpose buffer per warp (fp32 rows)
 constexpr uint32_t kWaitLimit = 1u << 20;  // suspended tries before a wait gives up
 constexpr uint32_t kSuspendNs = 1000;       // longest sleep of one try
 static_assert(A_COL + RING * A_SLOT_COLS <= TMEM_COLS, "tensor memory budget");
-static_assert(BSTAGES * B_STAGE + RAW_RING * RAW_STAGE_T + EPI_WARPS * STG_BYTES + 256 * 32 * 4 +
-                      2 * 1025 * 4 + 1024 <
-                  227 * 1024,
-              "shared memory budget");
-static_assert(BSTAGES < RING, "activation slots are released through the TMEM-slot barriers");
 static_assert(RING % GROUPS == 0 && RAW_RING % GROUPS == 0,
               "a group always meets its own slots");
 
-struct __align__(8) Smem {
-  uint8_t b[BSTAGES][B_STAGE];  // 1024-aligned (struct placed at 1024)
-  uint8_t raw[RAW_RING][RAW_STAGE_T];
-  uint8_t stg[EPI_WARPS][STG_BYTES];
+// Shared memory of one kernel form.  The activation producer can only run
+// NBS stages ahead of the MMAs (it refills a stage's slot once that stage's
+// MMAs are done), so a form takes as many 32-KB activation stages as its
+// packed-row slots (RAWB: 4 KB, or 5 KB with the transposed form's absmax)
+// and epilogue transpose buffers (STGB per warp: 32 rows of 32 outputs) leave
+// room for: 4 for the forward form with 16-bit outputs, 3 otherwise.
+template <int NBS, int RAWB, int STGB>
+struct __align__(8) SmemT {
+  static constexpr int kNBS = NBS;
+  uint8_t b[NBS][B_STAGE];  // 1024-aligned (struct placed at 1024)
+  uint8_t raw[RAW_RING][RAWB];
+  uint8_t stg[EPI_WARPS][STGB];
   uint32_t lut[256 * 32];
   uint64_t raw_full[RAW_RING], raw_empty[RAW_RING];
   // ready[s]: stage s's decoded weights (four decoder-warp arrivals) and its
@@ -113,6 +117,13 @@ struct __align__(8) Smem {
   int tile_prefix[1025];
   int off[1025];  // expert_offsets, copied once
 };
+template <typename OutT, bool TR>
+using SmemFor = typename std::conditional<(sizeof(OutT) == 2 && !TR), SmemT<4, RAW_STAGE, 2048>,
+                                          SmemT<3, RAW_STAGE_T, STG_BYTES>>::type;
+static_assert(sizeof(SmemT<4, RAW_STAGE, 2048>) + 1024 <= 227 * 1024, "shared memory budget");
+static_assert(sizeof(SmemT<3, RAW_STAGE_T, STG_BYTES>) + 1024 <= 227 * 1024,
+              "shared memory budget");
+static_assert(4 < RING, "activation slots are released through the TMEM-slot barriers");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -199,7 +210,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 constexpr uint32_t kPollLimit = 1u << 26;  // polls before a polled wait gives up (~1 s)
 
 // Bounded polled wait (see mbar_wait), for the single MMA-issuing thread.
-__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, Smem& sm,
+template <class SM>
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, SM& sm,
                                           int32_t* dev_err) {
   for (uint32_t i = 0; i < kPollLimit; ++i) {
     if (mbar_test_wait(bar, parity)) return true;
@@ -213,8 +225,8 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, Smem& 
 // Bounded wait: false (and the abort flag set) if the phase never completes
 // (kWaitLimit suspended tries, well under a second each way) or another role
 // already aborted.  CLUSTER: acquire at cluster scope.
-template <bool CLUSTER = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem& sm,
+template <bool CLUSTER = false, class SM>
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SM& sm,
                                           int32_t* dev_err) {
   if (CLUSTER ? mbar_try_wait_cl(bar, parity) : mbar_try_wait(bar, parity)) return true;
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
@@ -393,7 +405,8 @@ __constant__ float c_levels_tc[16] = {MOE_NF4_LEVEL_LIST};
 struct TileId {
   int expert, ntile, ttile;
 };
-__device__ __forceinline__ TileId tile_id(const Smem& sm, int E, int n_tiles, int t) {
+template <class SM>
+__device__ __forceinline__ TileId tile_id(const SM& sm, int E, int n_tiles, int t) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -407,7 +420,8 @@ __device__ __forceinline__ TileId tile_id(const Smem& sm, int E, int n_tiles, in
 struct TileInfo {
   int expert, row0, nrows, ntile;
 };
-__device__ __forceinline__ TileInfo tile_info(const Smem& sm, int E, int n_tiles, int t) {
+template <class SM>
+__device__ __forceinline__ TileInfo tile_info(const SM& sm, int E, int n_tiles, int t) {
   const TileId id = tile_id(sm, E, n_tiles, t);
   TileInfo ti;
   ti.expert = id.expert;
@@ -459,6 +473,8 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
     pdl_wait();
     pdl_trigger();
   }
+  using Smem = SmemFor<OutT, TR>;
+  constexpr int BSTAGES = Smem::kNBS;
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1063,7 +1079,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t smem = sizeof(Smem) + 1024;
+  const size_t smem = sizeof(SmemFor<OutT, false>) + 1024;
   auto kern = nf4_tc_kernel<FMT, EPI, OutT, PAIR, false>;
   cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
@@ -1141,7 +1157,7 @@ cudaError_t launch_t(const void* G, int G_rows, const uint8_t* packed, const flo
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t smem = sizeof(Smem) + 1024;
+  const size_t smem = sizeof(SmemFor<OutT, true>) + 1024;
   auto kern = nf4_tc_kernel<kFmtNF4, EPI, OutT, 1, true>;
   cudaError_t err = set_max_dynamic_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
   if (err != cudaSuccess) return err;
