@@ -20,12 +20,15 @@
 // * Persistent CTAs (one per SM) walk a list of work items built on the
 //   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
 //   rows; an expert with more routed rows yields one item per 16).
-// * One producer thread streams each item through a 5-stage ring with TMA
-//   tile loads, 256 k per stage: the packed rows (one 3-D box of 2 x 64 rows x
-//   128 bytes), for NF4 their absmax (one 3-D box of 2 x 64 rows x 4 fp32) and
-//   the routed activation rows (one 3-D box of the stage's four 64-k blocks x
-//   8 or 16 rows), with 128-byte swizzle: three copies per stage.
-// * Eight consumer warps each own 16 weight rows of the item and run
+// * Two consumer groups of eight warps take alternate items of the CTA's list,
+//   each through its own ring of stage slots (three and two of five).  One
+//   producer thread serves both rings, polling whichever group's next slot is
+//   free, with TMA tile loads, 256 k per stage: the packed rows (one 3-D box of
+//   2 x 64 rows x 128 bytes), for NF4 their absmax (one 3-D box of 2 x 64 rows
+//   x 4 fp32) and the routed activation rows (one 3-D box of the stage's four
+//   64-k blocks x 8 or 16 rows), with 128-byte swizzle: three copies per
+//   stage.  (17 warps leave 96 registers per thread.)
+// * The eight warps of a group each own 16 weight rows of the item and run
 //   mma.sync.m16n8k16 with the weights as the M side and the routed rows as N
 //   (swap-AB); the four 64-k blocks of a stage run as four interleaved MMA
 //   chains.  A lane turns each packed byte into an fp16 pair through ONE
@@ -55,10 +58,14 @@ namespace dec {
 constexpr int ROWS = 128;       // weight rows per item
 constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
+constexpr int kNAlign = 128;    // N granularity of the entry points (as the tensor-core form)
 constexpr int SB = SK / 2;      // packed bytes per row per stage
-constexpr int STAGES = 5;
-constexpr int CWARPS = 8;       // consumer warps, 16 weight rows each
-constexpr int THREADS = 32 * (CWARPS + 1);
+constexpr int CWARPS = ROWS / 16;  // consumer warps per group, 16 weight rows each
+constexpr int GROUPS = 2;       // consumer groups, each on its own items and ring
+constexpr int NSLOTS = 5;       // stage slots, both groups
+constexpr int kLoSlots = 2;     // slots below the table
+constexpr int PWARP = GROUPS * CWARPS;           // the producer warp
+constexpr int THREADS = 32 * (PWARP + 1);
 constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr int XBOX = 8 * 64 * 2;                 // one 8-row x 64-k fp16 box
 constexpr int XKBOX = (TOK / 8) * XBOX;          // 16 rows x 64 k
@@ -75,22 +82,37 @@ struct Layout {
   // Absolute shared-memory layout.  The dynamic window must start at or
   // below 1 KB (checked at run time).  Stages need 1 KB alignment (128-byte
   // swizzle).
-  static constexpr uint32_t kStage0 = 1024;                      // stages 0-1
-  static constexpr uint32_t kMisc = kStage0 + 2 * kStageBytes;   // barriers, item list
-  static constexpr uint32_t kLut = 65536;                        // table: 256 x 256 B
-  static constexpr uint32_t kStage2 = 2 * 65536;                 // stages 2-4
-  static constexpr uint32_t kEnd = kStage2 + (STAGES - 2) * kStageBytes;
+  static constexpr uint32_t kStage0 = 1024;                            // low slots
+  static constexpr uint32_t kMisc = kStage0 + kLoSlots * kStageBytes;  // barriers, item list
+  static constexpr uint32_t kLut = 65536;                              // table: 256 x 256 B
+  static constexpr uint32_t kStage2 = 2 * 65536;                       // high slots
+  static constexpr uint32_t kEnd = kStage2 + (NSLOTS - kLoSlots) * kStageBytes;
+  static __host__ __device__ constexpr uint32_t slot_addr(int slot) {
+    return slot < kLoSlots ? kStage0 + slot * kStageBytes
+                           : kStage2 + (slot - kLoSlots) * kStageBytes;
+  }
 };
 
 struct Misc {
-  uint64_t full[STAGES], empty[STAGES];
+  uint64_t full[NSLOTS], empty[NSLOTS];
   int abort_flag;
   int nitems;
   int item_prefix[1025];
+  int off[1025];  // expert_offsets, copied once (item lookups never touch global memory)
 };
 static_assert(Layout<kFmtNF4>::kMisc + sizeof(Misc) <= Layout<kFmtNF4>::kLut,
               "shared layout overlap");
 static_assert(Layout<kFmtNF4>::kEnd <= 227 * 1024 + 1024, "shared layout too large");
+static_assert(Layout<kFmtINT4>::kEnd <= 227 * 1024 + 1024, "shared layout too large");
+
+// Ring slots of consumer group g: [ring_base(g), ring_base(g) + ring_size(g)),
+// consecutive runs of ceil(NSLOTS / GROUPS) slots (the last run may be shorter).
+constexpr int kPerGroup = (NSLOTS + GROUPS - 1) / GROUPS;
+static_assert(NSLOTS - (GROUPS - 1) * kPerGroup >= 2, "every ring needs two slots");
+__host__ __device__ constexpr int ring_base(int g) { return g * kPerGroup; }
+__host__ __device__ constexpr int ring_size(int g) {
+  return NSLOTS - g * kPerGroup < kPerGroup ? NSLOTS - g * kPerGroup : kPerGroup;
+}
 
 __constant__ float c_levels_dec[16] = {MOE_NF4_LEVEL_LIST};
 
@@ -112,6 +134,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking probe of a phase (the producer polls several rings).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -193,8 +227,7 @@ struct Item {
   int expert, rtile, start, cnt;  // routed rows [start, start + cnt)
 };
 
-__device__ __forceinline__ Item item_info(const Misc& ms, const int32_t* offsets, int E,
-                                          int rtiles, int it) {
+__device__ __forceinline__ Item item_info(const Misc& ms, int E, int rtiles, int it) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -205,7 +238,7 @@ __device__ __forceinline__ Item item_info(const Misc& ms, const int32_t* offsets
   Item r;
   r.expert = lo;
   r.rtile = local - tc * rtiles;
-  const int s = offsets[lo], e = offsets[lo + 1];
+  const int s = ms.off[lo], e = ms.off[lo + 1];
   r.start = s + tc * TOK;
   r.cnt = min(TOK, e - r.start);
   return r;
@@ -219,17 +252,19 @@ __device__ __forceinline__ int weight_row(int r, int rtile, int N) {
   return rtile * ROWS + r;
 }
 
-// One item for one consumer warp, NT8 token tiles.  Warp w owns 16 weight
-// rows of the item (SwiGLU: gate rows 8 w .. 8 w + 7 and the matching up
-// rows) and all four 64-k blocks of every stage: four independent MMA chains
-// per token tile.  Returns false if a wait gave up.
+// One item for one consumer warp, NT8 token tiles.  Warp w (w-th of its
+// group) owns 16 weight rows of the item (SwiGLU: gate rows 8 w .. 8 w + 7 and
+// the matching up rows) and all four 64-k blocks of every stage: four
+// independent MMA chains per token tile.  The group's ring is slots
+// [rbase, rbase + rsize).  Returns false if a wait gave up.
 template <int FMT, int EPI, typename OutT, int NT8>
 __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, int K,
                                              const void* __restrict__ gscales,
                                              OutT* __restrict__ out, int32_t* dev_err,
-                                             int& stage, uint32_t& phase) {
+                                             int warp, int rbase, int rsize, int& stage,
+                                             uint32_t& phase) {
   using LY = Layout<FMT>;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int sg = ((g & 3) << 1) | (g >> 2);  // sigma(g)
   const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + sg : 16 * warp + sg;
@@ -274,9 +309,9 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
   for (int s = 0; s < KS; ++s) {
     uint2 nA = make_uint2(0, 0), nB = make_uint2(0, 0);
     if (FMT != kFmtNF4 && s + 1 < KS) fetch(s + 1, nA, nB);
-    const uint32_t base = stage < 2 ? LY::kStage0 + stage * LY::kStageBytes
-                                    : LY::kStage2 + (stage - 2) * LY::kStageBytes;
-    if (!mbar_wait(smem_u32(&ms.full[stage]), phase, ms, dev_err)) return false;
+    const int slot = rbase + stage;
+    const uint32_t base = LY::slot_addr(slot);
+    if (!mbar_wait(smem_u32(&ms.full[slot]), phase, ms, dev_err)) return false;
     const uint32_t wst = base, xst = base + kWBytes, ast = base + kWBytes + kXBytes;
     // per block b: the fp32 factor of its partial sums (NF4 absmax, INT4 s)
     // and the fp16-pair operand transform (INT4 {1024 + z}, MXFP4 2^(e-127))
@@ -366,8 +401,8 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
         }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&ms.empty[stage]));
-    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    if (lane == 0) mbar_arrive(smem_u32(&ms.empty[slot]));
+    if (++stage == rsize) { stage = 0; phase ^= 1; }
     cA = nA;
     cB = nB;
   }
@@ -416,7 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
   const int rtiles = N / ROWS;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NSLOTS; ++s) {
       mbar_init(smem_u32(&ms.full[s]), 1);
       mbar_init(smem_u32(&ms.empty[s]), CWARPS);
     }
@@ -442,7 +477,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
     }
     lut[b * 64 + l] = v;
   }
-  if (warp == CWARPS) {
+  if (warp == PWARP) {
     // item_prefix[e] = sum over e' < e of ceil(count / TOK) * rtiles
     bool bad = offsets[0] != 0 || offsets[E] != M_total;
     int run = 0;
@@ -450,7 +485,9 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
       const int e = b0 + lane;
       int c = 0;
       if (e < E) {
-        c = offsets[e + 1] - offsets[e];
+        const int o0 = offsets[e], o1 = offsets[e + 1];
+        ms.off[e] = o0;
+        c = o1 - o0;
         if (c < 0) { bad = true; c = 0; }
       }
       const int items = ((c + TOK - 1) / TOK) * rtiles;
@@ -465,6 +502,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
     }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) {
+      ms.off[E] = offsets[E];
       ms.item_prefix[E] = run;
       ms.nitems = bad ? 0 : run;
       if (bad) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
@@ -473,11 +511,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
   __syncthreads();
   const int total = ms.nitems;
   const int KS = K / SK;
-  auto stage_addr = [](int s) -> uint32_t {
-    return s < 2 ? LY::kStage0 + s * LY::kStageBytes : LY::kStage2 + (s - 2) * LY::kStageBytes;
-  };
 
-  if (warp == CWARPS) {
+  if (warp == PWARP) {
     // ---------------- producer
     if (lane == 0) {
       // the item's 128 weight rows as two 64-row halves (y, z .. z+1) of the
@@ -497,55 +532,98 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
         tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
         if (FMT == kFmtNF4) tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
       };
-      // Chain mode: the weights (and absmax) of the first ring's worth of
+      // Group g takes the CTA's items g, g + GROUPS, ...  One cursor per group
+      // (item, stage of the item, ring position); the loop serves whichever
+      // group's next slot is free.
+      const int step = GROUPS * gridDim.x;
+      int ci[GROUPS], cs[GROUPS], cgi[GROUPS], cst[GROUPS], cwy[GROUPS], cwz[GROUPS],
+          cnr[GROUPS], cstart[GROUPS], pre[GROUPS];
+      uint32_t cph[GROUPS];
+      auto load_item = [&](int g, int i) {
+        const Item it = item_info(ms, E, rtiles, i);
+        rows_of(it, cwy[g], cwz[g]);
+        cnr[g] = (it.cnt + 7) / 8;
+        cstart[g] = it.start;
+      };
+      int live = 0;
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) {
+        ci[g] = blockIdx.x + g * gridDim.x;
+        cs[g] = cgi[g] = cst[g] = pre[g] = 0;
+        cph[g] = 0;
+        if (ci[g] < total) { load_item(g, ci[g]); ++live; }
+      }
+      // Chain mode: the weights (and absmax) of each ring's first round of
       // stages are requested before the previous kernel (which writes A) has
       // finished; their barriers already expect the activation bytes too.
-      int pre = 0;
       if (chain) {
-        for (int i = blockIdx.x; i < total && pre < STAGES; i += gridDim.x) {
-          const Item it = item_info(ms, offsets, E, rtiles, i);
-          int wy, wz;
-          rows_of(it, wy, wz);
-          const int nr8 = (it.cnt + 7) / 8;
-          for (int s = 0; s < KS && pre < STAGES; ++s, ++pre)
-            issue_weights(stage_addr(pre), smem_u32(&ms.full[pre]), s, wy, wz, nr8);
+#pragma unroll
+        for (int g = 0; g < GROUPS; ++g) {
+          for (int i = ci[g]; i < total && pre[g] < ring_size(g); i += step) {
+            const Item it = item_info(ms, E, rtiles, i);
+            int wy, wz;
+            rows_of(it, wy, wz);
+            const int nr8 = (it.cnt + 7) / 8;
+            for (int s = 0; s < KS && pre[g] < ring_size(g); ++s, ++pre[g]) {
+              const int slot = ring_base(g) + pre[g];
+              issue_weights(LY::slot_addr(slot), smem_u32(&ms.full[slot]), s, wy, wz, nr8);
+            }
+          }
         }
         pdl_wait();
         pdl_trigger();
       }
-      int stage = 0, gi = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-        const Item it = item_info(ms, offsets, E, rtiles, i);
-        int wy, wz;
-        rows_of(it, wy, wz);
-        const int nr8 = (it.cnt + 7) / 8;
-        const CUtensorMap* xmap = nr8 > 1 ? &xmap16 : &xmap8;
-        for (int s = 0; s < KS; ++s, ++gi) {
-          const uint32_t full = smem_u32(&ms.full[stage]);
-          const uint32_t sb = stage_addr(stage);
-          if (gi >= pre) {  // stages gi < pre are slot gi, phase 0, weights already requested
-            if (!(ok = mbar_wait(smem_u32(&ms.empty[stage]), phase ^ 1, ms, dev_err))) break;
-            issue_weights(sb, full, s, wy, wz, nr8);
+      uint32_t idle = 0;
+      while (live > 0) {
+        bool moved = false;
+#pragma unroll
+        for (int g = 0; g < GROUPS; ++g) {
+          if (ci[g] >= total) continue;
+          const int slot = ring_base(g) + cst[g];
+          const uint32_t full = smem_u32(&ms.full[slot]);
+          const uint32_t sb = LY::slot_addr(slot);
+          // stages cgi < pre are the ring's first round, weights already requested
+          if (cgi[g] >= pre[g]) {
+            if (!mbar_test_wait(smem_u32(&ms.empty[slot]), cph[g] ^ 1)) continue;
+            issue_weights(sb, full, cs[g], cwy[g], cwz[g], cnr[g]);
           }
           // the stage's four 64-k blocks of the routed rows in one 3-D box
-          tma_load_3d(sb + kWBytes, xmap, full, 0, it.start, s * (SK / kBlock));
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          tma_load_3d(sb + kWBytes, cnr[g] > 1 ? &xmap16 : &xmap8, full, 0, cstart[g],
+                      cs[g] * (SK / kBlock));
+          moved = true;
+          ++cgi[g];
+          if (++cst[g] == ring_size(g)) { cst[g] = 0; cph[g] ^= 1; }
+          if (++cs[g] == KS) {
+            cs[g] = 0;
+            ci[g] += step;
+            if (ci[g] < total) load_item(g, ci[g]); else --live;
+          }
+        }
+        if (moved) {
+          idle = 0;
+        } else if (*reinterpret_cast<volatile int*>(&ms.abort_flag)) {
+          break;
+        } else if (++idle >= kSpinLimit) {
+          *reinterpret_cast<volatile int*>(&ms.abort_flag) = 1;
+          set_dev_err(dev_err, MOE_DEVERR_TIMEOUT);
+          break;
         }
       }
     }
   } else {
     // ---------------- consumers
+    const int g = warp / CWARPS;
     int stage = 0;
     uint32_t phase = 0;
-    for (int i = blockIdx.x; i < total; i += gridDim.x) {
-      const Item it = item_info(ms, offsets, E, rtiles, i);
+    for (int i = blockIdx.x + g * gridDim.x; i < total; i += GROUPS * gridDim.x) {
+      const Item it = item_info(ms, E, rtiles, i);
       bool ok;
       if (it.cnt > 8)
-        ok = consume_item<FMT, EPI, OutT, 2>(ms, it, N, K, gscales, out, dev_err, stage, phase);
+        ok = consume_item<FMT, EPI, OutT, 2>(ms, it, N, K, gscales, out, dev_err, warp % CWARPS,
+                                             ring_base(g), ring_size(g), stage, phase);
       else
-        ok = consume_item<FMT, EPI, OutT, 1>(ms, it, N, K, gscales, out, dev_err, stage, phase);
+        ok = consume_item<FMT, EPI, OutT, 1>(ms, it, N, K, gscales, out, dev_err, warp % CWARPS,
+                                             ring_base(g), ring_size(g), stage, phase);
       if (!ok) break;
     }
   }
@@ -651,7 +729,7 @@ namespace moe_launch {
 
 bool grouped_gemm_decode_supported(int N, int K) {
   // absmax rows must be a multiple of 16 bytes for the TMA map: K % 256.
-  return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
+  return N % moe::dec::kNAlign == 0 && K % moe::dec::SK == 0;
 }
 
 // Activations must be fp16 rows in permuted order (no gather).
@@ -664,7 +742,7 @@ cudaError_t grouped_gemm_decode(const void* A, int A_rows, const uint8_t* packed
 }
 
 bool grouped_gemm_int4_supported(int N, int K) {
-  return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
+  return N % moe::dec::kNAlign == 0 && K % moe::dec::SK == 0;
 }
 
 cudaError_t grouped_gemm_int4(const void* A, int A_rows, const uint8_t* packed,
@@ -676,7 +754,7 @@ cudaError_t grouped_gemm_int4(const void* A, int A_rows, const uint8_t* packed,
 }
 
 bool grouped_gemm_mxfp4_supported(int N, int K) {
-  return N % moe::dec::ROWS == 0 && K % moe::dec::SK == 0;
+  return N % moe::dec::kNAlign == 0 && K % moe::dec::SK == 0;
 }
 
 cudaError_t grouped_gemm_mxfp4(const void* A, int A_rows, const uint8_t* packed,
