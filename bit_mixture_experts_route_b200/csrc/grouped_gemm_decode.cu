@@ -99,6 +99,7 @@ struct Misc {
   int nitems;
   int item_prefix[1025];
   int off[1025];  // expert_offsets, copied once (item lookups never touch global memory)
+  int pre[GROUPS];  // stages of each ring's first round issued during the set-up
 };
 static_assert(Layout<kFmtNF4>::kMisc + sizeof(Misc) <= Layout<kFmtNF4>::kLut,
               "shared layout overlap");
@@ -436,10 +437,6 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
     int M_total, OutT* __restrict__ out, int32_t* dev_err, int chain) {
   using LY = Layout<FMT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  if (!chain) {  // nothing is read or written before the previous kernel is done
-    pdl_wait();
-    pdl_trigger();
-  }
   const uint32_t base = smem_u32(smem_raw);
   if (base > LY::kStage0) {  // layout assumption broken: do nothing, say so
     if (threadIdx.x == 0) set_dev_err(dev_err, MOE_DEVERR_LAYOUT);
@@ -449,35 +446,46 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem_raw + (LY::kLut - base));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rtiles = N / ROWS;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NSLOTS; ++s) {
-      mbar_init(smem_u32(&ms.full[s]), 1);
-      mbar_init(smem_u32(&ms.empty[s]), CWARPS);
-    }
-    ms.abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  // byte b -> its two weights as an fp16 pair, the lower k in the low half:
-  // NF4 {L[b >> 4], L[b & 15]}, MXFP4 {e2m1(b & 15), e2m1(b >> 4)}, INT4
-  // {1024 + (b >> 4), 1024 + (b & 15)} (0x6400 is fp16 1024, whose mantissa
-  // then holds the code).  One 256-byte row per byte value, lane l's copy at
-  // 4 l (the upper 128 bytes of each row are unused).
-  for (int i = threadIdx.x; i < 256 * 32; i += THREADS) {
-    const uint32_t b = (uint32_t)(i >> 5), l = (uint32_t)(i & 31);
-    uint32_t v;
-    if (FMT == kFmtNF4) {
-      const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
-                                       __float2half_rn(c_levels_dec[b & 15]));
-      v = *reinterpret_cast<const uint32_t*>(&h);
-    } else if (FMT == kFmtMXFP4) {
-      v = e2m1_h(b & 15u) | (e2m1_h(b >> 4) << 16);
+  const int KS = K / SK;
+  const int step = GROUPS * gridDim.x;  // group g takes the CTA's items g, g + GROUPS, ...
+  // the item's 128 weight rows as two 64-row halves (y, z .. z+1) of the 3-D
+  // weight (and absmax) maps: SwiGLU items take the gate rows and the
+  // matching up rows (z = 2e + half), plain items 128 consecutive rows
+  auto rows_of = [&](const Item& it, int& wy, int& wz) {
+    if (EPI == MOE_EPI_SWIGLU) {
+      wy = it.rtile * (ROWS / 2);
+      wz = 2 * it.expert;
     } else {
-      v = (0x6400u | (b >> 4)) | ((0x6400u | (b & 15u)) << 16);
+      wy = 0;
+      wz = it.expert * (N / (ROWS / 2)) + 2 * it.rtile;
     }
-    lut[b * 64 + l] = v;
-  }
+  };
+  auto issue_weights = [&](uint32_t sb, uint32_t full, int s, int wy, int wz, int nr8) {
+    mbar_arrive_expect_tx(full, kWBytes + LY::kA + nr8 * 4 * XBOX);
+    tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
+    if (FMT == kFmtNF4) tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
+  };
+  // the stage's four 64-k blocks of the routed rows in one 3-D box
+  auto issue_rows = [&](uint32_t sb, uint32_t full, int s, int start, int nr8) {
+    tma_load_3d(sb + kWBytes, nr8 > 1 ? &xmap16 : &xmap8, full, 0, start, s * (SK / kBlock));
+  };
+
   if (warp == PWARP) {
+    // Set-up: the barriers, then (after the previous kernel unless chained)
+    // the item list, then the first round of every ring, while the consumer
+    // warps build the decode table.
+    if (lane == 0) {
+      for (int s = 0; s < NSLOTS; ++s) {
+        mbar_init(smem_u32(&ms.full[s]), 1);
+        mbar_init(smem_u32(&ms.empty[s]), CWARPS);
+      }
+      ms.abort_flag = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (!chain) {  // nothing is read or written before the previous kernel is done
+      pdl_wait();
+      pdl_trigger();
+    }
     // item_prefix[e] = sum over e' < e of ceil(count / TOK) * rtiles
     bool bad = offsets[0] != 0 || offsets[E] != M_total;
     int run = 0;
@@ -507,35 +515,63 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
       ms.nitems = bad ? 0 : run;
       if (bad) set_dev_err(dev_err, MOE_DEVERR_BAD_OFFSETS);
     }
+    __syncwarp();
+    if (lane == 0) {
+      // The first round of each ring.  Chain mode: only the weights (and
+      // absmax), requested before the previous kernel (which writes A) has
+      // finished; their barriers already expect the activation bytes too.
+      const int total = ms.nitems;
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) {
+        int pre = 0;
+        for (int i = blockIdx.x + g * gridDim.x; i < total && pre < ring_size(g); i += step) {
+          const Item it = item_info(ms, E, rtiles, i);
+          int wy, wz;
+          rows_of(it, wy, wz);
+          const int nr8 = (it.cnt + 7) / 8;
+          for (int s = 0; s < KS && pre < ring_size(g); ++s, ++pre) {
+            const int slot = ring_base(g) + pre;
+            const uint32_t sb = LY::slot_addr(slot), full = smem_u32(&ms.full[slot]);
+            issue_weights(sb, full, s, wy, wz, nr8);
+            if (!chain) issue_rows(sb, full, s, it.start, nr8);
+          }
+        }
+        ms.pre[g] = pre;
+      }
+      if (chain) {
+        pdl_wait();
+        pdl_trigger();
+      }
+    }
+  } else {
+    // byte b -> its two weights as an fp16 pair, the lower k in the low half:
+    // NF4 {L[b >> 4], L[b & 15]}, MXFP4 {e2m1(b & 15), e2m1(b >> 4)}, INT4
+    // {1024 + (b >> 4), 1024 + (b & 15)} (0x6400 is fp16 1024, whose mantissa
+    // then holds the code).  One 256-byte row per byte value, lane l's copy at
+    // 4 l (the upper 128 bytes of each row are unused).
+    for (int i = threadIdx.x; i < 256 * 32; i += PWARP * 32) {
+      const uint32_t b = (uint32_t)(i >> 5), l = (uint32_t)(i & 31);
+      uint32_t v;
+      if (FMT == kFmtNF4) {
+        const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
+                                         __float2half_rn(c_levels_dec[b & 15]));
+        v = *reinterpret_cast<const uint32_t*>(&h);
+      } else if (FMT == kFmtMXFP4) {
+        v = e2m1_h(b & 15u) | (e2m1_h(b >> 4) << 16);
+      } else {
+        v = (0x6400u | (b >> 4)) | ((0x6400u | (b & 15u)) << 16);
+      }
+      lut[b * 64 + l] = v;
+    }
   }
   __syncthreads();
   const int total = ms.nitems;
-  const int KS = K / SK;
 
   if (warp == PWARP) {
     // ---------------- producer
     if (lane == 0) {
-      // the item's 128 weight rows as two 64-row halves (y, z .. z+1) of the
-      // 3-D weight (and absmax) maps: SwiGLU items take the gate rows and the
-      // matching up rows (z = 2e + half), plain items 128 consecutive rows
-      auto rows_of = [&](const Item& it, int& wy, int& wz) {
-        if (EPI == MOE_EPI_SWIGLU) {
-          wy = it.rtile * (ROWS / 2);
-          wz = 2 * it.expert;
-        } else {
-          wy = 0;
-          wz = it.expert * (N / (ROWS / 2)) + 2 * it.rtile;
-        }
-      };
-      auto issue_weights = [&](uint32_t sb, uint32_t full, int s, int wy, int wz, int nr8) {
-        mbar_arrive_expect_tx(full, kWBytes + LY::kA + nr8 * 4 * XBOX);
-        tma_load_3d(sb, &wmap, full, s * SB, wy, wz);
-        if (FMT == kFmtNF4) tma_load_3d(sb + kWBytes + kXBytes, &amap, full, s * 4, wy, wz);
-      };
-      // Group g takes the CTA's items g, g + GROUPS, ...  One cursor per group
-      // (item, stage of the item, ring position); the loop serves whichever
-      // group's next slot is free.
-      const int step = GROUPS * gridDim.x;
+      // One cursor per group (item, stage of the item, ring position); the
+      // loop serves whichever group's next slot is free.
       int ci[GROUPS], cs[GROUPS], cgi[GROUPS], cst[GROUPS], cwy[GROUPS], cwz[GROUPS],
           cnr[GROUPS], cstart[GROUPS], pre[GROUPS];
       uint32_t cph[GROUPS];
@@ -549,29 +585,10 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
 #pragma unroll
       for (int g = 0; g < GROUPS; ++g) {
         ci[g] = blockIdx.x + g * gridDim.x;
-        cs[g] = cgi[g] = cst[g] = pre[g] = 0;
+        cs[g] = cgi[g] = cst[g] = 0;
         cph[g] = 0;
+        pre[g] = ms.pre[g];
         if (ci[g] < total) { load_item(g, ci[g]); ++live; }
-      }
-      // Chain mode: the weights (and absmax) of each ring's first round of
-      // stages are requested before the previous kernel (which writes A) has
-      // finished; their barriers already expect the activation bytes too.
-      if (chain) {
-#pragma unroll
-        for (int g = 0; g < GROUPS; ++g) {
-          for (int i = ci[g]; i < total && pre[g] < ring_size(g); i += step) {
-            const Item it = item_info(ms, E, rtiles, i);
-            int wy, wz;
-            rows_of(it, wy, wz);
-            const int nr8 = (it.cnt + 7) / 8;
-            for (int s = 0; s < KS && pre[g] < ring_size(g); ++s, ++pre[g]) {
-              const int slot = ring_base(g) + pre[g];
-              issue_weights(LY::slot_addr(slot), smem_u32(&ms.full[slot]), s, wy, wz, nr8);
-            }
-          }
-        }
-        pdl_wait();
-        pdl_trigger();
       }
       uint32_t idle = 0;
       while (live > 0) {
@@ -582,14 +599,14 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
           const int slot = ring_base(g) + cst[g];
           const uint32_t full = smem_u32(&ms.full[slot]);
           const uint32_t sb = LY::slot_addr(slot);
-          // stages cgi < pre are the ring's first round, weights already requested
-          if (cgi[g] >= pre[g]) {
+          // stages cgi < pre are the ring's first round, issued during the
+          // set-up (in chain mode without their activation rows)
+          const bool fresh = cgi[g] >= pre[g];
+          if (fresh) {
             if (!mbar_test_wait(smem_u32(&ms.empty[slot]), cph[g] ^ 1)) continue;
             issue_weights(sb, full, cs[g], cwy[g], cwz[g], cnr[g]);
           }
-          // the stage's four 64-k blocks of the routed rows in one 3-D box
-          tma_load_3d(sb + kWBytes, cnr[g] > 1 ? &xmap16 : &xmap8, full, 0, cstart[g],
-                      cs[g] * (SK / kBlock));
+          if (fresh || chain) issue_rows(sb, full, cs[g], cstart[g], cnr[g]);
           moved = true;
           ++cgi[g];
           if (++cst[g] == ring_size(g)) { cst[g] = 0; cph[g] ^= 1; }
