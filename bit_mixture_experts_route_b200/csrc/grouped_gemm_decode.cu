@@ -20,18 +20,22 @@
 // * Persistent CTAs (one per SM) walk a list of work items built on the
 //   device from expert_offsets: (expert, 128 weight rows, up to 16 routed
 //   rows; an expert with more routed rows yields one item per 16).
-// * Two consumer groups of eight warps take alternate items of the CTA's list,
+// * Two consumer groups of four warps take alternate items of the CTA's list,
 //   each through its own ring of stage slots (three and two of five).  One
 //   producer thread serves both rings, polling whichever group's next slot is
 //   free, with TMA tile loads, 256 k per stage: the packed rows (one 3-D box of
 //   2 x 64 rows x 128 bytes), for NF4 their absmax (one 3-D box of 2 x 64 rows
 //   x 4 fp32) and the routed activation rows (one 3-D box of the stage's four
 //   64-k blocks x 8 or 16 rows), with 128-byte swizzle: three copies per
-//   stage.  (17 warps leave 96 registers per thread.)
-// * The eight warps of a group each own 16 weight rows of the item and run
-//   mma.sync.m16n8k16 with the weights as the M side and the routed rows as N
-//   (swap-AB); the four 64-k blocks of a stage run as four interleaved MMA
-//   chains.  A lane turns each packed byte into an fp16 pair through ONE
+//   stage.
+// * The four warps of a group each own 32 weight rows of the item (two m-tiles
+//   of 16) and run mma.sync.m16n8k16 with the weights as the M side and the
+//   routed rows as N (swap-AB); the four 64-k blocks of a stage run as four
+//   interleaved MMA chains.  Shared-memory bandwidth bounds the consumers
+//   (per weight: the 2-byte table entry, a quarter byte of packed code, the
+//   activation fragments, and the TMA writes); a warp reads the stage's
+//   activation fragments once for both of its m-tiles, which halves their
+//   share against 16 rows per warp.  A lane turns each packed byte into an fp16 pair through ONE
 //   byte_perm (which assembles the shared address of the byte's entry in a
 //   per-lane table: 0x10000 | byte << 8 | lane << 2) and one shared load; the
 //   table sits at shared address 64 KB, one 256-byte row per byte value, so
@@ -60,7 +64,8 @@ constexpr int TOK = 16;         // routed rows per item (max)
 constexpr int SK = 256;         // k per stage
 constexpr int kNAlign = 128;    // N granularity of the entry points (as the tensor-core form)
 constexpr int SB = SK / 2;      // packed bytes per row per stage
-constexpr int CWARPS = ROWS / 16;  // consumer warps per group, 16 weight rows each
+constexpr int MT = 2;           // m-tiles (16 weight rows each) per consumer warp
+constexpr int CWARPS = ROWS / (16 * MT);  // consumer warps per group
 constexpr int GROUPS = 2;       // consumer groups, each on its own items and ring
 constexpr int NSLOTS = 5;       // stage slots, both groups
 constexpr int kLoSlots = 2;     // slots below the table
@@ -254,10 +259,12 @@ __device__ __forceinline__ int weight_row(int r, int rtile, int N) {
 }
 
 // One item for one consumer warp, NT8 token tiles.  Warp w (w-th of its
-// group) owns 16 weight rows of the item (SwiGLU: gate rows 8 w .. 8 w + 7 and
-// the matching up rows) and all four 64-k blocks of every stage: four
-// independent MMA chains per token tile.  The group's ring is slots
-// [rbase, rbase + rsize).  Returns false if a wait gave up.
+// group) owns MT m-tiles of 16 weight rows; m-tile m holds the rows of
+// "virtual warp" v = MT w + m (SwiGLU: gate rows 8 v .. 8 v + 7 and the
+// matching up rows; plain: rows 16 v .. 16 v + 15).  It takes all four 64-k
+// blocks of every stage (four independent MMA chains per token tile) and reads
+// the stage's activation fragments once for its MT m-tiles.  The group's ring
+// is slots [rbase, rbase + rsize).  Returns false if a wait gave up.
 template <int FMT, int EPI, typename OutT, int NT8>
 __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, int K,
                                              const void* __restrict__ gscales,
@@ -268,8 +275,13 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int sg = ((g & 3) << 1) | (g >> 2);  // sigma(g)
-  const int rA = (EPI == MOE_EPI_SWIGLU) ? 8 * warp + sg : 16 * warp + sg;
-  const int rB = (EPI == MOE_EPI_SWIGLU) ? ROWS / 2 + 8 * warp + sg : 16 * warp + sg + 8;
+  int rA[MT], rB[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int v = MT * warp + m;
+    rA[m] = (EPI == MOE_EPI_SWIGLU) ? 8 * v + sg : 16 * v + sg;
+    rB[m] = (EPI == MOE_EPI_SWIGLU) ? ROWS / 2 + 8 * v + sg : 16 * v + sg + 8;
+  }
   // byte_perm source: 0x10000 | lane << 2 -> entry address of a byte
   const uint32_t lb = 0x10000u | ((uint32_t)lane << 2);
   // this lane's 8 packed bytes of block b in a 128-byte swizzled row whose
@@ -283,69 +295,52 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
   // INT4 / MXFP4 scales of rows rA and rB from global memory, one stage
   // ahead: INT4 the meta words of the stage's two 128-k groups, MXFP4 the
   // stage's eight scale bytes
-  const size_t gA = (size_t)it.expert * N + weight_row<EPI>(rA, it.rtile, N);
-  const size_t gB = (size_t)it.expert * N + weight_row<EPI>(rB, it.rtile, N);
-  auto fetch = [&](int s, uint2& mA, uint2& mB) {
-    if (FMT == kFmtINT4) {
-      const uint2* p = reinterpret_cast<const uint2*>(static_cast<const uint32_t*>(gscales));
-      mA = __ldg(p + gA * (K / I4_GROUP / 2) + s);
-      mB = __ldg(p + gB * (K / I4_GROUP / 2) + s);
-    } else if (FMT == kFmtMXFP4) {
-      const uint2* p = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(gscales));
-      mA = __ldg(p + gA * (K / MX_BLK / 8) + s);
-      mB = __ldg(p + gB * (K / MX_BLK / 8) + s);
+  size_t gA[MT], gB[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    gA[m] = (size_t)it.expert * N + weight_row<EPI>(rA[m], it.rtile, N);
+    gB[m] = (size_t)it.expert * N + weight_row<EPI>(rB[m], it.rtile, N);
+  }
+  auto fetch = [&](int s, uint2 (&mA)[MT], uint2 (&mB)[MT]) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (FMT == kFmtINT4) {
+        const uint2* p = reinterpret_cast<const uint2*>(static_cast<const uint32_t*>(gscales));
+        mA[m] = __ldg(p + gA[m] * (K / I4_GROUP / 2) + s);
+        mB[m] = __ldg(p + gB[m] * (K / I4_GROUP / 2) + s);
+      } else if (FMT == kFmtMXFP4) {
+        const uint2* p = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(gscales));
+        mA[m] = __ldg(p + gA[m] * (K / MX_BLK / 8) + s);
+        mB[m] = __ldg(p + gB[m] * (K / MX_BLK / 8) + s);
+      }
     }
   };
 
-  float acc[NT8][4];
+  float acc[MT][NT8][4];
 #pragma unroll
-  for (int j = 0; j < NT8; ++j)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[j][q] = 0.0f;
+    for (int j = 0; j < NT8; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[m][j][q] = 0.0f;
 
   bool bad_scale = false;
   const int KS = K / SK;
-  uint2 cA = make_uint2(0, 0), cB = make_uint2(0, 0);
+  uint2 cA[MT], cB[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) cA[m] = cB[m] = make_uint2(0, 0);
   if (FMT != kFmtNF4) fetch(0, cA, cB);
   for (int s = 0; s < KS; ++s) {
-    uint2 nA = make_uint2(0, 0), nB = make_uint2(0, 0);
+    uint2 nA[MT], nB[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) nA[m] = nB[m] = make_uint2(0, 0);
     if (FMT != kFmtNF4 && s + 1 < KS) fetch(s + 1, nA, nB);
     const int slot = rbase + stage;
     const uint32_t base = LY::slot_addr(slot);
     if (!mbar_wait(smem_u32(&ms.full[slot]), phase, ms, dev_err)) return false;
     const uint32_t wst = base, xst = base + kWBytes, ast = base + kWBytes + kXBytes;
-    // per block b: the fp32 factor of its partial sums (NF4 absmax, INT4 s)
-    // and the fp16-pair operand transform (INT4 {1024 + z}, MXFP4 2^(e-127))
-    float fA[4] = {1.f, 1.f, 1.f, 1.f}, fB[4] = {1.f, 1.f, 1.f, 1.f};
-    uint32_t zA[4] = {0, 0, 0, 0}, zB[4] = {0, 0, 0, 0};
-    if (FMT == kFmtNF4) {
-      const uint4 sa = lds128(ast + rA * 16), sb = lds128(ast + rB * 16);
-      fA[0] = __uint_as_float(sa.x); fA[1] = __uint_as_float(sa.y);
-      fA[2] = __uint_as_float(sa.z); fA[3] = __uint_as_float(sa.w);
-      fB[0] = __uint_as_float(sb.x); fB[1] = __uint_as_float(sb.y);
-      fB[2] = __uint_as_float(sb.z); fB[3] = __uint_as_float(sb.w);
-    } else if (FMT == kFmtINT4) {
-      const uint32_t mA[2] = {cA.x, cA.y}, mB[2] = {cB.x, cB.y};
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t a = mA[b >> 1], c = mB[b >> 1];  // group of this 64-k block
-        fA[b] = __half2float(__ushort_as_half((unsigned short)(a & 0xFFFFu)));
-        fB[b] = __half2float(__ushort_as_half((unsigned short)(c & 0xFFFFu)));
-        zA[b] = 0x64006400u | ((a >> 16) & 0xFu) * 0x00010001u;
-        zB[b] = 0x64006400u | ((c >> 16) & 0xFu) * 0x00010001u;
-      }
-    } else {
-      const uint32_t mA[2] = {cA.x, cA.y}, mB[2] = {cB.x, cB.y};
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        // a lane's 16 k of block b lie in scale block 2b + t/2 of the stage
-        const int sbi = 2 * b + (t >> 1);
-        zA[b] = mx_scale_h2((mA[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu, bad_scale);
-        zB[b] = mx_scale_h2((mB[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu, bad_scale);
-      }
-    }
+    // the stage's activation fragments, shared by the warp's m-tiles
     uint32_t xf[4][NT8][8];
-    uint2 wa[4], wb[4];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
 #pragma unroll
@@ -355,77 +350,119 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
         xf[b][j][0] = u.x; xf[b][j][1] = u.y; xf[b][j][2] = u.z; xf[b][j][3] = u.w;
         xf[b][j][4] = v.x; xf[b][j][5] = v.y; xf[b][j][6] = v.z; xf[b][j][7] = v.w;
       }
-      wa[b] = lds64(wst + rA * SB + woff[b]);
-      wb[b] = lds64(wst + rB * SB + woff[b]);
     }
-    float tmp[4][NT8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
-      const uint32_t s0 = 0x7604u | (lo << 4), s1 = 0x7604u | ((lo + 1) << 4);
+    for (int m = 0; m < MT; ++m) {
+      // per block b: the fp32 factor of its partial sums (NF4 absmax, INT4 s)
+      // and the fp16-pair operand transform (INT4 {1024 + z}, MXFP4 2^(e-127))
+      float fA[4] = {1.f, 1.f, 1.f, 1.f}, fB[4] = {1.f, 1.f, 1.f, 1.f};
+      uint32_t zA[4] = {0, 0, 0, 0}, zB[4] = {0, 0, 0, 0};
+      if (FMT == kFmtNF4) {
+        const uint4 sa = lds128(ast + rA[m] * 16), sb = lds128(ast + rB[m] * 16);
+        fA[0] = __uint_as_float(sa.x); fA[1] = __uint_as_float(sa.y);
+        fA[2] = __uint_as_float(sa.z); fA[3] = __uint_as_float(sa.w);
+        fB[0] = __uint_as_float(sb.x); fB[1] = __uint_as_float(sb.y);
+        fB[2] = __uint_as_float(sb.z); fB[3] = __uint_as_float(sb.w);
+      } else if (FMT == kFmtINT4) {
+        const uint32_t mA[2] = {cA[m].x, cA[m].y}, mB[2] = {cB[m].x, cB[m].y};
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t vA = (i < 2) ? wa[b].x : wa[b].y;
-        const uint32_t vB = (i < 2) ? wb[b].x : wb[b].y;
-        uint32_t af[4];
-        af[0] = lds32(__byte_perm(vA, lb, s0));
-        af[1] = lds32(__byte_perm(vB, lb, s0));
-        af[2] = lds32(__byte_perm(vA, lb, s1));
-        af[3] = lds32(__byte_perm(vB, lb, s1));
-        if (FMT == kFmtINT4) {
-          af[0] = hsub2_u(af[0], zA[b]); af[2] = hsub2_u(af[2], zA[b]);
-          af[1] = hsub2_u(af[1], zB[b]); af[3] = hsub2_u(af[3], zB[b]);
-        } else if (FMT == kFmtMXFP4) {
-          af[0] = hmul2_u(af[0], zA[b]); af[2] = hmul2_u(af[2], zA[b]);
-          af[1] = hmul2_u(af[1], zB[b]); af[3] = hmul2_u(af[3], zB[b]);
+        for (int b = 0; b < 4; ++b) {
+          const uint32_t a = mA[b >> 1], c = mB[b >> 1];  // group of this 64-k block
+          fA[b] = __half2float(__ushort_as_half((unsigned short)(a & 0xFFFFu)));
+          fB[b] = __half2float(__ushort_as_half((unsigned short)(c & 0xFFFFu)));
+          zA[b] = 0x64006400u | ((a >> 16) & 0xFu) * 0x00010001u;
+          zB[b] = 0x64006400u | ((c >> 16) & 0xFu) * 0x00010001u;
         }
+      } else {
+        const uint32_t mA[2] = {cA[m].x, cA[m].y}, mB[2] = {cB[m].x, cB[m].y};
 #pragma unroll
-        for (int j = 0; j < NT8; ++j) {
-          if (FMT == kFmtMXFP4)
-            mma_16816(acc[j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
-          else if (i == 0)
-            mma_16816_z(tmp[b][j], af, xf[b][j][0], xf[b][j][1]);
-          else
-            mma_16816(tmp[b][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
+        for (int b = 0; b < 4; ++b) {
+          // a lane's 16 k of block b lie in scale block 2b + t/2 of the stage
+          const int sbi = 2 * b + (t >> 1);
+          zA[b] = mx_scale_h2((mA[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu, bad_scale);
+          zB[b] = mx_scale_h2((mB[sbi >> 2] >> (8 * (sbi & 3))) & 0xFFu, bad_scale);
         }
       }
-    }
-    if (FMT != kFmtMXFP4) {
+      uint2 wa[4], wb[4];
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
+      for (int b = 0; b < 4; ++b) {
+        wa[b] = lds64(wst + rA[m] * SB + woff[b]);
+        wb[b] = lds64(wst + rB[m] * SB + woff[b]);
+      }
+      float tmp[4][NT8][4];
 #pragma unroll
-        for (int j = 0; j < NT8; ++j) {
-          acc[j][0] = fmaf(fA[b], tmp[b][j][0], acc[j][0]);
-          acc[j][1] = fmaf(fA[b], tmp[b][j][1], acc[j][1]);
-          acc[j][2] = fmaf(fB[b], tmp[b][j][2], acc[j][2]);
-          acc[j][3] = fmaf(fB[b], tmp[b][j][3], acc[j][3]);
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
+        const uint32_t s0 = 0x7604u | (lo << 4), s1 = 0x7604u | ((lo + 1) << 4);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const uint32_t vA = (i < 2) ? wa[b].x : wa[b].y;
+          const uint32_t vB = (i < 2) ? wb[b].x : wb[b].y;
+          uint32_t af[4];
+          af[0] = lds32(__byte_perm(vA, lb, s0));
+          af[1] = lds32(__byte_perm(vB, lb, s0));
+          af[2] = lds32(__byte_perm(vA, lb, s1));
+          af[3] = lds32(__byte_perm(vB, lb, s1));
+          if (FMT == kFmtINT4) {
+            af[0] = hsub2_u(af[0], zA[b]); af[2] = hsub2_u(af[2], zA[b]);
+            af[1] = hsub2_u(af[1], zB[b]); af[3] = hsub2_u(af[3], zB[b]);
+          } else if (FMT == kFmtMXFP4) {
+            af[0] = hmul2_u(af[0], zA[b]); af[2] = hmul2_u(af[2], zA[b]);
+            af[1] = hmul2_u(af[1], zB[b]); af[3] = hmul2_u(af[3], zB[b]);
+          }
+#pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            if (FMT == kFmtMXFP4)
+              mma_16816(acc[m][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
+            else if (i == 0)
+              mma_16816_z(tmp[b][j], af, xf[b][j][0], xf[b][j][1]);
+            else
+              mma_16816(tmp[b][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
+          }
         }
+      }
+      if (FMT != kFmtMXFP4) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int j = 0; j < NT8; ++j) {
+            acc[m][j][0] = fmaf(fA[b], tmp[b][j][0], acc[m][j][0]);
+            acc[m][j][1] = fmaf(fA[b], tmp[b][j][1], acc[m][j][1]);
+            acc[m][j][2] = fmaf(fB[b], tmp[b][j][2], acc[m][j][2]);
+            acc[m][j][3] = fmaf(fB[b], tmp[b][j][3], acc[m][j][3]);
+          }
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&ms.empty[slot]));
     if (++stage == rsize) { stage = 0; phase ^= 1; }
-    cA = nA;
-    cB = nB;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      cA[m] = nA[m];
+      cB[m] = nB[m];
+    }
   }
   if (bad_scale) set_dev_err(dev_err, MOE_DEVERR_RANGE);
 
-  // acc[j][q]: row rA (q < 2) or rB (q >= 2), routed row 8j + 2t + (q & 1)
+  // acc[m][j][q]: row rA[m] (q < 2) or rB[m] (q >= 2), routed row 8j + 2t + (q & 1)
 #pragma unroll
-  for (int j = 0; j < NT8; ++j) {
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int tok = 8 * j + 2 * t + q;
-      if (tok >= it.cnt) continue;
-      const size_t p = (size_t)(it.start + tok);
-      if (EPI == MOE_EPI_SWIGLU) {
-        store_checked(out, p * (N / 2) + it.rtile * (ROWS / 2) + rA,
-                      swiglu_f32(acc[j][q], acc[j][q + 2]), dev_err);
-      } else {
-        store_checked(out, p * N + it.rtile * ROWS + rA, acc[j][q], dev_err);
-        store_checked(out, p * N + it.rtile * ROWS + rB, acc[j][q + 2], dev_err);
+    for (int j = 0; j < NT8; ++j) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int tok = 8 * j + 2 * t + q;
+        if (tok >= it.cnt) continue;
+        const size_t p = (size_t)(it.start + tok);
+        if (EPI == MOE_EPI_SWIGLU) {
+          store_checked(out, p * (N / 2) + it.rtile * (ROWS / 2) + rA[m],
+                        swiglu_f32(acc[m][j][q], acc[m][j][q + 2]), dev_err);
+        } else {
+          store_checked(out, p * N + it.rtile * ROWS + rA[m], acc[m][j][q], dev_err);
+          store_checked(out, p * N + it.rtile * ROWS + rB[m], acc[m][j][q + 2], dev_err);
+        }
       }
     }
-  }
   return true;
 }
 
