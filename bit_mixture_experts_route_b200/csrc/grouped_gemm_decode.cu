@@ -31,15 +31,17 @@
 // * The four warps of a group each own 32 weight rows of the item (two m-tiles
 //   of 16) and run mma.sync.m16n8k16 with the weights as the M side and the
 //   routed rows as N (swap-AB); the four 64-k blocks of a stage run as four
-//   interleaved MMA chains.  Shared-memory bandwidth bounds the consumers
-//   (per weight: the 2-byte table entry, a quarter byte of packed code, the
-//   activation fragments, and the TMA writes); a warp reads the stage's
-//   activation fragments once for both of its m-tiles, which halves their
-//   share against 16 rows per warp.  A lane turns each packed byte into an fp16 pair through ONE
+//   interleaved MMA chains.
+// * NF4 and INT4: a lane turns each packed byte into an fp16 pair through ONE
 //   byte_perm (which assembles the shared address of the byte's entry in a
 //   per-lane table: 0x10000 | byte << 8 | lane << 2) and one shared load; the
 //   table sits at shared address 64 KB, one 256-byte row per byte value, so
-//   the lookups never conflict.
+//   the lookups never conflict.  MXFP4: the hardware E2M1 -> fp16 conversion,
+//   one instruction per byte and no table.
+// * Shared-memory bandwidth bounds the consumers: per weight the table entry
+//   (2 bytes), the packed code, the activation fragments and the TMA writes.
+//   A warp reads a stage's activation fragments once for both of its m-tiles,
+//   which halves their share against 16 rows per warp.
 // * Scales: NF4 scales each 64-k block's fp32 partial sum by the row's fp32
 //   absmax (the only weight rounding is the levels' fp16 one); INT4 subtracts
 //   the zero in fp16 (exact) and scales the block's fp32 partial sum by s;
@@ -208,6 +210,19 @@ __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
   __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// The four bytes of w, each two E2M1 codes, as four fp16 pairs (the low
+// nibble in the low half), by the hardware conversion.
+__device__ __forceinline__ void e2m1x8_to_h2(uint32_t w, uint32_t (&d)[4]) {
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, c2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, c3;\n\t}"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(w));
 }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -389,39 +404,57 @@ __device__ __forceinline__ bool consume_item(Misc& ms, const Item& it, int N, in
         wa[b] = lds64(wst + rA[m] * SB + woff[b]);
         wb[b] = lds64(wst + rB[m] * SB + woff[b]);
       }
-      float tmp[4][NT8][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
-        const uint32_t s0 = 0x7604u | (lo << 4), s1 = 0x7604u | ((lo + 1) << 4);
+      if (FMT == kFmtMXFP4) {
+        // MXFP4: codes to fp16 pairs by the hardware conversion (no table),
+        // times the block's power of two, straight into the accumulators
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          const uint32_t vA = (i < 2) ? wa[b].x : wa[b].y;
-          const uint32_t vB = (i < 2) ? wb[b].x : wb[b].y;
-          uint32_t af[4];
-          af[0] = lds32(__byte_perm(vA, lb, s0));
-          af[1] = lds32(__byte_perm(vB, lb, s0));
-          af[2] = lds32(__byte_perm(vA, lb, s1));
-          af[3] = lds32(__byte_perm(vB, lb, s1));
-          if (FMT == kFmtINT4) {
-            af[0] = hsub2_u(af[0], zA[b]); af[2] = hsub2_u(af[2], zA[b]);
-            af[1] = hsub2_u(af[1], zB[b]); af[3] = hsub2_u(af[3], zB[b]);
-          } else if (FMT == kFmtMXFP4) {
-            af[0] = hmul2_u(af[0], zA[b]); af[2] = hmul2_u(af[2], zA[b]);
-            af[1] = hmul2_u(af[1], zB[b]); af[3] = hmul2_u(af[3], zB[b]);
-          }
+          uint32_t pa[8], pb[8];  // fp16 pairs of bytes 0..7 of rows rA, rB in block b
+          e2m1x8_to_h2(wa[b].x, *reinterpret_cast<uint32_t(*)[4]>(&pa[0]));
+          e2m1x8_to_h2(wa[b].y, *reinterpret_cast<uint32_t(*)[4]>(&pa[4]));
+          e2m1x8_to_h2(wb[b].x, *reinterpret_cast<uint32_t(*)[4]>(&pb[0]));
+          e2m1x8_to_h2(wb[b].y, *reinterpret_cast<uint32_t(*)[4]>(&pb[4]));
 #pragma unroll
-          for (int j = 0; j < NT8; ++j) {
-            if (FMT == kFmtMXFP4)
+          for (int i = 0; i < 4; ++i) {
+            const int lo = (i >> 1) * 4 + (i & 1) * 2;  // byte feeding slots 2t, 2t+1
+            uint32_t af[4];
+            af[0] = hmul2_u(pa[lo], zA[b]);
+            af[1] = hmul2_u(pb[lo], zB[b]);
+            af[2] = hmul2_u(pa[lo + 1], zA[b]);
+            af[3] = hmul2_u(pb[lo + 1], zB[b]);
+#pragma unroll
+            for (int j = 0; j < NT8; ++j)
               mma_16816(acc[m][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
-            else if (i == 0)
-              mma_16816_z(tmp[b][j], af, xf[b][j][0], xf[b][j][1]);
-            else
-              mma_16816(tmp[b][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
           }
         }
-      }
-      if (FMT != kFmtMXFP4) {
+      } else {
+        float tmp[4][NT8][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t lo = (i & 1) * 2;  // byte of the word feeding slots 2t, 2t+1
+          const uint32_t s0 = 0x7604u | (lo << 4), s1 = 0x7604u | ((lo + 1) << 4);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t vA = (i < 2) ? wa[b].x : wa[b].y;
+            const uint32_t vB = (i < 2) ? wb[b].x : wb[b].y;
+            uint32_t af[4];
+            af[0] = lds32(__byte_perm(vA, lb, s0));
+            af[1] = lds32(__byte_perm(vB, lb, s0));
+            af[2] = lds32(__byte_perm(vA, lb, s1));
+            af[3] = lds32(__byte_perm(vB, lb, s1));
+            if (FMT == kFmtINT4) {
+              af[0] = hsub2_u(af[0], zA[b]); af[2] = hsub2_u(af[2], zA[b]);
+              af[1] = hsub2_u(af[1], zB[b]); af[3] = hsub2_u(af[3], zB[b]);
+            }
+#pragma unroll
+            for (int j = 0; j < NT8; ++j) {
+              if (i == 0)
+                mma_16816_z(tmp[b][j], af, xf[b][j][0], xf[b][j][1]);
+              else
+                mma_16816(tmp[b][j], af, xf[b][j][2 * i], xf[b][j][2 * i + 1]);
+            }
+          }
+        }
 #pragma unroll
         for (int b = 0; b < 4; ++b)
 #pragma unroll
@@ -582,19 +615,17 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(
     }
   } else {
     // byte b -> its two weights as an fp16 pair, the lower k in the low half:
-    // NF4 {L[b >> 4], L[b & 15]}, MXFP4 {e2m1(b & 15), e2m1(b >> 4)}, INT4
-    // {1024 + (b >> 4), 1024 + (b & 15)} (0x6400 is fp16 1024, whose mantissa
-    // then holds the code).  One 256-byte row per byte value, lane l's copy at
-    // 4 l (the upper 128 bytes of each row are unused).
-    for (int i = threadIdx.x; i < 256 * 32; i += PWARP * 32) {
+    // NF4 {L[b >> 4], L[b & 15]}, INT4 {1024 + (b >> 4), 1024 + (b & 15)}
+    // (0x6400 is fp16 1024, whose mantissa then holds the code).  One 256-byte
+    // row per byte value, lane l's copy at 4 l (the upper 128 bytes of each
+    // row are unused).  MXFP4 needs no table.
+    for (int i = threadIdx.x; FMT != kFmtMXFP4 && i < 256 * 32; i += PWARP * 32) {
       const uint32_t b = (uint32_t)(i >> 5), l = (uint32_t)(i & 31);
       uint32_t v;
       if (FMT == kFmtNF4) {
         const __half2 h = __halves2half2(__float2half_rn(c_levels_dec[b >> 4]),
                                          __float2half_rn(c_levels_dec[b & 15]));
         v = *reinterpret_cast<const uint32_t*>(&h);
-      } else if (FMT == kFmtMXFP4) {
-        v = e2m1_h(b & 15u) | (e2m1_h(b >> 4) << 16);
       } else {
         v = (0x6400u | (b >> 4)) | ((0x6400u | (b & 15u)) << 16);
       }
