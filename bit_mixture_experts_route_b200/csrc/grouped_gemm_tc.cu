@@ -22,8 +22,8 @@
 // flow through three rings: activations (3 x 32 KB shared), packed NF4 rows
 // (8 x 4 KB shared) and decoded weights (8 TMEM slots).  Waiting threads
 // sleep in the barrier unit rather than spin.  Warp roles (864 threads):
-//   warp 0      TMA producer: activation tiles [256 rows x 64 k] (128-byte
-//               swizzle)
+//   warp 0      TMA producer: activation tiles [the MMA's N rows x 64 k]
+//               (128-byte swizzle), one box of exactly that height
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 x K16 per stage
 //   warp 2      TMA producer: the tile's packed NF4 rows [128 rows x 32 B]
 //   warps 3-18  decoders: four groups of four warps (one per TMEM lane
@@ -65,9 +65,8 @@ namespace tc {
 constexpr int BM = 128;          // weight rows per tile (MMA M)
 constexpr int BN = 256;          // routed rows per tile (max MMA N)
 constexpr int BK = 64;           // k per stage = one NF4 block
-constexpr int B_BOX_ROWS = 128;        // TMA box: 64 k x 128 rows
-constexpr int B_BOX_BYTES = B_BOX_ROWS * BK * 2;  // 16 KB
-constexpr int B_STAGE = BN * BK * 2;   // 32 KB: a tile's routed rows, two boxes
+constexpr int B_STAGE = BN * BK * 2;   // 32 KB: a tile's routed rows (at most 256)
+constexpr int B_MAPS = BN / 16;        // activation box heights 16, 32, ..., 256 rows
 
 constexpr int RAW_RING = 8;            // packed-row ring (shared memory)
 constexpr int RING = 8;                // decoded-weight ring (tensor memory)
@@ -91,6 +90,12 @@ constexpr uint32_t kSuspendNs = 1000;       // longest sleep of one try
 static_assert(A_COL + RING * A_SLOT_COLS <= TMEM_COLS, "tensor memory budget");
 static_assert(RING % GROUPS == 0 && RAW_RING % GROUPS == 0,
               "a group always meets its own slots");
+
+// One tensor map of the activation (or gradient) rows per box height, 16 to
+// 256 rows in steps of 16: a stage loads exactly the rows its MMAs read.
+struct __align__(64) BMaps {
+  CUtensorMap m[B_MAPS];
+};
 
 // Shared memory of one kernel form.  The activation producer can only run
 // NBS stages ahead of the MMAs (it refills a stage's slot once that stage's
@@ -463,7 +468,7 @@ __device__ __forceinline__ void stage_scales(uint32_t sc, uint32_t& h0, uint32_t
 // gradient of h) and writes the gradient of gate_up's pre-activations.
 template <int FMT, int EPI, typename OutT, int PAIR, bool TR>
 __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
-    const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap bmap2,
+    const __grid_constant__ BMaps bmaps,
     const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap amap,
     const void* __restrict__ scales, const int32_t* __restrict__ offsets, int E, int N, int K,
     int M_total, OutT* __restrict__ out, const float* __restrict__ gu, int32_t* dev_err,
@@ -585,17 +590,18 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
       }
       // Activation slot S mod BSTAGES is free once the MMAs of stage
       // S - BSTAGES are done: the a_empty barrier of that stage's TMEM slot
-      // (one commit per stage serves both rings).  A stage is the tile's
-      // routed rows in whole 128-row boxes (rows past the tile are loaded and
-      // never read).  Pair form: each CTA loads its half of the routed rows
-      // into its own slot; both halves are counted on the leader's ready
-      // barrier.
+      // (one commit per stage serves both rings).  A stage is the rows the
+      // tile's MMAs read (its routed rows rounded up to the MMA's N, a
+      // multiple of 16; rows past the tile are loaded and never used), in
+      // one box of exactly that height.  Pair form: each CTA loads its half
+      // of them into its own slot; both halves are counted on the leader's
+      // ready barrier.
       int bs = 0, S = 0;
       bool ok = true;
       for (int t = t0; t < total && ok; t += tstep) {
         const TileInfo ti = tile_info(sm, E, n_tiles, t);
-        const int rows_b = mma_n(ti.nrows) / PAIR;
-        const int boxes = (rows_b + B_BOX_ROWS - 1) / B_BOX_ROWS;
+        const int rows_b = mma_n(ti.nrows) / PAIR;  // 16 .. 256, a multiple of 16
+        const CUtensorMap* bm = &bmaps.m[rows_b / 16 - 1];
         const int brow0 = ti.row0 + rank * rows_b;
         for (int ks = 0; ks < KT; ++ks, ++S) {
           if (S >= BSTAGES) {
@@ -610,9 +616,7 @@ __global__ void __launch_bounds__(THREADS, 1) nf4_tc_kernel(
           uint64_t* rdy = &sm.ready[S % RING];
           // leader: its own barrier; the pair's peer: the leader's
           const uint32_t bar = leader ? smem_u32(rdy) : cluster_addr(rdy, 0);
-          if (leader) mbar_arrive_expect_tx(rdy, PAIR * boxes * B_BOX_BYTES);
-          // one copy per stage: a 128-row box, or a 256-row box (bmap2)
-          const CUtensorMap* bm = boxes == 2 ? &bmap2 : &bmap;
+          if (leader) mbar_arrive_expect_tx(rdy, PAIR * rows_b * BK * 2);
           if (PAIR == 1)
             tma_load_2d(sm.b[bs], bm, rdy, ks * BK, brow0);
           else
@@ -1044,14 +1048,15 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
                    int32_t* dev_err, cudaStream_t s, bool chain) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
-  CUtensorMap map, map2, wmap;
+  BMaps bmaps;
+  CUtensorMap wmap;
   const cuuint32_t estr[3] = {1, 1, 1};
-  for (int rows : {B_BOX_ROWS, 2 * B_BOX_ROWS}) {
-    // routed activation rows: boxes of 64 k x 128 or 256 rows
+  for (int i = 0; i < B_MAPS; ++i) {
+    // routed activation rows: boxes of 64 k x 16 (i + 1) rows
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M_total};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {BK, (cuuint32_t)rows};
-    if (enc(rows == B_BOX_ROWS ? &map : &map2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+    const cuuint32_t box[2] = {BK, (cuuint32_t)(16 * (i + 1))};
+    if (enc(&bmaps.m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
             const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -1088,7 +1093,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
   const int64_t max_tiles = ((int64_t)M_total / BN + E) * (N / (BM * PAIR));
   if (PAIR == 1) {
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, map2, wmap, wmap, scales,
+    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, bmaps, wmap, wmap, scales,
                       offsets, E, N, K, M_total, reinterpret_cast<OutT*>(out),
                       static_cast<const float*>(nullptr), dev_err, chain ? 1 : 0);
   }
@@ -1109,7 +1114,7 @@ cudaError_t launch(const void* A, const uint8_t* packed, const void* scales,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map, map2, wmap, wmap, scales, offsets, E, N, K, M_total,
+  return cudaLaunchKernelEx(&cfg, kern, bmaps, wmap, wmap, scales, offsets, E, N, K, M_total,
                             reinterpret_cast<OutT*>(out), static_cast<const float*>(nullptr),
                             dev_err, chain ? 1 : 0);
 }
@@ -1123,13 +1128,14 @@ cudaError_t launch_t(const void* G, int G_rows, const uint8_t* packed, const flo
                      const float* gu, int32_t* dev_err, cudaStream_t s) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   const auto enc = encode_tiled_cached;
-  CUtensorMap map, map2, wmap, amap;
+  BMaps bmaps;
+  CUtensorMap wmap, amap;
   const cuuint32_t estr[2] = {1, 1};
-  for (int rows : {B_BOX_ROWS, 2 * B_BOX_ROWS}) {
+  for (int i = 0; i < B_MAPS; ++i) {
     const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G_rows};
     const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
-    const cuuint32_t box[2] = {BK, (cuuint32_t)rows};
-    if (enc(rows == B_BOX_ROWS ? &map : &map2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+    const cuuint32_t box[2] = {BK, (cuuint32_t)(16 * (i + 1))};
+    if (enc(&bmaps.m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
             const_cast<void*>(G), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -1163,7 +1169,7 @@ cudaError_t launch_t(const void* G, int G_rows, const uint8_t* packed, const flo
   if (err != cudaSuccess) return err;
   const int64_t max_tiles = ((int64_t)M_total / BN + E) * (K / BM);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
-  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, map, map2, wmap, amap,
+  return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, s, bmaps, wmap, amap,
                     static_cast<const void*>(absmax), offsets, E, N, K, M_total,
                     reinterpret_cast<OutT*>(out), gu, dev_err, 0);
 }
