@@ -484,25 +484,14 @@ moe_status_t moe_layer_forward(const void* X, const float* logits, int T, int E,
   void* hbuf = ws + off[6];
   void* yp = ws + off[7];
   const int M = T * k;
+  moe_status_t st = moe_route_permute(logits, T, E, k, renormalize, topk_idx, topk_w, offsets,
+                                      sorted_rows, inv_perm, rws, off[6] - off[5], stream);
+  if (st) return st;
   // Routed activation rows in expert order, fp16: both grouped kernels read
   // them without a gather or a conversion in their inner loops.
   void* xp = ws + off[8];
-  moe_status_t st;
-  if (moe_launch::route_rows_fusable(T, E, k, H) && X && aligned16(X) && logits &&
-      aligned16(logits)) {
-    // a few routed rows: the routing kernel writes them too (one launch less)
-    if ((st = check_device())) return st;
-    st = from_cuda(moe_launch::route_permute_rows(logits, T, E, k, renormalize ? 1 : 0, topk_idx,
-                                                  topk_w, offsets, sorted_rows, inv_perm, X, H,
-                                                  xp, dev_err, (cudaStream_t)stream));
-    if (st) return st;
-  } else {
-    st = moe_route_permute(logits, T, E, k, renormalize, topk_idx, topk_w, offsets, sorted_rows,
-                           inv_perm, rws, off[6] - off[5], stream);
-    if (st) return st;
-    st = moe_permute_rows(X, MOE_DT_BF16, T, H, sorted_rows, k, M, xp, dev_err, stream);
-    if (st) return st;
-  }
+  st = moe_permute_rows(X, MOE_DT_BF16, T, H, sorted_rows, k, M, xp, dev_err, stream);
+  if (st) return st;
   // The GEMMs run in chain mode: the offsets come from the routing two and
   // three kernels back, so each GEMM starts streaming its weights while the
   // kernel before it finishes.

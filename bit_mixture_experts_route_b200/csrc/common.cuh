@@ -308,16 +308,6 @@ bool route_noalloc_fits(int T, int E, int k);
 cudaError_t route_permute_noalloc(const float* logits, int T, int E, int k, int renorm,
                                   int32_t* topk_idx, float* topk_w, int32_t* offsets,
                                   int32_t* sorted_rows, int32_t* inv_perm, cudaStream_t s);
-// Routing and the permuted fp16 rows in one launch when the rows are few
-// (T*k*H <= kRouteRowsMaxElems, H % 8 == 0, the single-CTA routing sizes).
-// Past 32 KB of rows the routing CTA's copy costs more than the separate
-// permute launch it saves (measured on B200: -8 % per layer at 128 KB).
-constexpr int64_t kRouteRowsMaxElems = 16384;
-bool route_rows_fusable(int T, int E, int k, int H);
-cudaError_t route_permute_rows(const float* logits, int T, int E, int k, int renorm,
-                               int32_t* topk_idx, float* topk_w, int32_t* offsets,
-                               int32_t* sorted_rows, int32_t* inv_perm, const void* X, int H,
-                               void* Xp, int32_t* dev_err, cudaStream_t s);
 cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
                           int32_t* topk_idx, float* topk_w, int32_t* offsets,
                           int32_t* sorted_rows, int32_t* inv_perm, void* ws,

@@ -160,9 +160,7 @@ __global__ void __launch_bounds__(kThreads) route_tile_kernel(
 // CTA of 32 warps routes every token (warp per token), ranks the routed rows
 // stably (each warp walks a contiguous chunk of flat ids with
 // __match_any_sync, keeping per-warp expert counts), scans the counts into
-// expert offsets and scatters.  With X given (a few routed rows: the layer's
-// call), it also writes the routed rows of X in expert order as fp16, which
-// is what permute_rows_kernel does, with the same conversion and range flag.
+// expert offsets and scatters.
 constexpr int kSmallRows = 4096;
 constexpr int kSmallE = 256;
 constexpr int kSmallThreads = 1024;
@@ -172,19 +170,16 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
-    int32_t* __restrict__ inv_perm, const __nv_bfloat16* __restrict__ X, int H,
-    __half* __restrict__ Xp, int32_t* dev_err) {
+    int32_t* __restrict__ inv_perm) {
   pdl_wait();
   pdl_trigger();
   // 16-bit fields: rows, ranks and counts are all < kSmallRows = 4096
   __shared__ int16_t s_eid[kSmallRows];
-  __shared__ int16_t s_sorted[kSmallRows];  // position -> flat id (row copy)
   __shared__ uint16_t s_rank[kSmallRows];
   __shared__ uint16_t s_wc[32][kSmallE];   // per-warp expert counts, then prefixes
   __shared__ int s_off[kSmallE + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 32 * kSmallE; i += kSmallThreads) (&s_wc[0][0])[i] = 0;
-  for (int i = threadIdx.x; i < T * k; i += kSmallThreads) s_sorted[i] = -1;
   // (made visible by the __syncthreads after the routing loop)
 
   for (int t = warp; t < T; t += 32) {
@@ -266,39 +261,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     if (pos < 0 || pos >= n) continue;
     sorted_rows[pos] = f;
     inv_perm[f] = pos;
-    s_sorted[pos] = (int16_t)f;
   }
-  if (X == nullptr) return;
-  __syncthreads();
-  // routed row p = token s_sorted[p] / k, bf16 -> fp16 in 16-byte chunks of
-  // 8 elements (H % 8 == 0, rows 16-byte aligned: checked by the host), spread
-  // over all threads, four loads in flight per thread before its stores
-  bool ovf = false;
-  const int cpr = H / 8;  // chunks per row
-  const int nch = n * cpr;
-  for (int c0 = threadIdx.x; c0 < nch; c0 += 4 * kSmallThreads) {
-    uint4 u[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + j * kSmallThreads;
-      if (c < nch) {
-        const int p = c / cpr;
-        const int f = s_sorted[p];  // every position is written; a stray value reads row 0
-        const int tok = (f >= 0 && f < n) ? f / k : 0;
-        u[j] = *reinterpret_cast<const uint4*>(X + (size_t)tok * H + (size_t)(c - p * cpr) * 8);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + j * kSmallThreads;
-      if (c >= nch) break;
-      const uint4 o = make_uint4(bf16x2_to_f16x2(u[j].x), bf16x2_to_f16x2(u[j].y),
-                                 bf16x2_to_f16x2(u[j].z), bf16x2_to_f16x2(u[j].w));
-      ovf |= any_f16x8_nonfinite(o);
-      *reinterpret_cast<uint4*>(Xp + (size_t)c * 8) = o;
-    }
-  }
-  if (__any_sync(0xffffffffu, ovf) && lane == 0) set_dev_err(dev_err, MOE_DEVERR_RANGE);
 }
 
 // Exclusive scan of s[0..n) in place for n <= 1024 with kThreads threads.
@@ -406,9 +369,7 @@ cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
   if ((int64_t)T * k <= moe::kSmallRows && E <= moe::kSmallE) {
 #define MOE_ROUTE_SMALL(NP)                                                             \
   moe::launch_pdl(moe::route_small_kernel<NP>, dim3(1), dim3(moe::kSmallThreads), 0, s, logits, \
-                  T, E, k, renorm, topk_idx, topk_w, offsets, sorted_rows, inv_perm,          \
-                  static_cast<const __nv_bfloat16*>(nullptr), 0, static_cast<__half*>(nullptr),  \
-                  static_cast<int32_t*>(nullptr))
+                  T, E, k, renorm, topk_idx, topk_w, offsets, sorted_rows, inv_perm)
     if (E <= 32) return MOE_ROUTE_SMALL(1);
     if (E <= 64) return MOE_ROUTE_SMALL(2);
     if (E <= 128) return MOE_ROUTE_SMALL(4);
@@ -434,30 +395,6 @@ cudaError_t route_permute(const float* logits, int T, int E, int k, int renorm,
   return moe::launch_pdl(moe::permute_scatter_kernel, dim3(ntiles), dim3(moe::kThreads), 0, s,
                          topk_idx, rank, tile_counts, T, E, k, ntiles, offsets, sorted_rows,
                          inv_perm);
-}
-
-bool route_rows_fusable(int T, int E, int k, int H) {
-  const int64_t n = (int64_t)T * k;
-  return T > 0 && n <= moe::kSmallRows && E <= moe::kSmallE && H % 8 == 0 &&
-         n * H <= kRouteRowsMaxElems;
-}
-
-// Routing plus the routed rows of bf16 X in expert order as fp16, in one
-// launch (route_rows_fusable: a few rows, copied by the routing CTA).
-cudaError_t route_permute_rows(const float* logits, int T, int E, int k, int renorm,
-                               int32_t* topk_idx, float* topk_w, int32_t* offsets,
-                               int32_t* sorted_rows, int32_t* inv_perm, const void* X, int H,
-                               void* Xp, int32_t* dev_err, cudaStream_t s) {
-  if (!route_rows_fusable(T, E, k, H)) return cudaErrorNotSupported;
-#define MOE_ROUTE_ROWS(NP)                                                              \
-  moe::launch_pdl(moe::route_small_kernel<NP>, dim3(1), dim3(moe::kSmallThreads), 0, s, logits, \
-                  T, E, k, renorm, topk_idx, topk_w, offsets, sorted_rows, inv_perm,          \
-                  static_cast<const __nv_bfloat16*>(X), H, static_cast<__half*>(Xp), dev_err)
-  if (E <= 32) return MOE_ROUTE_ROWS(1);
-  if (E <= 64) return MOE_ROUTE_ROWS(2);
-  if (E <= 128) return MOE_ROUTE_ROWS(4);
-  return MOE_ROUTE_ROWS(8);
-#undef MOE_ROUTE_ROWS
 }
 
 // ---------------------------------------------------------------------------

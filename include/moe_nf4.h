@@ -537,12 +537,14 @@ moe_status_t moe_unpermute_combine(const void* Yp, moe_dtype_t yp_dtype,
 
 /*
  * Whole layer in one call (route -> permute -> gate_up+SwiGLU -> down ->
- * combine), each step the entry point above, all on `stream`.
+ * combine), each step the entry point above, all on `stream`.  The two
+ * grouped GEMMs run chained (each requests its first weights while the
+ * kernel before it finishes).
  *   X bf16 [T, H]; logits fp32 [T, E]; gate_up stack [E, 2I, H];
  *   down stack [E, H, I]; Y fp32 [T, H].
  *   workspace: moe_layer_workspace_size bytes; it holds the routing outputs
- *   and the fp16 intermediates [T*k, H] (permuted X, tensor-core path
- *   only), [T*k, I] and [T*k, H].
+ *   and the fp16 intermediates [T*k, H] (permuted X), [T*k, I] and
+ *   [T*k, H].
  */
 moe_status_t moe_layer_workspace_size(int T, int E, int k, int H, int I,
                                       size_t* bytes);
