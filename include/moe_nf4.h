@@ -497,8 +497,9 @@ moe_status_t moe_nf4_grouped_gemm(const void* A, moe_dtype_t a_dtype,
  * order, converted to fp16: Xp[p, :] = fp16(X[sorted_rows[p] / k, :]) for
  * p < M_total.  This is the activation side of the permutation (the
  * permuted rows one grouped launch reads as contiguous per-expert
- * segments, "grouped-nf4-gemm & experts-4bit", first bullet); the tensor-core
- * grouped GEMM reads its activations this way, through TMA.
+ * segments, "grouped-nf4-gemm & experts-4bit", first bullet); the decode
+ * and tensor-core grouped GEMMs read their activations this way, through
+ * TMA.
  *   X   [T, K] BF16 or F16; sorted_rows int32 [M_total]; Xp fp16 [M_total, K]
  *   K % 8 == 0; ids with f < 0, f >= M_total or f / k >= T give zero rows
  *   and MOE_DEVERR_BAD_INDEX.  Pointers 16-byte aligned.
